@@ -110,11 +110,14 @@ def norm_gate(y, g=None, gamma=None, eps: float = 1e-6, act: str | int = "silu")
 
 
 def run_unit(kp, qp, v, alpha, beta, M_init, b: int, h: int, *, S1: int, W: int, R: int,
-             rows=None, want_y=None, t_end=None, select_mode: str = "product_key"):
+             rows=None, want_y=None, t_end=None, select_mode: str = "product_key",
+             threads: int = 1, selection=None):
     """Steps 1-3 for one (sequence b, head h) over tokens [0, t_end).
 
     rows: tracked slot rows (int array) or None for all N rows.
     want_y: bool array [t_end] of tokens whose read result is wanted, or None (all).
+    threads: token chunks of the selection (independent per token) run on this many
+    threads.  selection: a previous result's (idx_w, wt_w, idx_r, wt_r) to reuse.
     Returns dict(idx_w, wt_w, idx_r, wt_r, y [t_end, d_v] float64 (NaN where unwanted),
     M [n_rows, d_v] float32, rows).
     """
@@ -128,16 +131,30 @@ def run_unit(kp, qp, v, alpha, beta, M_init, b: int, h: int, *, S1: int, W: int,
     def sel(x, K):
         idx = np.empty((t_end, K), np.int32)
         wt = np.empty((t_end, K), np.float64)
-        base = x[b, :t_end, h, :]  # strided view: row t at stride H*S
-        xs = np.ascontiguousarray(base)
-        rc = lib.sdm_oracle_select(_ptr(xs), t_end, S, S1, S2, K, _MODE[select_mode],
-                                   _ptr(idx), _ptr(wt), None)
-        if rc != 0:
-            raise ValueError(f"sdm_oracle_select failed ({rc})")
+        xs = np.ascontiguousarray(x[b, :t_end, h, :], dtype=np.float32)
+
+        def chunk(rng):
+            t0, t1 = rng
+            rc = lib.sdm_oracle_select(xs[t0:].ctypes.data, t1 - t0, S, S1, S2, K,
+                                       _MODE[select_mode], idx[t0:].ctypes.data,
+                                       wt[t0:].ctypes.data, None)
+            if rc != 0:
+                raise ValueError(f"sdm_oracle_select failed ({rc})")
+
+        n = max(1, min(threads, t_end))
+        bounds = [(t_end * i // n, t_end * (i + 1) // n) for i in range(n)]
+        if n > 1:
+            with ThreadPoolExecutor(n) as ex:
+                list(ex.map(chunk, bounds))
+        else:
+            chunk(bounds[0])
         return idx, wt
 
-    idx_w, wt_w = sel(kp, W)
-    idx_r, wt_r = sel(qp, R)
+    if selection is None:
+        idx_w, wt_w = sel(kp, W)
+        idx_r, wt_r = sel(qp, R)
+    else:
+        idx_w, wt_w, idx_r, wt_r = selection
 
     v_u = np.ascontiguousarray(v[b, :t_end, h, :], dtype=np.float32)
     a_u = np.ascontiguousarray(alpha[b, :t_end, h], dtype=np.float32)

@@ -46,16 +46,28 @@ typedef struct {
     int64_t i; /* index (per-half index, or flat slot index) */
 } scored_t;
 
-/* (score descending, index ascending).  C compares -0.0f == +0.0f as equal, so the
- * two zeros fall through to the index tie-break, as the reading requires. */
-static int cmp_scored(const void *pa, const void *pb) {
-    const scored_t *a = (const scored_t *)pa;
-    const scored_t *b = (const scored_t *)pb;
-    if (a->s > b->s) return -1;
-    if (a->s < b->s) return 1;
-    if (a->i < b->i) return -1;
-    if (a->i > b->i) return 1;
-    return 0;
+/* Does a come before b in (score descending, index ascending) order?  C compares
+ * -0.0f == +0.0f as equal, so the two zeros fall through to the index tie-break. */
+static int before(const scored_t *a, const scored_t *b) {
+    if (a->s != b->s) return a->s > b->s;
+    return a->i < b->i;
+}
+
+/* Keeps best[0 .. *n) as the first (at most K) items seen so far, in order: the new item
+ * is inserted at its place and the item pushed past position K falls off. */
+static void keep_top(scored_t *best, int *n, int K, scored_t c) {
+    int pos = *n;
+    if (pos == K) {
+        if (!before(&c, &best[K - 1])) return;
+        pos = K - 1;
+    } else {
+        (*n)++;
+    }
+    while (pos > 0 && before(&c, &best[pos - 1])) {
+        best[pos] = best[pos - 1];
+        --pos;
+    }
+    best[pos] = c;
 }
 
 /* Softmax of the selected scores over the selected set [P1 step 2: k_t^(i) is the
@@ -94,47 +106,53 @@ int sdm_oracle_select(const float *halves, long n, long row_stride, int S1, int 
     const int K2 = K < S2 ? K : S2;
     if ((long)K1 * (long)K2 < (long)K) return ORACLE_ERR_ARG;
 
-    long cap = mode == 0 ? (long)K1 * K2 : N;
-    scored_t *h1 = (scored_t *)malloc(sizeof(scored_t) * (size_t)S1);
-    scored_t *h2 = (scored_t *)malloc(sizeof(scored_t) * (size_t)S2);
-    scored_t *cand = (scored_t *)malloc(sizeof(scored_t) * (size_t)cap);
-    if (!h1 || !h2 || !cand) {
-        free(h1); free(h2); free(cand);
+    scored_t *h1 = (scored_t *)malloc(sizeof(scored_t) * (size_t)K1);
+    scored_t *h2 = (scored_t *)malloc(sizeof(scored_t) * (size_t)K2);
+    scored_t *top = (scored_t *)malloc(sizeof(scored_t) * (size_t)K);
+    if (!h1 || !h2 || !top) {
+        free(h1); free(h2); free(top);
         return ORACLE_ERR_NOMEM;
     }
     for (long r = 0; r < n; ++r) {
         const float *k1 = halves + r * row_stride; /* first half, length S1 */
         const float *k2 = k1 + S1;                 /* second half, length S2 */
         long nc = 0;
+        int ntop = 0;
         if (mode == 0) {
-            for (int a = 0; a < S1; ++a) { h1[a].s = k1[a]; h1[a].i = a; }
-            for (int b = 0; b < S2; ++b) { h2[b].s = k2[b]; h2[b].i = b; }
-            qsort(h1, (size_t)S1, sizeof(scored_t), cmp_scored);
-            qsort(h2, (size_t)S2, sizeof(scored_t), cmp_scored);
+            int n1 = 0, n2 = 0;
+            for (int a = 0; a < S1; ++a) {
+                scored_t c = {k1[a], a};
+                keep_top(h1, &n1, K1, c);
+            }
+            for (int b = 0; b < S2; ++b) {
+                scored_t c = {k2[b], b};
+                keep_top(h2, &n2, K2, c);
+            }
             for (int a = 0; a < K1; ++a) {
                 for (int b = 0; b < K2; ++b) {
-                    float s = h1[a].s + h2[b].s; /* one fp32 addition */
-                    cand[nc].s = s;
-                    cand[nc].i = h1[a].i * (int64_t)S2 + h2[b].i;
+                    scored_t c;
+                    c.s = h1[a].s + h2[b].s; /* one fp32 addition */
+                    c.i = h1[a].i * (int64_t)S2 + h2[b].i;
+                    keep_top(top, &ntop, K, c);
                     ++nc;
                 }
             }
         } else {
             for (int a = 0; a < S1; ++a) {
                 for (int b = 0; b < S2; ++b) {
-                    float s = k1[a] + k2[b];
-                    cand[nc].s = s;
-                    cand[nc].i = (int64_t)a * S2 + b;
+                    scored_t c;
+                    c.s = k1[a] + k2[b];
+                    c.i = (int64_t)a * S2 + b;
+                    keep_top(top, &ntop, K, c);
                     ++nc;
                 }
             }
         }
-        qsort(cand, (size_t)nc, sizeof(scored_t), cmp_scored);
-        for (int j = 0; j < K; ++j) idx[r * K + j] = (int32_t)cand[j].i;
-        softmax_selected(cand, K, wt + r * K);
+        for (int j = 0; j < K; ++j) idx[r * K + j] = (int32_t)top[j].i;
+        softmax_selected(top, K, wt + r * K);
         if (n_scored) *n_scored = nc;
     }
-    free(h1); free(h2); free(cand);
+    free(h1); free(h2); free(top);
     return ORACLE_OK;
 }
 

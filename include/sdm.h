@@ -1,0 +1,159 @@
+/*
+ * sdm.h -- C ABI of the B200 (sm_100a) Sparse Delta Memory memory pass.
+ *
+ * The pass follows the four-step method of "Sparse Delta Memory: Scaling the State of
+ * Linear RNNs through Sparsity" (paper.rainbus.top summary, method paragraph), for one
+ * SDM layer whose inputs are already projected:
+ *   step 1  product-key top-k slot selection (write keys and read queries),
+ *   step 2  gated delta write on the selected write slots only,
+ *   step 3  sparse read of the selected read slots, after the token's write,
+ *   step 4  RMS normalisation and elementwise output gating (the head-mixing
+ *           projection W_o is not part of this library).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer is a DEVICE pointer owned by the caller, 16-byte aligned, to a
+ *    contiguous row-major array.  The library allocates no memory; scratch space comes
+ *    from the caller through `ws` (size from sdm_workspace_size).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *    Calls are asynchronous on that stream; calls on different streams may run
+ *    concurrently as long as they touch disjoint outputs.
+ *  - Arguments are validated on the host before anything is launched.  A rejected call
+ *    returns SDM_ERR_INVALID_ARG (or SDM_ERR_UNSUPPORTED) and has no effect.  A failed
+ *    launch returns SDM_ERR_CUDA.  Conditions detected on the device are recorded in a
+ *    per-device status word that sdm_get_device_status() reads and clears.
+ *  - Shapes: N = S1*S2 memory slots per head; the flat slot index of the pair
+ *    (i1 in the first half, i2 in the second) is i1*S2 + i2.
+ *  - Selection order, at every stage: score descending, then slot index ascending;
+ *    -0 and +0 are the same score.  Scores are sums of two fp32 half scores (bf16
+ *    halves are widened exactly), added once in fp32 round-to-nearest.  NaN scores
+ *    are outside the supported domain.
+ *  - Slot weights: softmax (temperature 1) of the selected scores over the selected set
+ *    ("sparse key value" k^(i) of the write, q^(i) of the read).
+ *  - Limits: 1 <= S1, S2 <= 4096; 1 <= W, R <= min(S1, S2, 128); d_v a multiple of 4
+ *    (fp32 inputs) or of 8 (bf16 inputs), 8 <= d_v <= 1024 for bf16, 4 <= d_v <= 1024 for
+ *    fp32.  N <= 2^31 - 1.
+ */
+#ifndef SDM_H
+#define SDM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SDM_OK = 0,
+    SDM_ERR_INVALID_ARG = 1,  /* a pointer, size, alignment or enum is not accepted     */
+    SDM_ERR_UNSUPPORTED = 2,  /* valid request that this build does not implement      */
+    SDM_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed            */
+    SDM_ERR_DEVICE_CHECK = 4, /* a kernel found an out-of-range index in its inputs     */
+    SDM_ERR_TIMEOUT = 5       /* a bounded wait inside a kernel ran out                 */
+} sdm_status;
+
+typedef enum { SDM_F32 = 0, SDM_BF16 = 1 } sdm_dtype;
+typedef enum { SDM_ENGINE_AUTO = 0, SDM_ENGINE_SEQ = 1, SDM_ENGINE_SLOT = 2 } sdm_engine;
+typedef enum { SDM_INIT_FROM_M0 = 0, SDM_CONTINUE = 1 } sdm_init;
+typedef enum { SDM_GATE_SILU = 0, SDM_GATE_SIGMOID = 1, SDM_GATE_IDENTITY = 2 } sdm_gate_act;
+
+/* Problem shape.  B sequences, T tokens, H heads, S1 + S2 half scores per (token, head),
+ * W write slots and R read slots per token, d_v value width.  in_dtype (an sdm_dtype)
+ * is the element type of the score halves, v and the gate; alpha, beta, M0, M, y and o
+ * are always fp32. */
+typedef struct {
+    int32_t B, T, H, S1, S2, W, R, d_v;
+    int32_t in_dtype;
+} sdm_shape;
+
+/*
+ * Step 1 alone: product-key top-K selection [paper.rainbus.top summary, method step 1;
+ * ai-paper-analysis.pages.dev SDM write-up, 步骤 1].  For each of the B*T*H rows of
+ * `halves` ([B,T,H,S1+S2], first half then second half, in_dtype) the K slots with the
+ * largest outer-sum scores, in selection order, and their softmax weights.
+ *   idx [B,T,H,K] int32 flat slot indices; wt [B,T,H,K] fp32 weights.
+ * Uses shape.B, T, H, S1, S2, in_dtype; K replaces W/R (1 <= K <= min(S1, S2, 128)).
+ */
+sdm_status sdm_select(const void *halves, sdm_shape shape, int32_t K, int32_t *idx, float *wt,
+                      void *stream);
+
+/* Bytes of scratch that sdm_scan_forward needs for this shape and engine (the
+ * selections of every token: B*T*H*(W+R) indices and weights, plus engine buffers).
+ * Returns 0 for an invalid shape. */
+size_t sdm_workspace_size(sdm_shape shape, int32_t engine);
+
+/*
+ * Learnable initial memory [ai-paper-analysis.pages.dev SDM write-up, section on the
+ * learned initial state M0; m.163.com article, section 三]: M0 [H,N,d_v] is shared by
+ * every sequence, so M[b,h,:,:] = M0[h,:,:] for every b.  M [B,H,N,d_v]; M must not
+ * overlap M0.
+ */
+sdm_status sdm_state_init(const float *M0, float *M, sdm_shape shape, void *stream);
+
+/*
+ * Prefill: steps 1-4 over T tokens for every (b, h) [paper.rainbus.top summary, method
+ * steps 1-4].  Token t of sequence b, head h:
+ *   I_w, k = top-W selection of kp[b,t,h,:];  I_r, q = top-R selection of qp[b,t,h,:]
+ *   for i in I_w:  M~ = alpha[b,t,h] * M[b,h,i,:]
+ *                  M[b,h,i,:] = M~ + beta[b,t,h] * k_i * (v[b,t,h,:] - M~)
+ *   y[b,t,h,:] = sum_{i in I_r} q_i * M[b,h,i,:]        (after token t's write)
+ *   o[b,t,h,:] = y * rsqrt(mean(y^2) + eps) * gamma * act(gate[b,t,h,:])
+ * Arguments:
+ *   kp, qp   [B,T,H,S1+S2] in_dtype     v, gate [B,T,H,d_v] in_dtype (gate nullable:
+ *                                        no gating factor)
+ *   alpha, beta [B,T,H] fp32             M0 [H,N,d_v] fp32 (read only with
+ *                                        init == SDM_INIT_FROM_M0, may then be NULL
+ *                                        otherwise)
+ *   M        [B,H,N,d_v] fp32, in/out: the recurrent state.  init == SDM_INIT_FROM_M0
+ *            first sets it to M0; SDM_CONTINUE resumes from its current contents.
+ *   y        [B,T,H,d_v] fp32 out.       o [B,T,H,d_v] fp32 out, nullable (no step 4)
+ *   gamma    [d_v] fp32, nullable (unit weight).   eps >= 0.   act: sdm_gate_act.
+ *   sel_out  nullable int32 out: the selected write slots [B,T,H,W] followed by the
+ *            read slots [B,T,H,R], in selection order (for parity checks).
+ *   engine   sdm_engine; ws / ws_bytes caller scratch of at least
+ *            sdm_workspace_size(shape, engine) bytes, 256-byte aligned.
+ * T == 0 is valid: only the initialisation (if requested) happens.
+ */
+sdm_status sdm_scan_forward(const void *kp, const void *qp, const void *v, const float *alpha,
+                            const float *beta, const float *M0, float *M, int32_t init,
+                            float *y, const void *gate, const float *gamma, float eps,
+                            int32_t act, float *o, int32_t *sel_out, int32_t engine, void *ws,
+                            size_t ws_bytes, sdm_shape shape, void *stream);
+
+/*
+ * Decode: steps 1-4 for ONE token of each of B sequences and H heads, in one fused
+ * launch [paper.rainbus.top summary, method steps 1-4; m.163.com article, section 八,
+ * on decode].  Same arithmetic as sdm_scan_forward with T = 1 and SDM_CONTINUE:
+ *   kp, qp [B,H,S1+S2] in_dtype; v, gate [B,H,d_v] in_dtype (gate nullable);
+ *   alpha, beta [B,H] fp32; M [B,H,N,d_v] fp32 in/out; y [B,H,d_v] fp32 out;
+ *   o [B,H,d_v] fp32 out, nullable; gamma [d_v] nullable;
+ *   sel_out nullable: write slots [B,H,W] followed by read slots [B,H,R].
+ * shape.T is ignored.  No scratch memory is used.
+ */
+sdm_status sdm_decode_step(const void *kp, const void *qp, const void *v, const float *alpha,
+                           const float *beta, float *M, float *y, const void *gate,
+                           const float *gamma, float eps, int32_t act, float *o,
+                           int32_t *sel_out, sdm_shape shape, void *stream);
+
+/*
+ * Step 4 alone [paper.rainbus.top summary, method step 4]: for each of the B*T*H rows
+ * of y [B,T,H,d_v] (fp32), o = y * rsqrt(mean(y^2) + eps) * gamma * act(gate).
+ * gate [B,T,H,d_v] in_dtype, nullable; gamma [d_v] fp32, nullable.  o may equal y.
+ */
+sdm_status sdm_norm_gate(const float *y, const void *gate, const float *gamma, float eps,
+                         int32_t act, sdm_shape shape, float *o, void *stream);
+
+/* Synchronises `stream`, then reads and clears the calling device's status word:
+ * SDM_OK, SDM_ERR_DEVICE_CHECK (an index outside [0, N) reached a kernel) or
+ * SDM_ERR_TIMEOUT (a bounded wait expired).  SDM_ERR_CUDA if the synchronisation fails. */
+sdm_status sdm_get_device_status(void *stream);
+
+/* Static, human-readable name of a status code. */
+const char *sdm_status_string(sdm_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDM_H */

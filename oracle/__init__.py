@@ -72,11 +72,13 @@ def _ptr(a):
     return None if a is None else a.ctypes.data
 
 
-def select(halves, S1: int, K: int, mode: str = "product_key", return_scored: bool = False):
+def select(halves, S1: int, K: int, mode: str = "product_key", return_scored: bool = False,
+           threads: int = 1):
     """Top-K slot selection of every row of ``halves`` [..., S1+S2] (float32).
 
     Returns (idx int32 [..., K], wt float64 [..., K]) in selection order, and the
-    number of candidate sums scored per row when ``return_scored``.
+    number of candidate sums scored per row when ``return_scored``.  Rows are
+    independent; ``threads`` splits them into that many chunks.
     """
     h = np.ascontiguousarray(halves, dtype=np.float32)
     S = h.shape[-1]
@@ -86,10 +88,23 @@ def select(halves, S1: int, K: int, mode: str = "product_key", return_scored: bo
     idx = np.empty((n, K), np.int32)
     wt = np.empty((n, K), np.float64)
     scored = ctypes.c_long(0)
-    rc = _load().sdm_oracle_select(_ptr(rows), n, S, S1, S2, K, _MODE[mode], _ptr(idx),
-                                   _ptr(wt), ctypes.byref(scored))
-    if rc != 0:
-        raise ValueError(f"sdm_oracle_select failed ({rc})")
+    lib = _load()
+
+    def chunk(rng):
+        r0, r1 = rng
+        rc = lib.sdm_oracle_select(rows[r0:].ctypes.data, r1 - r0, S, S1, S2, K, _MODE[mode],
+                                   idx[r0:].ctypes.data, wt[r0:].ctypes.data,
+                                   ctypes.byref(scored))
+        if rc != 0:
+            raise ValueError(f"sdm_oracle_select failed ({rc})")
+
+    nt = max(1, min(int(threads), n))
+    bounds = [(n * i // nt, n * (i + 1) // nt) for i in range(nt)]
+    if nt > 1:
+        with ThreadPoolExecutor(nt) as ex:
+            list(ex.map(chunk, bounds))
+    elif n:
+        chunk(bounds[0])
     out = (idx.reshape(h.shape[:-1] + (K,)), wt.reshape(h.shape[:-1] + (K,)))
     return out + (scored.value,) if return_scored else out
 

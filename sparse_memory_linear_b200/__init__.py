@@ -1,0 +1,27 @@
+"""B200-native Sparse Delta Memory (SDM) memory pass.
+
+Python binding of libsdm.so, whose C ABI is declared in include/sdm.h.  The binding only
+marshals arguments (shapes, data pointers and the current CUDA stream of torch tensors)
+and allocates outputs with torch; every step of the pass runs in the sm_100a kernels
+behind the ABI.  There is no fallback: if the library is missing the calls raise.
+"""
+
+from ._binding import (  # noqa: F401
+    ACT,
+    ENGINE,
+    SDM_BF16,
+    SDM_F32,
+    SdmError,
+    SdmShape,
+    library,
+    library_path,
+    sdm_decode_step,
+    sdm_get_device_status,
+    sdm_norm_gate,
+    sdm_scan_forward,
+    sdm_select,
+    sdm_state_init,
+    sdm_status_string,
+    sdm_workspace_size,
+    shape_of,
+)

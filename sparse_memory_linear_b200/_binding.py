@@ -1,0 +1,244 @@
+"""ctypes binding of libsdm.so (C ABI in include/sdm.h): argument marshalling only."""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+SDM_F32, SDM_BF16 = 0, 1
+ENGINE = {"auto": 0, "seq": 1, "slot": 2}
+INIT = {"m0": 0, "continue": 1}
+ACT = {"silu": 0, "sigmoid": 1, "identity": 2}
+_STATUS = {0: "SDM_OK", 1: "SDM_ERR_INVALID_ARG", 2: "SDM_ERR_UNSUPPORTED", 3: "SDM_ERR_CUDA",
+           4: "SDM_ERR_DEVICE_CHECK", 5: "SDM_ERR_TIMEOUT"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libsdm.so")
+
+
+class SdmShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "T", "H", "S1", "S2", "W", "R", "d_v",
+                                               "in_dtype")]
+
+    def __repr__(self):
+        return "SdmShape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+class SdmError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = int(status)
+        super().__init__(f"{what}: {_STATUS.get(self.status, self.status)}")
+
+
+_lib = None
+
+
+def library():
+    """The loaded libsdm.so.  Raises if it has not been built: there is no other path."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise RuntimeError(
+            f"{library_path} is missing; build it with "
+            "`python -c 'import __graft_entry__ as g; g.build()'` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(library_path)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    S = SdmShape
+    sig = {
+        "sdm_select": ([P, S, I, P, P, P], I),
+        "sdm_workspace_size": ([S, I], Z),
+        "sdm_state_init": ([P, P, S, P], I),
+        "sdm_scan_forward": ([P, P, P, P, P, P, P, I, P, P, P, F, I, P, P, I, P, Z, S, P], I),
+        "sdm_decode_step": ([P, P, P, P, P, P, P, P, P, F, I, P, P, S, P], I),
+        "sdm_norm_gate": ([P, P, P, F, I, S, P, P], I),
+        "sdm_get_device_status": ([P], I),
+        "sdm_status_string": ([I], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device=None):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise SdmError(rc, what)
+
+
+def _in_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SDM_BF16
+    if t.dtype == torch.float32:
+        return SDM_F32
+    raise TypeError(f"inputs must be bfloat16 or float32, got {t.dtype}")
+
+
+def _need(t, name, dtype=None, device=None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    return t
+
+
+def shape_of(B, T, H, S1, S2, W, R, d_v, in_dtype) -> SdmShape:
+    return SdmShape(int(B), int(T), int(H), int(S1), int(S2), int(W), int(R), int(d_v),
+                    int(in_dtype))
+
+
+def sdm_status_string(status: int) -> str:
+    return library().sdm_status_string(int(status)).decode()
+
+
+def sdm_workspace_size(shape: SdmShape, engine: str = "auto") -> int:
+    return int(library().sdm_workspace_size(shape, ENGINE[engine]))
+
+
+def sdm_select(halves: torch.Tensor, K: int, *, S1: int | None = None, idx=None, wt=None,
+               stream=None):
+    """Top-K product-key selection of every row of ``halves`` [..., S1+S2].
+    Returns (idx int32 [..., K], wt float32 [..., K])."""
+    _need(halves, "halves")
+    S = halves.shape[-1]
+    S1 = S // 2 if S1 is None else int(S1)
+    rows = halves.numel() // S if S else 0
+    lead = tuple(halves.shape[:-1])
+    idx = torch.empty(lead + (K,), dtype=torch.int32, device=halves.device) if idx is None else idx
+    wt = torch.empty(lead + (K,), dtype=torch.float32, device=halves.device) if wt is None else wt
+    _need(idx, "idx", torch.int32, halves.device)
+    _need(wt, "wt", torch.float32, halves.device)
+    shape = shape_of(rows, 1, 1, S1, S - S1, 1, 1, 8, _in_dtype(halves))
+    _check(library().sdm_select(_p(halves), shape, int(K), _p(idx), _p(wt),
+                                _stream(stream, halves.device)), "sdm_select")
+    return idx, wt
+
+
+def sdm_state_init(M0: torch.Tensor, M: torch.Tensor, *, d_v: int | None = None, stream=None):
+    """M[b, h] = M0[h] for every b.  M0 [H, N, d_v], M [B, H, N, d_v] float32."""
+    _need(M0, "M0", torch.float32)
+    _need(M, "M", torch.float32, M0.device)
+    B, H, N, dv = M.shape
+    shape = shape_of(B, 1, H, 1, N, 1, 1, dv, SDM_F32)
+    _check(library().sdm_state_init(_p(M0), _p(M), shape, _stream(stream, M.device)),
+           "sdm_state_init")
+    return M
+
+
+def sdm_scan_forward(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | None = None,
+                     M0=None, init: str = "m0", y=None, gate=None, gamma=None,
+                     eps: float = 1e-6, act: str = "silu", o=None, want_o: bool = True,
+                     sel_out=None, want_sel: bool = False, engine: str = "auto", ws=None,
+                     stream=None):
+    """Prefill over T tokens.  kp, qp [B,T,H,S1+S2]; v, gate [B,T,H,d_v]; alpha, beta
+    [B,T,H]; M [B,H,N,d_v] (in/out); M0 [H,N,d_v] (init="m0").
+    Returns dict(y, o, sel): sel holds [B,T,H,W] write slots then [B,T,H,R] read slots."""
+    dev = kp.device
+    _need(kp, "kp", device=dev)
+    dt = kp.dtype
+    _need(qp, "qp", dt, dev)
+    _need(v, "v", dt, dev)
+    _need(gate, "gate", dt, dev)
+    _need(alpha, "alpha", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(M, "M", torch.float32, dev)
+    _need(M0, "M0", torch.float32, dev)
+    _need(gamma, "gamma", torch.float32, dev)
+    B, T, H, S = kp.shape
+    S1 = S // 2 if S1 is None else int(S1)
+    d_v = v.shape[-1]
+    shape = shape_of(B, T, H, S1, S - S1, W, R, d_v, _in_dtype(kp))
+    if y is None:
+        y = torch.empty((B, T, H, d_v), dtype=torch.float32, device=dev)
+    if o is None and want_o:
+        o = torch.empty((B, T, H, d_v), dtype=torch.float32, device=dev)
+    if sel_out is None and want_sel:
+        sel_out = torch.empty(B * T * H * (W + R), dtype=torch.int32, device=dev)
+    _need(y, "y", torch.float32, dev)
+    _need(o, "o", torch.float32, dev)
+    _need(sel_out, "sel_out", torch.int32, dev)
+    need = sdm_workspace_size(shape, engine)
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _need(ws, "ws", torch.uint8, dev)
+    _check(library().sdm_scan_forward(
+        _p(kp), _p(qp), _p(v), _p(alpha), _p(beta), _p(M0), _p(M), INIT[init], _p(y), _p(gate),
+        _p(gamma), float(eps), ACT[act], _p(o), _p(sel_out), ENGINE[engine], _p(ws),
+        ws.numel(), shape, _stream(stream, dev)), "sdm_scan_forward")
+    return dict(y=y, o=o, sel=sel_out)
+
+
+def sdm_decode_step(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | None = None,
+                    y=None, gate=None, gamma=None, eps: float = 1e-6, act: str = "silu", o=None,
+                    want_o: bool = True, sel_out=None, want_sel: bool = False, stream=None):
+    """One token for each (b, h).  kp, qp [B,H,S1+S2]; v, gate [B,H,d_v]; alpha, beta [B,H];
+    M [B,H,N,d_v] in/out.  Returns dict(y, o, sel)."""
+    dev = kp.device
+    _need(kp, "kp", device=dev)
+    dt = kp.dtype
+    _need(qp, "qp", dt, dev)
+    _need(v, "v", dt, dev)
+    _need(gate, "gate", dt, dev)
+    _need(alpha, "alpha", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(M, "M", torch.float32, dev)
+    _need(gamma, "gamma", torch.float32, dev)
+    B, H, S = kp.shape
+    S1 = S // 2 if S1 is None else int(S1)
+    d_v = v.shape[-1]
+    shape = shape_of(B, 1, H, S1, S - S1, W, R, d_v, _in_dtype(kp))
+    if y is None:
+        y = torch.empty((B, H, d_v), dtype=torch.float32, device=dev)
+    if o is None and want_o:
+        o = torch.empty((B, H, d_v), dtype=torch.float32, device=dev)
+    if sel_out is None and want_sel:
+        sel_out = torch.empty(B * H * (W + R), dtype=torch.int32, device=dev)
+    _check(library().sdm_decode_step(
+        _p(kp), _p(qp), _p(v), _p(alpha), _p(beta), _p(M), _p(y), _p(gate), _p(gamma),
+        float(eps), ACT[act], _p(o), _p(sel_out), shape, _stream(stream, dev)),
+        "sdm_decode_step")
+    return dict(y=y, o=o, sel=sel_out)
+
+
+def sdm_norm_gate(y, *, gate=None, gamma=None, eps: float = 1e-6, act: str = "silu", o=None,
+                  stream=None):
+    """o = y * rsqrt(mean(y^2) + eps) * gamma * act(gate) over the last axis of y."""
+    _need(y, "y", torch.float32)
+    _need(gate, "gate", device=y.device)
+    _need(gamma, "gamma", torch.float32, y.device)
+    d_v = y.shape[-1]
+    rows = y.numel() // d_v
+    o = torch.empty_like(y) if o is None else o
+    _need(o, "o", torch.float32, y.device)
+    dt = _in_dtype(gate) if gate is not None else SDM_F32
+    shape = shape_of(rows, 1, 1, 1, 1, 1, 1, d_v, dt)
+    _check(library().sdm_norm_gate(_p(y), _p(gate), _p(gamma), float(eps), ACT[act], shape,
+                                   _p(o), _stream(stream, y.device)), "sdm_norm_gate")
+    return o
+
+
+def sdm_get_device_status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device status code."""
+    return int(library().sdm_get_device_status(_stream(stream)))

@@ -1,0 +1,424 @@
+// sdm.cu -- the C ABI of the SDM memory pass (declared in include/sdm.h): host-side
+// validation, scratch layout, launch configuration and dispatch to the sm_100a kernels.
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "norm_init.cuh"
+#include "scan_seq.cuh"
+#include "select.cuh"
+
+using namespace sdm;
+
+namespace {
+
+constexpr int MAX_DEVICES = 64;
+constexpr size_t WS_ALIGN = 256;
+
+#define SDM_CUDA_TRY(expr)                       \
+  do {                                           \
+    if ((expr) != cudaSuccess) {                 \
+      (void)cudaGetLastError();                  \
+      return SDM_ERR_CUDA;                       \
+    }                                            \
+  } while (0)
+
+struct DeviceInfo {
+  int sms = 0;
+  int max_smem_optin = 0;
+  bool attrs_set = false;
+};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev[MAX_DEVICES];
+
+sdm_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  SDM_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= MAX_DEVICES) return SDM_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.attrs_set) {
+    SDM_CUDA_TRY(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    SDM_CUDA_TRY(cudaDeviceGetAttribute(&d.max_smem_optin,
+                                        cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+    const int m = d.max_smem_optin;
+    SDM_CUDA_TRY(cudaFuncSetAttribute(sel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+    SDM_CUDA_TRY(cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+#define SDM_SEQ_ATTR(CW, D) \
+  SDM_CUDA_TRY(cudaFuncSetAttribute(seq_scan_kernel<CW, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+    SDM_SEQ_ATTR(4, 4) SDM_SEQ_ATTR(4, 8) SDM_SEQ_ATTR(8, 4) SDM_SEQ_ATTR(8, 8)
+    SDM_SEQ_ATTR(16, 4) SDM_SEQ_ATTR(16, 8) SDM_SEQ_ATTR(32, 4) SDM_SEQ_ATTR(32, 8)
+#undef SDM_SEQ_ATTR
+    d.attrs_set = true;
+  }
+  *out = &d;
+  return SDM_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Shape rules shared by every entry point (T may be 0 where the caller allows it).
+bool shape_ok(const sdm_shape& s, bool allow_t0) {
+  if (s.B < 1 || s.H < 1 || s.T < (allow_t0 ? 0 : 1)) return false;
+  if (s.S1 < 1 || s.S2 < 1 || s.S1 > SMAX || s.S2 > SMAX) return false;
+  if (s.in_dtype != SDM_F32 && s.in_dtype != SDM_BF16) return false;
+  const int smin = s.S1 < s.S2 ? s.S1 : s.S2;
+  if (s.W < 1 || s.R < 1 || s.W > smin || s.R > smin || s.W > KMAX || s.R > KMAX) return false;
+  const int dmul = s.in_dtype == SDM_BF16 ? 8 : 4;
+  if (s.d_v < dmul || s.d_v > 1024 || s.d_v % dmul != 0) return false;
+  if ((long long)s.S1 * s.S2 > 2147483647LL) return false;
+  return true;
+}
+
+size_t state_elems(const sdm_shape& s) {
+  return (size_t)s.B * s.H * (size_t)s.S1 * s.S2 * s.d_v;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+struct WsLayout {
+  int ldw, ldr;
+  size_t off_idx_w, off_wt_w, off_idx_r, off_wt_r, total;
+};
+
+WsLayout ws_layout(const sdm_shape& s) {
+  WsLayout L;
+  L.ldw = (int)round_up((size_t)s.W, 4);
+  L.ldr = (int)round_up((size_t)s.R, 4);
+  const size_t rows = (size_t)s.B * s.T * s.H;
+  L.off_idx_w = 0;
+  L.off_wt_w = round_up(L.off_idx_w + rows * L.ldw * 4, WS_ALIGN);
+  L.off_idx_r = round_up(L.off_wt_w + rows * L.ldw * 4, WS_ALIGN);
+  L.off_wt_r = round_up(L.off_idx_r + rows * L.ldr * 4, WS_ALIGN);
+  L.total = round_up(L.off_wt_r + rows * L.ldr * 4, WS_ALIGN);
+  return L;
+}
+
+// Selection of one or two jobs over `rows` score rows.
+sdm_status launch_select(const SelJob& j0, const SelJob* j1, long long rows, int S1, int S2,
+                         int bf16, cudaStream_t st) {
+  DeviceInfo* di;
+  sdm_status rc = device_info(&di);
+  if (rc != SDM_OK) return rc;
+  if (rows == 0) return SDM_OK;
+  const int K1 = j1 ? j1->K : j0.K;
+  int warps = 8;
+  size_t smem = sel_smem_bytes(S1, S2, j0.K, K1, warps);
+  while (warps > 1 && smem > (size_t)di->max_smem_optin / 2) {
+    warps >>= 1;
+    smem = sel_smem_bytes(S1, S2, j0.K, K1, warps);
+  }
+  if (smem > (size_t)di->max_smem_optin) return SDM_ERR_UNSUPPORTED;
+  int per_sm = 0;
+  SDM_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sel_kernel, warps * 32, smem));
+  if (per_sm < 1) return SDM_ERR_UNSUPPORTED;
+  const long long total_rows = rows * (j1 ? 2 : 1);
+  long long grid = (long long)di->sms * per_sm;
+  const long long need = (total_rows + warps - 1) / warps;
+  if (grid > need) grid = need;
+  const int kmax = j0.K > K1 ? j0.K : K1;
+  sel_kernel<<<(unsigned)grid, warps * 32, smem, st>>>(j0, j1 ? *j1 : j0, rows, j1 ? 2 : 1, S1,
+                                                       S2, bf16, kmax);
+  SDM_CUDA_TRY(cudaGetLastError());
+  return SDM_OK;
+}
+
+int env_int(const char* name, int dflt) {
+  const char* v = getenv(name);
+  return v ? atoi(v) : dflt;
+}
+
+template <int CW, int D>
+sdm_status launch_seq_t(const SeqArgs& a, int grid, size_t smem, cudaStream_t st) {
+  seq_scan_kernel<CW, D><<<grid, SEQ_THREADS, smem, st>>>(a);
+  SDM_CUDA_TRY(cudaGetLastError());
+  return SDM_OK;
+}
+
+// Column-slice width CW and prefetch distance D of the sequential engine: one CTA per
+// (sequence, head, slice) and all CTAs resident at once; wider slices while there are
+// enough CTAs to cover the SMs, then narrower ones.
+sdm_status launch_seq(const SeqArgs& a, cudaStream_t st) {
+  DeviceInfo* di;
+  sdm_status rc = device_info(&di);
+  if (rc != SDM_OK) return rc;
+  const int v_esz = a.v_bf16 ? 2 : 4;
+  const int bh = a.B * a.H;
+  const int cws[4] = {32, 16, 8, 4};
+  int CW = 0;
+  const int force_cw = env_int("SDM_SEQ_CW", 0);
+  for (int i = 0; i < 4; ++i) {
+    const int c = cws[i];
+    if (a.d_v % c != 0 || c * v_esz < 16) continue;
+    if (force_cw) {
+      if (c == force_cw) CW = c;
+      continue;
+    }
+    CW = c;
+    if ((long long)bh * (a.d_v / c) * 5 >= (long long)di->sms * 4) break;
+  }
+  if (CW == 0) return SDM_ERR_UNSUPPORTED;
+  int D = env_int("SDM_SEQ_D", CW >= 32 ? 4 : 8);
+  if (D != 4 && D != 8) D = 4;
+  SeqLayout L = seq_layout(a.ldw, a.ldr, CW, v_esz, D);
+  if (L.total > (size_t)di->max_smem_optin && D == 8) {
+    D = 4;
+    L = seq_layout(a.ldw, a.ldr, CW, v_esz, D);
+  }
+  if (L.total > (size_t)di->max_smem_optin) return SDM_ERR_UNSUPPORTED;
+  const int grid = bh * (a.d_v / CW);
+  const size_t smem = L.total;
+#define SDM_SEQ_CASE(C, DD) \
+  if (CW == C && D == DD) return launch_seq_t<C, DD>(a, grid, smem, st);
+  SDM_SEQ_CASE(32, 4) SDM_SEQ_CASE(32, 8) SDM_SEQ_CASE(16, 4) SDM_SEQ_CASE(16, 8)
+  SDM_SEQ_CASE(8, 4) SDM_SEQ_CASE(8, 8) SDM_SEQ_CASE(4, 4) SDM_SEQ_CASE(4, 8)
+#undef SDM_SEQ_CASE
+  return SDM_ERR_UNSUPPORTED;
+}
+
+sdm_status launch_norm_gate(const float* y, const void* gate, int gate_bf16, const float* gamma,
+                            float eps, int act, long long rows, int d_v, float* o,
+                            cudaStream_t st) {
+  DeviceInfo* di;
+  sdm_status rc = device_info(&di);
+  if (rc != SDM_OK) return rc;
+  if (rows == 0) return SDM_OK;
+  long long blocks = (rows + 7) / 8;
+  const long long cap = (long long)di->sms * 8;
+  if (blocks > cap) blocks = cap;
+  norm_gate_kernel<<<(unsigned)blocks, 256, 0, st>>>(y, gate, gate_bf16, gamma, eps, act, rows,
+                                                     d_v, o);
+  SDM_CUDA_TRY(cudaGetLastError());
+  return SDM_OK;
+}
+
+sdm_status launch_state_init(const float* M0, float* M, const sdm_shape& s, cudaStream_t st) {
+  DeviceInfo* di;
+  sdm_status rc = device_info(&di);
+  if (rc != SDM_OK) return rc;
+  const long long per_head4 = (long long)s.S1 * s.S2 * s.d_v / 4;
+  const long long total = per_head4 * s.B * s.H;
+  long long blocks = (total + 255) / 256;
+  const long long cap = (long long)di->sms * 16;
+  if (blocks > cap) blocks = cap;
+  state_init_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(M0),
+                                                      reinterpret_cast<float4*>(M), s.B, s.H,
+                                                      per_head4);
+  SDM_CUDA_TRY(cudaGetLastError());
+  return SDM_OK;
+}
+
+bool act_ok(int act) { return act >= SDM_GATE_SILU && act <= SDM_GATE_IDENTITY; }
+
+}  // namespace
+
+extern "C" {
+
+const char* sdm_status_string(sdm_status status) {
+  switch (status) {
+    case SDM_OK: return "SDM_OK";
+    case SDM_ERR_INVALID_ARG: return "SDM_ERR_INVALID_ARG";
+    case SDM_ERR_UNSUPPORTED: return "SDM_ERR_UNSUPPORTED";
+    case SDM_ERR_CUDA: return "SDM_ERR_CUDA";
+    case SDM_ERR_DEVICE_CHECK: return "SDM_ERR_DEVICE_CHECK";
+    case SDM_ERR_TIMEOUT: return "SDM_ERR_TIMEOUT";
+  }
+  return "SDM_ERR_UNKNOWN";
+}
+
+size_t sdm_workspace_size(sdm_shape shape, int32_t engine) {
+  if (!shape_ok(shape, true)) return 0;
+  if (engine < SDM_ENGINE_AUTO || engine > SDM_ENGINE_SLOT) return 0;
+  return ws_layout(shape).total;
+}
+
+sdm_status sdm_select(const void* halves, sdm_shape shape, int32_t K, int32_t* idx, float* wt,
+                      void* stream) {
+  sdm_shape s = shape;  // only B, T, H, S1, S2 and in_dtype matter here
+  s.W = s.R = 1;
+  s.d_v = s.in_dtype == SDM_BF16 ? 8 : 4;
+  if (!shape_ok(s, true)) return SDM_ERR_INVALID_ARG;
+  const int smin = s.S1 < s.S2 ? s.S1 : s.S2;
+  if (K < 1 || K > smin || K > KMAX) return SDM_ERR_INVALID_ARG;
+  if (!halves || !idx || !wt) return SDM_ERR_INVALID_ARG;
+  if (!aligned16(halves) || !aligned16(idx) || !aligned16(wt)) return SDM_ERR_INVALID_ARG;
+  SelJob j{halves, idx, wt, K, K};
+  return launch_select(j, nullptr, (long long)s.B * s.T * s.H, s.S1, s.S2,
+                       s.in_dtype == SDM_BF16, static_cast<cudaStream_t>(stream));
+}
+
+sdm_status sdm_state_init(const float* M0, float* M, sdm_shape shape, void* stream) {
+  // only B, H, N = S1*S2 and d_v matter here
+  if (shape.B < 1 || shape.H < 1 || shape.S1 < 1 || shape.S2 < 1) return SDM_ERR_INVALID_ARG;
+  if (shape.d_v < 4 || shape.d_v > 1024 || shape.d_v % 4 != 0) return SDM_ERR_INVALID_ARG;
+  if ((long long)shape.S1 * shape.S2 > 2147483647LL) return SDM_ERR_INVALID_ARG;
+  if (!M0 || !M || !aligned16(M0) || !aligned16(M)) return SDM_ERR_INVALID_ARG;
+  const size_t n = state_elems(shape) * 4;
+  if (overlaps(M, n, M0, n / shape.B)) return SDM_ERR_INVALID_ARG;
+  return launch_state_init(M0, M, shape, static_cast<cudaStream_t>(stream));
+}
+
+sdm_status sdm_norm_gate(const float* y, const void* gate, const float* gamma, float eps,
+                         int32_t act, sdm_shape shape, float* o, void* stream) {
+  sdm_shape s = shape;  // only B, T, H, d_v and in_dtype matter here
+  s.S1 = s.S2 = 1;
+  s.W = s.R = 1;
+  if (!shape_ok(s, true)) return SDM_ERR_INVALID_ARG;
+  if (!y || !o || !act_ok(act) || !(eps >= 0.0f)) return SDM_ERR_INVALID_ARG;
+  if (!aligned16(y) || !aligned16(o) || (gate && !aligned16(gate)) ||
+      (gamma && !aligned16(gamma)))
+    return SDM_ERR_INVALID_ARG;
+  return launch_norm_gate(y, gate, s.in_dtype == SDM_BF16, gamma, eps, act,
+                          (long long)s.B * s.T * s.H, s.d_v, o,
+                          static_cast<cudaStream_t>(stream));
+}
+
+sdm_status sdm_scan_forward(const void* kp, const void* qp, const void* v, const float* alpha,
+                            const float* beta, const float* M0, float* M, int32_t init,
+                            float* y, const void* gate, const float* gamma, float eps,
+                            int32_t act, float* o, int32_t* sel_out, int32_t engine, void* ws,
+                            size_t ws_bytes, sdm_shape shape, void* stream) {
+  const sdm_shape& s = shape;
+  if (!shape_ok(s, true)) return SDM_ERR_INVALID_ARG;
+  if (init != SDM_INIT_FROM_M0 && init != SDM_CONTINUE) return SDM_ERR_INVALID_ARG;
+  if (engine < SDM_ENGINE_AUTO || engine > SDM_ENGINE_SLOT) return SDM_ERR_INVALID_ARG;
+  if (!act_ok(act) || !(eps >= 0.0f)) return SDM_ERR_INVALID_ARG;
+  if (!M || !aligned16(M)) return SDM_ERR_INVALID_ARG;
+  if (init == SDM_INIT_FROM_M0) {
+    if (!M0 || !aligned16(M0)) return SDM_ERR_INVALID_ARG;
+    const size_t n = state_elems(s) * 4;
+    if (overlaps(M, n, M0, n / s.B)) return SDM_ERR_INVALID_ARG;
+  }
+  if (s.T > 0) {
+    if (!kp || !qp || !v || !alpha || !beta || !y) return SDM_ERR_INVALID_ARG;
+    const void* ptrs[] = {kp, qp, v, alpha, beta, y, gate, gamma, o, sel_out};
+    for (const void* p : ptrs)
+      if (p && !aligned16(p)) return SDM_ERR_INVALID_ARG;
+    const WsLayout WL = ws_layout(s);
+    if (!ws || ws_bytes < WL.total || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN) != 0)
+      return SDM_ERR_INVALID_ARG;
+  }
+  if (engine == SDM_ENGINE_SLOT) return SDM_ERR_UNSUPPORTED;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  sdm_status rc;
+  if (init == SDM_INIT_FROM_M0) {
+    rc = launch_state_init(M0, M, s, st);
+    if (rc != SDM_OK) return rc;
+  }
+  if (s.T == 0) return SDM_OK;
+
+  const WsLayout WL = ws_layout(s);
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  int32_t* idx_w = reinterpret_cast<int32_t*>(w + WL.off_idx_w);
+  float* wt_w = reinterpret_cast<float*>(w + WL.off_wt_w);
+  int32_t* idx_r = reinterpret_cast<int32_t*>(w + WL.off_idx_r);
+  float* wt_r = reinterpret_cast<float*>(w + WL.off_wt_r);
+  const long long rows = (long long)s.B * s.T * s.H;
+  const int bf16 = s.in_dtype == SDM_BF16;
+
+  SelJob jw{kp, idx_w, wt_w, s.W, WL.ldw};
+  SelJob jr{qp, idx_r, wt_r, s.R, WL.ldr};
+  rc = launch_select(jw, &jr, rows, s.S1, s.S2, bf16, st);
+  if (rc != SDM_OK) return rc;
+  if (sel_out) {
+    SDM_CUDA_TRY(cudaMemcpy2DAsync(sel_out, (size_t)s.W * 4, idx_w, (size_t)WL.ldw * 4,
+                                   (size_t)s.W * 4, (size_t)rows, cudaMemcpyDeviceToDevice, st));
+    SDM_CUDA_TRY(cudaMemcpy2DAsync(sel_out + (size_t)rows * s.W, (size_t)s.R * 4, idx_r,
+                                   (size_t)WL.ldr * 4, (size_t)s.R * 4, (size_t)rows,
+                                   cudaMemcpyDeviceToDevice, st));
+  }
+
+  SeqArgs a;
+  a.idx_w = idx_w;
+  a.wt_w = wt_w;
+  a.idx_r = idx_r;
+  a.wt_r = wt_r;
+  a.alpha = alpha;
+  a.beta = beta;
+  a.v = v;
+  a.M = M;
+  a.y = y;
+  a.B = s.B;
+  a.T = s.T;
+  a.H = s.H;
+  a.N = s.S1 * s.S2;
+  a.W = s.W;
+  a.R = s.R;
+  a.ldw = WL.ldw;
+  a.ldr = WL.ldr;
+  a.d_v = s.d_v;
+  a.v_bf16 = bf16;
+  rc = launch_seq(a, st);
+  if (rc != SDM_OK) return rc;
+
+  if (o) {
+    rc = launch_norm_gate(y, gate, bf16, gamma, eps, act, rows, s.d_v, o, st);
+    if (rc != SDM_OK) return rc;
+  }
+  return SDM_OK;
+}
+
+sdm_status sdm_decode_step(const void* kp, const void* qp, const void* v, const float* alpha,
+                           const float* beta, float* M, float* y, const void* gate,
+                           const float* gamma, float eps, int32_t act, float* o,
+                           int32_t* sel_out, sdm_shape shape, void* stream) {
+  sdm_shape s = shape;
+  s.T = 1;
+  if (!shape_ok(s, false)) return SDM_ERR_INVALID_ARG;
+  if (!act_ok(act) || !(eps >= 0.0f)) return SDM_ERR_INVALID_ARG;
+  if (!kp || !qp || !v || !alpha || !beta || !M || !y) return SDM_ERR_INVALID_ARG;
+  const void* ptrs[] = {kp, qp, v, alpha, beta, M, y, gate, gamma, o, sel_out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return SDM_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  sdm_status rc = device_info(&di);
+  if (rc != SDM_OK) return rc;
+  const DecLayout L = dec_layout(s.S1, s.S2, s.W, s.R, s.d_v);
+  if (L.total > (size_t)di->max_smem_optin) return SDM_ERR_UNSUPPORTED;
+  DecodeArgs a;
+  a.kp = kp;
+  a.qp = qp;
+  a.v = v;
+  a.alpha = alpha;
+  a.beta = beta;
+  a.M = M;
+  a.y = y;
+  a.gate = gate;
+  a.gamma = gamma;
+  a.o = o;
+  a.sel_out = sel_out;
+  a.eps = eps;
+  a.act = act;
+  a.BH = s.B * s.H;
+  a.S1 = s.S1;
+  a.S2 = s.S2;
+  a.W = s.W;
+  a.R = s.R;
+  a.N = s.S1 * s.S2;
+  a.d_v = s.d_v;
+  a.in_bf16 = s.in_dtype == SDM_BF16;
+  decode_kernel<<<a.BH, DEC_THREADS, L.total, static_cast<cudaStream_t>(stream)>>>(a);
+  SDM_CUDA_TRY(cudaGetLastError());
+  return SDM_OK;
+}
+
+sdm_status sdm_get_device_status(void* stream) {
+  SDM_CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  unsigned int v = 0, zero = 0;
+  SDM_CUDA_TRY(cudaMemcpyFromSymbol(&v, g_status, sizeof(v)));
+  SDM_CUDA_TRY(cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)));
+  if (v & STATUS_TIMEOUT) return SDM_ERR_TIMEOUT;
+  if (v & STATUS_BAD_INDEX) return SDM_ERR_DEVICE_CHECK;
+  return SDM_OK;
+}
+
+}  // extern "C"

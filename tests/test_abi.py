@@ -1,0 +1,119 @@
+"""The C ABI without a GPU: the library loads, exports every entry point the header
+declares, sizes its scratch, and rejects bad arguments on the host before any launch."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def sdm():
+    from sparse_memory_linear_b200.build import build_library
+    build_library()
+    import sparse_memory_linear_b200 as m
+    m.library()
+    return m
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "sdm.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sdm_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(sdm):
+    names = declared_functions()
+    assert "sdm_scan_forward" in names and "sdm_decode_step" in names
+    lib = ctypes.CDLL(sdm.library_path)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_library_is_the_in_tree_build(sdm):
+    sdm.library()
+    maps = open("/proc/self/maps").read()
+    assert sdm.library_path in maps
+
+
+def good_shape(sdm, **kw):
+    d = dict(B=2, T=16, H=3, S1=32, S2=32, W=8, R=8, d_v=64, in_dtype=sdm.SDM_BF16)
+    d.update(kw)
+    return sdm.shape_of(**d)
+
+
+def test_workspace_size(sdm):
+    s = good_shape(sdm, W=6, R=8)
+    rows = 2 * 16 * 3
+    # four regions (idx and weights of writes and reads), rows padded to 4 entries
+    def r256(x):
+        return (x + 255) // 256 * 256
+    want = r256(rows * 8 * 4) * 2 + r256(rows * 8 * 4) * 2
+    assert sdm.sdm_workspace_size(s) == want
+    assert sdm.sdm_workspace_size(good_shape(sdm, W=40)) == 0  # W > S
+    assert sdm.sdm_workspace_size(good_shape(sdm, d_v=12)) == 0  # bf16 needs d_v % 8 == 0
+
+
+FAKE = 0x10000  # aligned, never dereferenced: validation rejects the call first
+
+
+def scan(sdm, shape, **over):
+    args = dict(kp=FAKE, qp=FAKE, v=FAKE, alpha=FAKE, beta=FAKE, M0=FAKE + 0x100000000,
+                M=FAKE, init=0, y=FAKE, gate=None, gamma=None, eps=1e-6, act=0, o=None,
+                sel=None, engine=0, ws=FAKE, ws_bytes=1 << 40)
+    args.update(over)
+    P = ctypes.c_void_p
+    return sdm.library().sdm_scan_forward(
+        P(args["kp"]), P(args["qp"]), P(args["v"]), P(args["alpha"]), P(args["beta"]),
+        P(args["M0"]), P(args["M"]), args["init"], P(args["y"]), P(args["gate"]),
+        P(args["gamma"]), args["eps"], args["act"], P(args["o"]), P(args["sel"]),
+        args["engine"], P(args["ws"]), args["ws_bytes"], shape, None)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(kp=None), dict(qp=None), dict(v=None), dict(alpha=None), dict(beta=None),
+    dict(M=None), dict(y=None), dict(ws=None), dict(M0=None),
+    dict(kp=FAKE + 4), dict(M=FAKE + 8), dict(ws=FAKE + 16), dict(gate=FAKE + 2),
+    dict(ws_bytes=16), dict(init=7), dict(engine=9), dict(act=3), dict(eps=-1.0),
+    dict(M0=FAKE),  # M0 overlaps M
+])
+def test_scan_rejects_bad_arguments(sdm, bad):
+    assert scan(sdm, good_shape(sdm), **bad) == 1
+
+
+@pytest.mark.parametrize("kw", [
+    dict(W=0), dict(R=0), dict(W=33), dict(R=40), dict(S1=0), dict(S2=5000), dict(B=0),
+    dict(H=0), dict(T=-1), dict(d_v=12), dict(d_v=0), dict(d_v=2048), dict(in_dtype=5),
+    dict(S1=256, S2=256, W=129, R=8),
+])
+def test_scan_rejects_bad_shapes(sdm, kw):
+    assert scan(sdm, good_shape(sdm, **kw)) == 1
+
+
+def test_decode_and_select_and_norm_reject_bad_arguments(sdm):
+    lib = sdm.library()
+    P = ctypes.c_void_p
+    s = good_shape(sdm)
+    # decode: missing M, then misaligned v
+    assert lib.sdm_decode_step(P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), None, P(FAKE),
+                               None, None, 1e-6, 0, None, None, s, None) == 1
+    assert lib.sdm_decode_step(P(FAKE), P(FAKE), P(FAKE + 4), P(FAKE), P(FAKE), P(FAKE),
+                               P(FAKE), None, None, 1e-6, 0, None, None, s, None) == 1
+    # select: K out of range, null output
+    assert lib.sdm_select(P(FAKE), s, 0, P(FAKE), P(FAKE), None) == 1
+    assert lib.sdm_select(P(FAKE), s, 33, P(FAKE), P(FAKE), None) == 1
+    assert lib.sdm_select(P(FAKE), s, 8, None, P(FAKE), None) == 1
+    # norm: bad activation, null y
+    assert lib.sdm_norm_gate(P(FAKE), None, None, 1e-6, 5, s, P(FAKE), None) == 1
+    assert lib.sdm_norm_gate(None, None, None, 1e-6, 0, s, P(FAKE), None) == 1
+    # state init: overlapping M and M0
+    assert lib.sdm_state_init(P(FAKE), P(FAKE), s, None) == 1
+
+
+def test_status_strings(sdm):
+    assert sdm.sdm_status_string(0) == "SDM_OK"
+    assert sdm.sdm_status_string(4) == "SDM_ERR_DEVICE_CHECK"
+    assert sdm.sdm_status_string(99) == "SDM_ERR_UNKNOWN"

@@ -1,0 +1,511 @@
+#!/usr/bin/env python
+"""Benchmark of the SDM memory pass on B200.
+
+Headline: prefill of the long skewed workload (B=1, H=4, T=262144, N=1048576 = 1024 x 1024,
+W=R=64, d_v=256, bf16 inputs, fp32 state) -- one step is one sdm_scan_forward call doing
+every step of the pass: M0 broadcast, product-key selection, sparse gated delta write,
+sparse read and RMSNorm + gate.  Reported as token*heads/s (whole job), beside the HBM
+roofline of the scan kernel, the end-to-end figure through the C ABI with host buffers,
+and the CPU oracle timed on the host cores.  A second object reports decode on the
+batched-decode workload (64 sequences x 8 heads, N=262144, d_v=128): 256 successive
+sdm_decode_step calls, as plain launches and replayed from a CUDA graph.
+
+Multi-GPU: the pass has no exchange step (every (sequence, head) is independent), so each
+rank runs its own batch of the same shape (weak scaling), timed between barriers and
+reduced as the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sdm|reference]
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import sdm_synth  # noqa: E402
+
+METRIC = "SDM layer tokens*heads/s (prefill & decode) and HBM GB/s as % of B200 peak"
+UNIT = "token*heads/s"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------------- helpers
+def algorithmic_bytes(wl) -> int:
+    """Bytes per token-head the pass must move: the W rows read and rewritten and the R
+    rows read (fp32 state), both score halves and v.  Gate, alpha/beta, y/o and the
+    selection scratch are not counted."""
+    s_in = 2 if wl.in_dtype == torch.bfloat16 else 4
+    return (2 * wl.W + wl.R) * wl.d_v * 4 + 2 * (wl.S1 + wl.S2) * s_in + wl.d_v * s_in
+
+
+def scan_kernel_bytes(wl) -> int:
+    """Bytes per token-head of the scan engine alone: the state rows only."""
+    return (2 * wl.W + wl.R) * wl.d_v * 4
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_PATH) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class Dist:
+    """torch.distributed plumbing: barrier and max over ranks (nccl on GPUs, gloo on CPU)."""
+
+    def __init__(self, backend: str | None = None):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import torch.distributed as dist
+            if backend is None:
+                backend = "nccl" if torch.cuda.is_available() else "gloo"
+            self.backend = backend
+            if backend == "nccl":
+                torch.cuda.set_device(self.local_rank)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local_rank)
+                                    if backend == "nccl" else None)
+            self.pg = dist
+
+    def _dev(self):
+        if self.pg is not None and self.backend == "nccl":
+            return torch.device("cuda", self.local_rank)
+        return torch.device("cpu")
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if self.pg is None:
+            return float(x)
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self._dev())
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum(self, x: float) -> float:
+        if self.pg is None:
+            return float(x)
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self._dev())
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+            self.pg = None
+
+
+def weak_scaling_value(units_per_rank: float, max_seconds: float, world: int) -> float:
+    """Whole-job throughput: every rank processed units_per_rank in at most max_seconds."""
+    return units_per_rank * world / max_seconds
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.05):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # clocks are reported as unavailable, never guessed
+            self.nv = None
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+                r = get(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def report(self):
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        busy = [s for s in self.samples]
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+def timed(fn, steps: int, warmup: int, dist: Dist, stream):
+    """Runs fn warmup times untimed, then times exactly `steps` calls with CUDA events on
+    `stream`, bracketed by barrier + synchronize.  Returns max-over-ranks seconds."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    return dist.max(a.elapsed_time(b) / 1e3)
+
+
+# ----------------------------------------------------------------- the CUDA path
+def bench_prefill(args, dist: Dist, dev):
+    import sparse_memory_linear_b200 as sdm
+
+    wl = sdm_synth.WORKLOADS[args.workload]
+    stream = torch.cuda.current_stream(dev)
+    g = {k: v.to(dev) for k, v in sdm_synth.make_inputs(wl, device=dev).items()}
+    torch.cuda.synchronize()
+    M = torch.empty((wl.B, wl.H, wl.N, wl.d_v), dtype=torch.float32, device=dev)
+    shape = sdm.shape_of(wl.B, wl.T, wl.H, wl.S1, wl.S2, wl.W, wl.R, wl.d_v,
+                         sdm.SDM_BF16 if wl.in_dtype == torch.bfloat16 else sdm.SDM_F32)
+    ws = torch.empty(sdm.sdm_workspace_size(shape), dtype=torch.uint8, device=dev)
+    y = torch.empty((wl.B, wl.T, wl.H, wl.d_v), dtype=torch.float32, device=dev)
+    o = torch.empty_like(y)
+
+    def step():
+        sdm.sdm_scan_forward(g["kp"], g["qp"], g["v"], g["alpha"], g["beta"], M, W=wl.W,
+                             R=wl.R, S1=wl.S1, M0=g["M0"], init="m0", gate=g["gate"], y=y,
+                             o=o, ws=ws, stream=stream)
+
+    sdm.sdm_profile_enable(True)
+    with ClockSampler(dev.index) as clk:
+        secs = timed(step, args.steps, args.warmup, dist, stream)
+    prof = sdm.sdm_profile_read()
+    sdm.sdm_profile_enable(False)
+    if sdm.sdm_get_device_status() != 0:
+        raise RuntimeError("device status word set during the benchmark")
+
+    th = wl.B * wl.T * wl.H
+    value = weak_scaling_value(th * args.steps, secs, dist.world)
+    # per-kernel averages over warm-up and timed launches (events on the launching stream)
+    launches = {k: n for k, (ms, n) in prof.items() if n}
+    avg_ms = {k: ms / n for k, (ms, n) in prof.items() if n}
+    scan_kind = "scan_slot" if prof["scan_slot"][1] else "scan_seq"
+    peak, peak_kind = hbm_peak()
+    scan_bytes = th * scan_kernel_bytes(wl)
+    achieved = scan_bytes / (avg_ms[scan_kind] * 1e-3) / 1e9
+    step_ms = secs / args.steps * 1e3
+    res = {
+        "value": value,
+        "ms_per_step": step_ms,
+        "clocks": clk.report(),
+        "kernels_avg_ms": avg_ms,
+        "kernels_share": {k: avg_ms[k] / sum(avg_ms.values()) for k in avg_ms},
+        "gpu_launches": sum(launches.values()) * args.steps // (args.steps + args.warmup),
+        "roofline": {
+            "kernel": f"seq_scan_kernel" if scan_kind == "scan_seq" else "slot_scan_kernel",
+            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "peak_kind": f"{peak_kind} (burst copy)",
+            "traffic": None,
+            "algorithmic_bytes_per_launch": scan_bytes,
+            "bytes_per_token_head": scan_kernel_bytes(wl),
+        },
+        "whole_step_hbm": {
+            "bytes_per_token_head": algorithmic_bytes(wl),
+            "GBps": th * algorithmic_bytes(wl) / (step_ms * 1e-3) / 1e9,
+        },
+    }
+
+    # end to end through the same call with host buffers: inputs copied in from pinned
+    # host memory and the layer output copied back, every step
+    if not args.no_e2e:
+        host = {k: torch.empty_like(g[k], device="cpu").pin_memory().copy_(g[k])
+                for k in ("kp", "qp", "v", "alpha", "beta", "gate")}
+        o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = o_host.numel() * o_host.element_size()
+
+        def step_e2e():
+            for k, t in host.items():
+                g[k].copy_(t, non_blocking=True)
+            step()
+            o_host.copy_(o, non_blocking=True)
+
+        secs_e = timed(step_e2e, max(1, min(args.steps, 3)), 1, dist, stream)
+        res["e2e"] = {"value": weak_scaling_value(th * max(1, min(args.steps, 3)), secs_e,
+                                                  dist.world),
+                      "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        del host, o_host
+    res["_inputs"] = (wl, g)
+    return res
+
+
+def bench_decode(args, dist: Dist, dev):
+    import sparse_memory_linear_b200 as sdm
+
+    wl = sdm_synth.WORKLOADS[args.decode_workload]
+    stream = torch.cuda.current_stream(dev)
+    nsteps = wl.T
+    steps = [{k: t.to(dev) for k, t in sdm_synth.make_inputs(wl, device=dev, step=s).items()}
+             for s in range(nsteps)]
+    M0 = steps[0].pop("M0")
+    M = torch.empty((wl.B, wl.H, wl.N, wl.d_v), dtype=torch.float32, device=dev)
+    sdm.sdm_state_init(M0, M)
+    y = torch.empty((wl.B, wl.H, wl.d_v), dtype=torch.float32, device=dev)
+    o = torch.empty_like(y)
+
+    def run_all():
+        for s in steps:
+            sdm.sdm_decode_step(s["kp"], s["qp"], s["v"], s["alpha"], s["beta"], M, W=wl.W,
+                                R=wl.R, S1=wl.S1, gate=s["gate"], y=y, o=o, stream=stream)
+
+    reps = max(1, args.steps // 2)
+    sdm.sdm_profile_enable(True)
+    secs = timed(run_all, reps, 1, dist, stream)
+    prof = sdm.sdm_profile_read()
+    sdm.sdm_profile_enable(False)
+    ms_k, n_k = prof["decode"]
+    per_step = secs / (reps * nsteps)
+    th = wl.B * wl.H
+    peak, peak_kind = hbm_peak()
+    step_bytes = th * algorithmic_bytes(wl)
+    kernel_s = ms_k / n_k * 1e-3
+    out = {
+        "workload": wl.note, "steps_per_run": nsteps, "runs": reps,
+        "value": weak_scaling_value(th, per_step, dist.world), "unit": UNIT,
+        "us_per_step": per_step * 1e6,
+        "roofline": {"kernel": "decode_kernel", "bound": "hbm",
+                     "achieved": step_bytes / kernel_s / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": step_bytes / kernel_s / 1e9 / peak,
+                     "peak_kind": f"{peak_kind} (burst copy)",
+                     "algorithmic_bytes_per_launch": step_bytes, "kernel_us": kernel_s * 1e6},
+    }
+    # the same 256 steps captured once into a CUDA graph and replayed
+    try:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            run_all()
+        stream.wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            for s in steps:
+                sdm.sdm_decode_step(s["kp"], s["qp"], s["v"], s["alpha"], s["beta"], M,
+                                    W=wl.W, R=wl.R, S1=wl.S1, gate=s["gate"], y=y, o=o,
+                                    stream=side)
+        secs_g = timed(graph.replay, reps, 1, dist, stream)
+        out["graph_us_per_step"] = secs_g / (reps * nsteps) * 1e6
+        out["graph_value"] = weak_scaling_value(th, secs_g / (reps * nsteps), dist.world)
+        del graph
+    except Exception as e:  # reported, not hidden
+        out["graph_error"] = repr(e)
+    if sdm.sdm_get_device_status() != 0:
+        raise RuntimeError("device status word set during the decode benchmark")
+    del M, steps
+    torch.cuda.empty_cache()
+    return out
+
+
+# ------------------------------------------------------------- the CPU oracle arm
+def cpu_units_sample(wl, tokens: int, g=None):
+    """Host arrays of the first `tokens` tokens of sequence 0 (every head) of a workload,
+    taken from device tensors when given, else drawn on the host."""
+    if g is None:
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        sub = wl.replace(B=1, T=tokens)
+        d = sdm_synth.make_inputs(sub, device=dev)
+    else:
+        d = {k: (t[:1, :tokens] if k != "M0" else t) for k, t in g.items()}
+    return {k: v.float().cpu().numpy() for k, v in d.items()}
+
+
+def oracle_sample_time(wl, tokens: int, threads: int, g=None):
+    """The oracle, as it stands, over the first `tokens` tokens of every head of sequence 0
+    (all N rows tracked), one head per thread.  Returns (token-heads, seconds, cores)."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+
+    h = cpu_units_sample(wl, tokens, g)
+    units = [(0, hh) for hh in range(wl.H)]
+    cores = max(1, min(threads, len(units)))
+
+    def one(u):
+        b, hh = u
+        oracle.run_unit(h["kp"], h["qp"], h["v"], h["alpha"], h["beta"], h["M0"], b, hh,
+                        S1=wl.S1, W=wl.W, R=wl.R)
+        return u
+
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(cores) as ex:
+        list(ex.map(one, units))
+    secs = time.perf_counter() - t0
+    return tokens * len(units), secs, cores
+
+
+def run_reference(args, dist: Dist):
+    """The reference arm: the CPU oracle on the same workload, metric and unit."""
+    if dist.rank != 0:
+        return None
+    wl = sdm_synth.WORKLOADS[args.workload]
+    tokens = args.reference_tokens
+    cores = max(1, min(os.cpu_count() or 1, wl.H))
+    for _ in range(args.warmup):
+        oracle_sample_time(wl, max(16, tokens // 8), cores)
+    done, secs = 0, 0.0
+    for _ in range(args.steps):
+        n, s, cores = oracle_sample_time(wl, tokens, cores)
+        done += n
+        secs += s
+    value = done / secs
+    sample = (f"first {tokens} tokens of sequence 0, all {wl.H} heads, every step; "
+              f"{wl.note}")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded counter-based generator)",
+        "config": {"workload": wl.name, "shape": wl.note},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# --------------------------------------------------------------------------- main
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__,
+                                 formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["sdm", "reference"], default="sdm")
+    ap.add_argument("--workload", default="long_skew")
+    ap.add_argument("--decode-workload", default="decode")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=8192,
+                    help="tokens per head of the CPU-oracle sample")
+    ap.add_argument("--reference-tokens", type=int, default=2048)
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="run one part (profiling of a small case)")
+    ap.add_argument("--override", default="",
+                    help="workload fields to change, e.g. B=1,T=4096 (prefill workload)")
+    ap.add_argument("--decode-override", default="",
+                    help="workload fields to change for the decode workload, e.g. B=8")
+    args = ap.parse_args(argv)
+    for attr, key in (("override", "workload"), ("decode_override", "decode_workload")):
+        kv = getattr(args, attr)
+        if kv:
+            base = sdm_synth.WORKLOADS[getattr(args, key)]
+            fields = {k: int(v) for k, v in (x.split("=") for x in kv.split(","))}
+            name = f"{base.name}[{kv}]"
+            sdm_synth.WORKLOADS[name] = base.replace(name=name, **fields)
+            setattr(args, key, name)
+    if args.warmup < 3 and args.impl == "sdm":
+        ap.error("--warmup must be at least 3")
+
+    dist = Dist()
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, dist)
+            if line is not None:
+                print(json.dumps(line), flush=True)
+            return 0
+        if dist.world != args.gpus:
+            if dist.world > 1:
+                raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={dist.world}")
+        dev = torch.device("cuda", dist.local_rank)
+        torch.cuda.set_device(dev)
+        import sparse_memory_linear_b200 as sdm
+        sdm.library()
+
+        if args.only == "decode":
+            out = bench_decode(args, dist, dev)
+            if dist.rank == 0:
+                print(json.dumps({"decode": out}), flush=True)
+            return 0
+        if args.only == "prefill":
+            args.no_decode = True
+        pre = bench_prefill(args, dist, dev)
+        wl, g = pre.pop("_inputs")
+        line = {
+            "metric": METRIC, "value": pre["value"], "unit": UNIT, "n_gpus": dist.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": pre["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded counter-based generator; bf16 inputs, fp32 state)",
+            "config": {"workload": wl.name, "shape": wl.note, "global_batch": wl.B * dist.world,
+                       "seq_len": wl.T, "heads": wl.H, "parallelism": f"replicas x{dist.world}",
+                       "l2": "inputs larger than L2 (9 GB of inputs, 4 GB state per step)",
+                       "step": "sdm_scan_forward: M0 init + select + scan + norm/gate"},
+            "roofline": pre["roofline"], "whole_step_hbm": pre["whole_step_hbm"],
+            "kernels_avg_ms": pre["kernels_avg_ms"], "kernels_share": pre["kernels_share"],
+            "gpu_launches": pre["gpu_launches"], "clocks": pre["clocks"],
+        }
+        if "e2e" in pre:
+            line["e2e"] = pre["e2e"]
+        if not args.no_cpu_baseline and dist.world == 1 and dist.rank == 0:
+            n, s, cores = oracle_sample_time(wl, args.cpu_tokens, os.cpu_count() or 1, g)
+            line["cpu_baseline"] = {
+                "value": n / s, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": f"first {args.cpu_tokens} tokens of sequence 0, all {wl.H} heads "
+                          f"({n} token-heads, {s:.1f} s wall, one head per thread)"}
+        del g
+        torch.cuda.empty_cache()
+        if not args.no_decode:
+            line["decode"] = bench_decode(args, dist, dev)
+        if dist.rank == 0:
+            print(json.dumps(line), flush=True)
+        return 0
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -144,6 +144,28 @@ sdm_status sdm_decode_step(const void *kp, const void *qp, const void *v, const 
 sdm_status sdm_norm_gate(const float *y, const void *gate, const float *gamma, float eps,
                          int32_t act, sdm_shape shape, float *o, void *stream);
 
+/* Kinds of kernel launch reported by the timing calls below. */
+typedef enum {
+    SDM_KERNEL_STATE_INIT = 0, /* M0 broadcast into M                         */
+    SDM_KERNEL_SELECT = 1,     /* step 1 pre-pass                             */
+    SDM_KERNEL_SCAN_SEQ = 2,   /* steps 2-3, token-sequential engine          */
+    SDM_KERNEL_SCAN_SLOT = 3,  /* steps 2-3, slot-parallel engine             */
+    SDM_KERNEL_NORM_GATE = 4,  /* step 4                                      */
+    SDM_KERNEL_DECODE = 5,     /* fused decode step                           */
+    SDM_KERNEL_KINDS = 8
+} sdm_kernel_kind;
+
+/* Kernel timing.  While enabled (on != 0), every kernel launch the library makes is
+ * bracketed by two CUDA events recorded on the launch's stream (a few microseconds of
+ * host time per launch, nothing on the device).  Enabling or disabling drops what was
+ * recorded.  Do not enable it while a stream is being captured into a CUDA graph. */
+sdm_status sdm_profile_enable(int32_t on);
+
+/* Waits for the launches recorded since the last enable/read and returns, per
+ * sdm_kernel_kind, the summed device time in milliseconds (ms[SDM_KERNEL_KINDS]) and the
+ * number of launches (launches[SDM_KERNEL_KINDS]); then forgets them. */
+sdm_status sdm_profile_read(double *ms, int64_t *launches);
+
 /* Synchronises `stream`, then reads and clears the calling device's status word:
  * SDM_OK, SDM_ERR_DEVICE_CHECK (an index outside [0, N) reached a kernel) or
  * SDM_ERR_TIMEOUT (a bounded wait expired).  SDM_ERR_CUDA if the synchronisation fails. */

@@ -18,6 +18,8 @@ from ._binding import (  # noqa: F401
     sdm_decode_step,
     sdm_get_device_status,
     sdm_norm_gate,
+    sdm_profile_enable,
+    sdm_profile_read,
     sdm_scan_forward,
     sdm_select,
     sdm_state_init,

@@ -56,6 +56,8 @@ def library():
         "sdm_norm_gate": ([P, P, P, F, I, S, P, P], I),
         "sdm_get_device_status": ([P], I),
         "sdm_status_string": ([I], ctypes.c_char_p),
+        "sdm_profile_enable": ([I], I),
+        "sdm_profile_read": ([P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -237,6 +239,23 @@ def sdm_norm_gate(y, *, gate=None, gamma=None, eps: float = 1e-6, act: str = "si
     _check(library().sdm_norm_gate(_p(y), _p(gate), _p(gamma), float(eps), ACT[act], shape,
                                    _p(o), _stream(stream, y.device)), "sdm_norm_gate")
     return o
+
+
+KERNEL_KINDS = ("state_init", "select", "scan_seq", "scan_slot", "norm_gate", "decode")
+
+
+def sdm_profile_enable(on: bool = True):
+    """Brackets every library launch with CUDA events on its stream (off by default)."""
+    _check(library().sdm_profile_enable(1 if on else 0), "sdm_profile_enable")
+
+
+def sdm_profile_read() -> dict:
+    """{kind: (total ms, launches)} of the launches recorded since the last enable/read."""
+    ms = (ctypes.c_double * 8)()
+    n = (ctypes.c_int64 * 8)()
+    _check(library().sdm_profile_read(ctypes.cast(ms, ctypes.c_void_p),
+                                      ctypes.cast(n, ctypes.c_void_p)), "sdm_profile_read")
+    return {k: (ms[i], n[i]) for i, k in enumerate(KERNEL_KINDS)}
 
 
 def sdm_get_device_status(stream=None) -> int:

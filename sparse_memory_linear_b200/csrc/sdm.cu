@@ -4,6 +4,7 @@
 #include <string.h>
 
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "decode.cuh"
@@ -58,6 +59,39 @@ sdm_status device_info(DeviceInfo** out) {
   *out = &d;
   return SDM_OK;
 }
+
+// Kernel timing, off by default: when on, every launch is bracketed by two CUDA events
+// recorded on the launch's stream; sdm_profile_read() waits for them and sums per kind.
+struct ProfRec {
+  int kind;
+  cudaEvent_t start, stop;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof_pending;
+
+struct ProfScope {
+  bool on = false;
+  ProfRec rec{};
+  cudaStream_t st;
+  ProfScope(int kind, cudaStream_t stream) : st(stream) {
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    if (!g_prof_on) return;
+    rec.kind = kind;
+    if (cudaEventCreate(&rec.start) != cudaSuccess) return;
+    if (cudaEventCreate(&rec.stop) != cudaSuccess) {
+      cudaEventDestroy(rec.start);
+      return;
+    }
+    on = cudaEventRecord(rec.start, st) == cudaSuccess;
+  }
+  ~ProfScope() {
+    if (!on) return;
+    cudaEventRecord(rec.stop, st);
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    g_prof_pending.push_back(rec);
+  }
+};
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -251,6 +285,7 @@ sdm_status sdm_select(const void* halves, sdm_shape shape, int32_t K, int32_t* i
   if (!halves || !idx || !wt) return SDM_ERR_INVALID_ARG;
   if (!aligned16(halves) || !aligned16(idx) || !aligned16(wt)) return SDM_ERR_INVALID_ARG;
   SelJob j{halves, idx, wt, K, K};
+  ProfScope ps(SDM_KERNEL_SELECT, static_cast<cudaStream_t>(stream));
   return launch_select(j, nullptr, (long long)s.B * s.T * s.H, s.S1, s.S2,
                        s.in_dtype == SDM_BF16, static_cast<cudaStream_t>(stream));
 }
@@ -263,6 +298,7 @@ sdm_status sdm_state_init(const float* M0, float* M, sdm_shape shape, void* stre
   if (!M0 || !M || !aligned16(M0) || !aligned16(M)) return SDM_ERR_INVALID_ARG;
   const size_t n = state_elems(shape) * 4;
   if (overlaps(M, n, M0, n / shape.B)) return SDM_ERR_INVALID_ARG;
+  ProfScope ps(SDM_KERNEL_STATE_INIT, static_cast<cudaStream_t>(stream));
   return launch_state_init(M0, M, shape, static_cast<cudaStream_t>(stream));
 }
 
@@ -276,6 +312,7 @@ sdm_status sdm_norm_gate(const float* y, const void* gate, const float* gamma, f
   if (!aligned16(y) || !aligned16(o) || (gate && !aligned16(gate)) ||
       (gamma && !aligned16(gamma)))
     return SDM_ERR_INVALID_ARG;
+  ProfScope ps(SDM_KERNEL_NORM_GATE, static_cast<cudaStream_t>(stream));
   return launch_norm_gate(y, gate, s.in_dtype == SDM_BF16, gamma, eps, act,
                           (long long)s.B * s.T * s.H, s.d_v, o,
                           static_cast<cudaStream_t>(stream));
@@ -311,6 +348,7 @@ sdm_status sdm_scan_forward(const void* kp, const void* qp, const void* v, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   sdm_status rc;
   if (init == SDM_INIT_FROM_M0) {
+    ProfScope ps(SDM_KERNEL_STATE_INIT, st);
     rc = launch_state_init(M0, M, s, st);
     if (rc != SDM_OK) return rc;
   }
@@ -327,7 +365,10 @@ sdm_status sdm_scan_forward(const void* kp, const void* qp, const void* v, const
 
   SelJob jw{kp, idx_w, wt_w, s.W, WL.ldw};
   SelJob jr{qp, idx_r, wt_r, s.R, WL.ldr};
-  rc = launch_select(jw, &jr, rows, s.S1, s.S2, bf16, st);
+  {
+    ProfScope ps(SDM_KERNEL_SELECT, st);
+    rc = launch_select(jw, &jr, rows, s.S1, s.S2, bf16, st);
+  }
   if (rc != SDM_OK) return rc;
   if (sel_out) {
     SDM_CUDA_TRY(cudaMemcpy2DAsync(sel_out, (size_t)s.W * 4, idx_w, (size_t)WL.ldw * 4,
@@ -357,10 +398,14 @@ sdm_status sdm_scan_forward(const void* kp, const void* qp, const void* v, const
   a.ldr = WL.ldr;
   a.d_v = s.d_v;
   a.v_bf16 = bf16;
-  rc = launch_seq(a, st);
+  {
+    ProfScope ps(SDM_KERNEL_SCAN_SEQ, st);
+    rc = launch_seq(a, st);
+  }
   if (rc != SDM_OK) return rc;
 
   if (o) {
+    ProfScope ps(SDM_KERNEL_NORM_GATE, st);
     rc = launch_norm_gate(y, gate, bf16, gamma, eps, act, rows, s.d_v, o, st);
     if (rc != SDM_OK) return rc;
   }
@@ -406,6 +451,7 @@ sdm_status sdm_decode_step(const void* kp, const void* qp, const void* v, const 
   a.N = s.S1 * s.S2;
   a.d_v = s.d_v;
   a.in_bf16 = s.in_dtype == SDM_BF16;
+  ProfScope ps(SDM_KERNEL_DECODE, static_cast<cudaStream_t>(stream));
   decode_kernel<<<a.BH, DEC_THREADS, L.total, static_cast<cudaStream_t>(stream)>>>(a);
   SDM_CUDA_TRY(cudaGetLastError());
   return SDM_OK;
@@ -419,6 +465,49 @@ sdm_status sdm_get_device_status(void* stream) {
   if (v & STATUS_TIMEOUT) return SDM_ERR_TIMEOUT;
   if (v & STATUS_BAD_INDEX) return SDM_ERR_DEVICE_CHECK;
   return SDM_OK;
+}
+
+sdm_status sdm_profile_enable(int32_t on) {
+  std::vector<ProfRec> drop;
+  {
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    g_prof_on = on != 0;
+    drop.swap(g_prof_pending);
+  }
+  for (ProfRec& r : drop) {
+    cudaEventSynchronize(r.stop);
+    cudaEventDestroy(r.start);
+    cudaEventDestroy(r.stop);
+  }
+  return SDM_OK;
+}
+
+sdm_status sdm_profile_read(double* ms, int64_t* launches) {
+  if (!ms || !launches) return SDM_ERR_INVALID_ARG;
+  std::vector<ProfRec> recs;
+  {
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    recs.swap(g_prof_pending);
+  }
+  for (int k = 0; k < SDM_KERNEL_KINDS; ++k) {
+    ms[k] = 0.0;
+    launches[k] = 0;
+  }
+  sdm_status rc = SDM_OK;
+  for (ProfRec& r : recs) {
+    float t = 0.0f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess ||
+        cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess) {
+      (void)cudaGetLastError();
+      rc = SDM_ERR_CUDA;
+    } else if (r.kind >= 0 && r.kind < SDM_KERNEL_KINDS) {
+      ms[r.kind] += t;
+      launches[r.kind] += 1;
+    }
+    cudaEventDestroy(r.start);
+    cudaEventDestroy(r.stop);
+  }
+  return rc;
 }
 
 }  // extern "C"

@@ -152,6 +152,7 @@ typedef enum {
     SDM_KERNEL_SCAN_SLOT = 3,  /* steps 2-3, slot-parallel engine             */
     SDM_KERNEL_NORM_GATE = 4,  /* step 4                                      */
     SDM_KERNEL_DECODE = 5,     /* fused decode step                           */
+    SDM_KERNEL_SLOT_SORT = 6,  /* slot engine: event build and radix sort      */
     SDM_KERNEL_KINDS = 8
 } sdm_kernel_kind;
 

@@ -241,7 +241,8 @@ def sdm_norm_gate(y, *, gate=None, gamma=None, eps: float = 1e-6, act: str = "si
     return o
 
 
-KERNEL_KINDS = ("state_init", "select", "scan_seq", "scan_slot", "norm_gate", "decode")
+KERNEL_KINDS = ("state_init", "select", "scan_seq", "scan_slot", "norm_gate", "decode",
+                "slot_sort")
 
 
 def sdm_profile_enable(on: bool = True):

@@ -10,6 +10,7 @@
 #include "decode.cuh"
 #include "norm_init.cuh"
 #include "scan_seq.cuh"
+#include "scan_slot.cuh"
 #include "select.cuh"
 
 using namespace sdm;
@@ -120,10 +121,26 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 
 struct WsLayout {
   int ldw, ldr;
-  size_t off_idx_w, off_wt_w, off_idx_r, off_wt_r, total;
+  size_t off_idx_w, off_wt_w, off_idx_r, off_wt_r;
+  // slot engine
+  int chunk, n_chunks, ntiles;
+  long long events;
+  size_t off_k0, off_k1, off_v0, off_v1, off_hist, off_tot, off_offs;
+  size_t total;
 };
 
-WsLayout ws_layout(const sdm_shape& s) {
+// Tokens per chunk of the slot engine: the y rows (fp32) and v rows of one chunk of every
+// (sequence, head) should fit in about a quarter of the L2.
+int slot_chunk_tokens(const sdm_shape& s) {
+  const size_t per_token = (size_t)s.B * s.H * s.d_v * (4 + (s.in_dtype == SDM_BF16 ? 2 : 4));
+  size_t c = ((size_t)32 << 20) / (per_token ? per_token : 1);
+  size_t p = 1;
+  while (p * 2 <= c) p *= 2;
+  if (p > (size_t)s.T) p = s.T > 0 ? (size_t)s.T : 1;
+  return (int)p;
+}
+
+WsLayout ws_layout(const sdm_shape& s, int engine) {
   WsLayout L;
   L.ldw = (int)round_up((size_t)s.W, 4);
   L.ldr = (int)round_up((size_t)s.R, 4);
@@ -133,7 +150,47 @@ WsLayout ws_layout(const sdm_shape& s) {
   L.off_idx_r = round_up(L.off_wt_w + rows * L.ldw * 4, WS_ALIGN);
   L.off_wt_r = round_up(L.off_idx_r + rows * L.ldr * 4, WS_ALIGN);
   L.total = round_up(L.off_wt_r + rows * L.ldr * 4, WS_ALIGN);
+  L.chunk = slot_chunk_tokens(s);
+  L.n_chunks = s.T > 0 ? (s.T + L.chunk - 1) / L.chunk : 0;
+  L.events = (long long)rows * (s.W + s.R);
+  L.ntiles = (int)((L.events + RS_TILE - 1) / RS_TILE);
+  L.off_k0 = L.off_k1 = L.off_v0 = L.off_v1 = L.off_hist = L.off_tot = L.off_offs = 0;
+  if (engine == SDM_ENGINE_SLOT) {
+    const size_t E = (size_t)L.events;
+    L.off_k0 = L.total;
+    L.off_k1 = round_up(L.off_k0 + E * 4, WS_ALIGN);
+    L.off_v0 = round_up(L.off_k1 + E * 4, WS_ALIGN);
+    L.off_v1 = round_up(L.off_v0 + E * 8, WS_ALIGN);
+    L.off_hist = round_up(L.off_v1 + E * 8, WS_ALIGN);
+    L.off_tot = round_up(L.off_hist + (size_t)RS_BINS * L.ntiles * 4, WS_ALIGN);
+    L.off_offs = round_up(L.off_tot + RS_BINS * 4, WS_ALIGN);
+    L.total = round_up(L.off_offs + ((size_t)L.n_chunks + 1) * 4, WS_ALIGN);
+  }
   return L;
+}
+
+// The slot engine needs every event key below 2^32 - 1 and the event count below 2^32.
+bool slot_engine_fits(const sdm_shape& s) {
+  const WsLayout L = ws_layout(s, SDM_ENGINE_SEQ);
+  const unsigned long long keys =
+      (unsigned long long)L.n_chunks * s.B * s.H * (unsigned long long)s.S1 * s.S2;
+  return keys < 0xffffffffull && (unsigned long long)L.events < 0xffffffffull &&
+         s.T < (1 << 24);
+}
+
+// Engine of an AUTO request: the sequential engine needs enough (sequence, head, column
+// slice) units to fill the GPU; below that the slot engine, whose parallelism is the
+// number of distinct slots touched, does better.
+int pick_engine(const sdm_shape& s, int requested, int sms) {
+  const char* env = getenv("SDM_ENGINE");
+  if (requested == SDM_ENGINE_AUTO && env) {
+    if (!strcmp(env, "seq")) requested = SDM_ENGINE_SEQ;
+    if (!strcmp(env, "slot")) requested = SDM_ENGINE_SLOT;
+  }
+  if (requested != SDM_ENGINE_AUTO) return requested;
+  if (!slot_engine_fits(s)) return SDM_ENGINE_SEQ;
+  const long long units = (long long)s.B * s.H * (s.d_v / 32 > 0 ? s.d_v / 32 : 1);
+  return (units < 2LL * sms && s.d_v >= 128) ? SDM_ENGINE_SLOT : SDM_ENGINE_SEQ;
 }
 
 // Selection of one or two jobs over `rows` score rows.
@@ -250,6 +307,103 @@ sdm_status launch_state_init(const float* M0, float* M, const sdm_shape& s, cuda
   return SDM_OK;
 }
 
+template <int NQ, int G>
+sdm_status launch_slot_chunks(const SlotArgs& a, int n_chunks, const DeviceInfo* di,
+                              cudaStream_t st) {
+  int per_sm = 0;
+  SDM_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, slot_chunk_kernel<NQ, G>,
+                                                             SLOT_THREADS, 0));
+  const int grid = di->sms * (per_sm > 0 ? per_sm : 1);
+  for (int c = 0; c < n_chunks; ++c) {
+    slot_chunk_kernel<NQ, G><<<grid, SLOT_THREADS, 0, st>>>(a, c);
+    SDM_CUDA_TRY(cudaGetLastError());
+  }
+  return SDM_OK;
+}
+
+// Steps 2-3 with the slot-parallel engine: events, radix sort, chunk offsets, then one
+// launch per time chunk.
+sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
+                       const float* alpha, const float* beta, const void* v, float* M, float* y,
+                       const DeviceInfo* di, cudaStream_t st) {
+  uint32_t* k0 = reinterpret_cast<uint32_t*>(w + WL.off_k0);
+  uint32_t* k1 = reinterpret_cast<uint32_t*>(w + WL.off_k1);
+  uint2* v0 = reinterpret_cast<uint2*>(w + WL.off_v0);
+  uint2* v1 = reinterpret_cast<uint2*>(w + WL.off_v1);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(w + WL.off_hist);
+  uint32_t* tot = reinterpret_cast<uint32_t*>(w + WL.off_tot);
+  uint32_t* offs = reinterpret_cast<uint32_t*>(w + WL.off_offs);
+  const long long E = WL.events;
+  const int N = s.S1 * s.S2;
+  {
+    ProfScope ps(SDM_KERNEL_SLOT_SORT, st);
+    EventArgs ea;
+    ea.idx_w = reinterpret_cast<const int32_t*>(w + WL.off_idx_w);
+    ea.wt_w = reinterpret_cast<const float*>(w + WL.off_wt_w);
+    ea.idx_r = reinterpret_cast<const int32_t*>(w + WL.off_idx_r);
+    ea.wt_r = reinterpret_cast<const float*>(w + WL.off_wt_r);
+    ea.keys = k0;
+    ea.vals = v0;
+    ea.y = y;
+    ea.B = s.B;
+    ea.T = s.T;
+    ea.H = s.H;
+    ea.N = N;
+    ea.W = s.W;
+    ea.R = s.R;
+    ea.ldw = WL.ldw;
+    ea.ldr = WL.ldr;
+    ea.d_v = s.d_v;
+    ea.chunk = WL.chunk;
+    long long blocks = (E + 255) / 256;
+    if (blocks > (long long)di->sms * 16) blocks = (long long)di->sms * 16;
+    slot_events_kernel<<<(unsigned)blocks, 256, 0, st>>>(ea);
+    SDM_CUDA_TRY(cudaGetLastError());
+    // LSD radix sort over the bits the keys use
+    const unsigned long long maxkey =
+        (unsigned long long)WL.n_chunks * s.B * s.H * (unsigned long long)N - 1ull;
+    int bits = 0;
+    while (bits < 32 && (maxkey >> bits) != 0ull) ++bits;
+    for (int shift = 0; shift < bits; shift += 8) {
+      radix_hist_kernel<<<WL.ntiles, RS_THREADS, 0, st>>>(k0, E, shift, hist, WL.ntiles);
+      radix_scan_kernel<<<RS_BINS, 1024, 0, st>>>(hist, WL.ntiles, tot);
+      radix_scatter_kernel<<<WL.ntiles, RS_THREADS, 0, st>>>(k0, v0, k1, v1, E, shift, hist, tot,
+                                                            WL.ntiles);
+      SDM_CUDA_TRY(cudaGetLastError());
+      uint32_t* tk = k0;
+      k0 = k1;
+      k1 = tk;
+      uint2* tv = v0;
+      v0 = v1;
+      v1 = tv;
+    }
+    slot_chunk_offsets_kernel<<<(WL.n_chunks + 1 + 127) / 128, 128, 0, st>>>(
+        k0, E, WL.n_chunks, (uint32_t)((unsigned long long)s.B * s.H * N), offs);
+    SDM_CUDA_TRY(cudaGetLastError());
+  }
+  SlotArgs a;
+  a.keys = k0;
+  a.vals = v0;
+  a.offs = offs;
+  a.alpha = alpha;
+  a.beta = beta;
+  a.v = v;
+  a.M = M;
+  a.y = y;
+  a.B = s.B;
+  a.T = s.T;
+  a.H = s.H;
+  a.N = N;
+  a.d_v = s.d_v;
+  a.v_bf16 = s.in_dtype == SDM_BF16;
+  ProfScope ps(SDM_KERNEL_SCAN_SLOT, st);
+  const int d4 = s.d_v / 4;
+  if (d4 <= 32) return launch_slot_chunks<1, 8>(a, WL.n_chunks, di, st);
+  if (d4 <= 64) return launch_slot_chunks<2, 8>(a, WL.n_chunks, di, st);
+  if (d4 <= 128) return launch_slot_chunks<4, 4>(a, WL.n_chunks, di, st);
+  return launch_slot_chunks<8, 2>(a, WL.n_chunks, di, st);
+}
+
 bool act_ok(int act) { return act >= SDM_GATE_SILU && act <= SDM_GATE_IDENTITY; }
 
 }  // namespace
@@ -271,7 +425,10 @@ const char* sdm_status_string(sdm_status status) {
 size_t sdm_workspace_size(sdm_shape shape, int32_t engine) {
   if (!shape_ok(shape, true)) return 0;
   if (engine < SDM_ENGINE_AUTO || engine > SDM_ENGINE_SLOT) return 0;
-  return ws_layout(shape).total;
+  if (engine == SDM_ENGINE_SLOT && !slot_engine_fits(shape)) return 0;
+  // AUTO may pick either engine: size for the larger
+  if (engine == SDM_ENGINE_AUTO && slot_engine_fits(shape)) engine = SDM_ENGINE_SLOT;
+  return ws_layout(shape, engine).total;
 }
 
 sdm_status sdm_select(const void* halves, sdm_shape shape, int32_t K, int32_t* idx, float* wt,
@@ -339,14 +496,18 @@ sdm_status sdm_scan_forward(const void* kp, const void* qp, const void* v, const
     const void* ptrs[] = {kp, qp, v, alpha, beta, y, gate, gamma, o, sel_out};
     for (const void* p : ptrs)
       if (p && !aligned16(p)) return SDM_ERR_INVALID_ARG;
-    const WsLayout WL = ws_layout(s);
-    if (!ws || ws_bytes < WL.total || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN) != 0)
+    if (engine == SDM_ENGINE_SLOT && !slot_engine_fits(s)) return SDM_ERR_UNSUPPORTED;
+    const size_t need = sdm_workspace_size(s, engine);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN) != 0)
       return SDM_ERR_INVALID_ARG;
   }
-  if (engine == SDM_ENGINE_SLOT) return SDM_ERR_UNSUPPORTED;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   sdm_status rc;
+  DeviceInfo* di;
+  rc = device_info(&di);
+  if (rc != SDM_OK) return rc;
+  engine = pick_engine(s, engine, di->sms);
   if (init == SDM_INIT_FROM_M0) {
     ProfScope ps(SDM_KERNEL_STATE_INIT, st);
     rc = launch_state_init(M0, M, s, st);
@@ -354,7 +515,7 @@ sdm_status sdm_scan_forward(const void* kp, const void* qp, const void* v, const
   }
   if (s.T == 0) return SDM_OK;
 
-  const WsLayout WL = ws_layout(s);
+  const WsLayout WL = ws_layout(s, engine);
   unsigned char* w = static_cast<unsigned char*>(ws);
   int32_t* idx_w = reinterpret_cast<int32_t*>(w + WL.off_idx_w);
   float* wt_w = reinterpret_cast<float*>(w + WL.off_wt_w);
@@ -376,6 +537,16 @@ sdm_status sdm_scan_forward(const void* kp, const void* qp, const void* v, const
     SDM_CUDA_TRY(cudaMemcpy2DAsync(sel_out + (size_t)rows * s.W, (size_t)s.R * 4, idx_r,
                                    (size_t)WL.ldr * 4, (size_t)s.R * 4, (size_t)rows,
                                    cudaMemcpyDeviceToDevice, st));
+  }
+
+  if (engine == SDM_ENGINE_SLOT) {
+    rc = launch_slot(s, WL, w, alpha, beta, v, M, y, di, st);
+    if (rc != SDM_OK) return rc;
+    if (o) {
+      ProfScope ps(SDM_KERNEL_NORM_GATE, st);
+      rc = launch_norm_gate(y, gate, bf16, gamma, eps, act, rows, s.d_v, o, st);
+    }
+    return rc;
   }
 
   SeqArgs a;

@@ -116,11 +116,15 @@ def device_inputs(wl, **kw):
     return {k: t.to(DEV) for k, t in sdm_synth.make_inputs(wl, **kw).items()}
 
 
+ENGINES = ["seq", "slot"]
+
+
+@pytest.mark.parametrize("engine", ENGINES)
 @pytest.mark.parametrize("act", ["silu", "sigmoid", "identity"])
-def test_scan_tiny_full(sdm, act):
+def test_scan_tiny_full(sdm, act, engine):
     wl = sdm_synth.WORKLOADS["tiny"]
     g = device_inputs(wl, with_gamma=True)
-    out, M = run_scan(sdm, wl, g, gamma=g["gamma"], act=act)
+    out, M = run_scan(sdm, wl, g, gamma=g["gamma"], act=act, engine=engine)
     ref = full_check(wl, g, out, M, gamma=g["gamma"], act=act)
     # rows never written keep M0 bit for bit
     untouched = np.setdiff1d(np.arange(wl.N), ref["idx_w"].ravel())
@@ -128,10 +132,11 @@ def test_scan_tiny_full(sdm, act):
     assert (host(M[0, 0])[untouched].tobytes() == host(g["M0"][0])[untouched].tobytes())
 
 
-def test_scan_small_full(sdm):
+@pytest.mark.parametrize("engine", ENGINES)
+def test_scan_small_full(sdm, engine):
     wl = sdm_synth.WORKLOADS["small"]
     g = device_inputs(wl)
-    out, M = run_scan(sdm, wl, g)
+    out, M = run_scan(sdm, wl, g, engine=engine)
     full_check(wl, g, out, M)
 
 
@@ -143,10 +148,11 @@ def test_scan_small_full(sdm):
     dict(B=2, H=2, T=65, S1=128, S2=128, W=128, R=128, d_v=256, in_dtype=BF16),  # K = 128
     dict(B=1, H=2, T=30, S1=8, S2=8, W=8, R=8, d_v=512, in_dtype=BF16),    # every slot hit
 ])
-def test_scan_edge_shapes(sdm, kw):
+@pytest.mark.parametrize("engine", ENGINES)
+def test_scan_edge_shapes(sdm, kw, engine):
     wl = sdm_synth.WORKLOADS["tiny"].replace(**kw, seed=99 + kw["T"])
     g = device_inputs(wl, with_gamma=True)
-    out, M = run_scan(sdm, wl, g, gamma=g["gamma"])
+    out, M = run_scan(sdm, wl, g, gamma=g["gamma"], engine=engine)
     full_check(wl, g, out, M, gamma=g["gamma"])
 
 
@@ -160,29 +166,32 @@ def test_scan_without_gate_or_output(sdm):
     assert torch.equal(out2["y"], out["y"]) and torch.equal(M2, M)
 
 
-def test_scan_all_scores_equal(sdm):
+@pytest.mark.parametrize("engine", ENGINES)
+def test_scan_all_scores_equal(sdm, engine):
     """Every token selects the same slots (all sums tie): each token's rows were written
-    by every token before it, so the rows come from forwarding, never from the gather."""
+    by every token before it (the sequential engine forwards them from shared memory;
+    the slot engine sees one long segment per slot)."""
     wl = sdm_synth.WORKLOADS["tiny"].replace(B=1, H=2, T=70, S1=32, S2=32, W=16, R=16,
                                             d_v=64, in_dtype=BF16, seed=7)
     g = device_inputs(wl)
     g["kp"].zero_()
     g["qp"].zero_()
     g["qp"][..., 0] = 1.0
-    out, M = run_scan(sdm, wl, g)
+    out, M = run_scan(sdm, wl, g, engine=engine)
     full_check(wl, g, out, M)
 
 
-def test_scan_continue_equals_one_pass(sdm):
+@pytest.mark.parametrize("engine", ENGINES)
+def test_scan_continue_equals_one_pass(sdm, engine):
     wl = sdm_synth.WORKLOADS["small"].replace(B=1, T=300, seed=11)
     g = device_inputs(wl)
-    out, M = run_scan(sdm, wl, g)
+    out, M = run_scan(sdm, wl, g, engine=engine)
     T1 = 113
     first = {k: (t[:, :T1].contiguous() if k not in ("M0",) else t) for k, t in g.items()}
     second = {k: (t[:, T1:].contiguous() if k not in ("M0",) else t) for k, t in g.items()}
     w1, w2 = wl.replace(T=T1), wl.replace(T=wl.T - T1)
-    o1, M1 = run_scan(sdm, w1, first)
-    o2, M1 = run_scan(sdm, w2, second, init="continue", M=M1)
+    o1, M1 = run_scan(sdm, w1, first, engine=engine)
+    o2, M1 = run_scan(sdm, w2, second, init="continue", M=M1, engine=engine)
     assert_close(host(torch.cat([o1["y"], o2["y"]], 1)), host(out["y"]), "y split", atol=1e-6,
                  rtol=1e-5)
     assert_close(host(M1), host(M), "M split", atol=1e-6, rtol=1e-5)
@@ -199,11 +208,12 @@ def test_scan_zero_tokens_only_initialises(sdm):
     assert torch.equal(M, g["M0"].expand_as(M))
 
 
-def test_scan_layer1p4b_sampled(sdm):
+@pytest.mark.parametrize("engine", ["auto"] + ENGINES)
+def test_scan_layer1p4b_sampled(sdm, engine):
     """The 1.4B-like layer at full size, launched as the benchmark launches it."""
     wl = sdm_synth.WORKLOADS["layer1p4b"]
     g = device_inputs(wl)
-    out, M = run_scan(sdm, wl, g)
+    out, M = run_scan(sdm, wl, g, engine=engine)
     rng = np.random.default_rng(1)
     for (b, h) in [(0, 0), (3, 7), (2, 5)]:
         toks = [0, 1, 2, wl.T - 1] + list(rng.integers(0, wl.T, 12))
@@ -215,11 +225,12 @@ def test_scan_layer1p4b_sampled(sdm):
         assert torch.equal(M[b, h, ut], g["M0"][h, ut])
 
 
-def test_scan_long_skew_sampled(sdm):
+@pytest.mark.parametrize("engine", ["auto"] + ENGINES)
+def test_scan_long_skew_sampled(sdm, engine):
     """The long skewed prefill at full size (hot slots written thousands of times)."""
     wl = sdm_synth.WORKLOADS["long_skew"]
     g = device_inputs(wl)
-    out, M = run_scan(sdm, wl, g)
+    out, M = run_scan(sdm, wl, g, engine=engine)
     rng = np.random.default_rng(2)
     for (b, h) in [(0, 1)]:
         toks = [0, 1, wl.T // 2, wl.T - 1] + list(rng.integers(0, wl.T, 12))

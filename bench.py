@@ -183,12 +183,15 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
-def timed(fn, steps: int, warmup: int, dist: Dist, stream):
+def timed(fn, steps: int, warmup: int, dist: Dist, stream, after_warmup=None):
     """Runs fn warmup times untimed, then times exactly `steps` calls with CUDA events on
-    `stream`, bracketed by barrier + synchronize.  Returns max-over-ranks seconds."""
+    `stream`, bracketed by barrier + synchronize.  Returns max-over-ranks seconds.
+    after_warmup() runs between the two (e.g. to start per-kernel timing)."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
+    if after_warmup is not None:
+        after_warmup()
     dist.barrier()
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
@@ -222,9 +225,15 @@ def bench_prefill(args, dist: Dist, dev):
                              R=wl.R, S1=wl.S1, M0=g["M0"], init="m0", gate=g["gate"], y=y,
                              o=o, ws=ws, stream=stream)
 
-    sdm.sdm_profile_enable(True)
+    marks = {}
+
+    def start_timing():
+        sdm.sdm_profile_enable(True)
+        marks["launches"] = sdm.sdm_launch_count()
+
     with ClockSampler(dev.index) as clk:
-        secs = timed(step, args.steps, args.warmup, dist, stream)
+        secs = timed(step, args.steps, args.warmup, dist, stream, after_warmup=start_timing)
+    launched = sdm.sdm_launch_count() - marks["launches"]
     prof = sdm.sdm_profile_read()
     sdm.sdm_profile_enable(False)
     if sdm.sdm_get_device_status() != 0:
@@ -232,7 +241,7 @@ def bench_prefill(args, dist: Dist, dev):
 
     th = wl.B * wl.T * wl.H
     value = weak_scaling_value(th * args.steps, secs, dist.world)
-    # per-kernel averages over warm-up and timed launches (events on the launching stream)
+    # per-kernel averages over the timed launches (events on the launching stream)
     launches = {k: n for k, (ms, n) in prof.items() if n}
     avg_ms = {k: ms / n for k, (ms, n) in prof.items() if n}
     scan_kind = "scan_slot" if prof["scan_slot"][1] else "scan_seq"
@@ -246,7 +255,7 @@ def bench_prefill(args, dist: Dist, dev):
         "clocks": clk.report(),
         "kernels_avg_ms": avg_ms,
         "kernels_share": {k: avg_ms[k] / sum(avg_ms.values()) for k in avg_ms},
-        "gpu_launches": sum(launches.values()) * args.steps // (args.steps + args.warmup),
+        "gpu_launches": int(launched),
         "roofline": {
             "kernel": f"seq_scan_kernel" if scan_kind == "scan_seq" else "slot_scan_kernel",
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -305,8 +314,8 @@ def bench_decode(args, dist: Dist, dev):
                                 R=wl.R, S1=wl.S1, gate=s["gate"], y=y, o=o, stream=stream)
 
     reps = max(1, args.steps // 2)
-    sdm.sdm_profile_enable(True)
-    secs = timed(run_all, reps, 1, dist, stream)
+    secs = timed(run_all, reps, 1, dist, stream,
+                 after_warmup=lambda: sdm.sdm_profile_enable(True))
     prof = sdm.sdm_profile_read()
     sdm.sdm_profile_enable(False)
     ms_k, n_k = prof["decode"]

@@ -167,6 +167,9 @@ sdm_status sdm_profile_enable(int32_t on);
  * number of launches (launches[SDM_KERNEL_KINDS]); then forgets them. */
 sdm_status sdm_profile_read(double *ms, int64_t *launches);
 
+/* Number of kernels this library has launched in this process, on every device. */
+uint64_t sdm_launch_count(void);
+
 /* Synchronises `stream`, then reads and clears the calling device's status word:
  * SDM_OK, SDM_ERR_DEVICE_CHECK (an index outside [0, N) reached a kernel) or
  * SDM_ERR_TIMEOUT (a bounded wait expired).  SDM_ERR_CUDA if the synchronisation fails. */

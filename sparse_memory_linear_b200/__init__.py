@@ -17,6 +17,7 @@ from ._binding import (  # noqa: F401
     library_path,
     sdm_decode_step,
     sdm_get_device_status,
+    sdm_launch_count,
     sdm_norm_gate,
     sdm_profile_enable,
     sdm_profile_read,

@@ -58,6 +58,7 @@ def library():
         "sdm_status_string": ([I], ctypes.c_char_p),
         "sdm_profile_enable": ([I], I),
         "sdm_profile_read": ([P, P], I),
+        "sdm_launch_count": ([], ctypes.c_uint64),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -257,6 +258,11 @@ def sdm_profile_read() -> dict:
     _check(library().sdm_profile_read(ctypes.cast(ms, ctypes.c_void_p),
                                       ctypes.cast(n, ctypes.c_void_p)), "sdm_profile_read")
     return {k: (ms[i], n[i]) for i, k in enumerate(KERNEL_KINDS)}
+
+
+def sdm_launch_count() -> int:
+    """Kernels launched by the library in this process so far."""
+    return int(library().sdm_launch_count())
 
 
 def sdm_get_device_status(stream=None) -> int:

@@ -249,54 +249,102 @@ __device__ __forceinline__ void load_v(const void* v, size_t off, bool bf16, int
   }
 }
 
-// One chunk: warps walk tiles of 32 sorted events; a warp handles every slot segment that
-// starts in its tile, to the segment's end.
-// G write events have their v rows loaded together (G * NQ float4 registers).
-template <int NQ, int G>
+// Per-warp shared memory of slot_chunk_kernel: a ring of PF state rows (128*NQ floats each)
+// and the segment heads of one span of events.
+constexpr int SLOT_SPAN = 256;
+
+__host__ __device__ constexpr inline size_t slot_warp_smem(int NQ, int PF) {
+  return (size_t)PF * 128 * NQ * 4 + (size_t)SLOT_SPAN * 4;
+}
+
+// One chunk.  Warps take spans of SLOT_SPAN sorted events; a warp handles every slot segment
+// that starts in its span, to the segment's end.  It first lists the span's segment heads,
+// then streams the segments' state rows into a ring of PF shared-memory rows with cp.async,
+// PF - 1 segments ahead of the one it applies, so that every warp keeps several HBM row
+// reads in flight.  G write events have their v rows (L2 resident) loaded together.
+template <int NQ, int G, int PF>
 __global__ void __launch_bounds__(SLOT_THREADS) slot_chunk_kernel(SlotArgs a, int chunk) {
+  extern __shared__ __align__(16) unsigned char smem[];
   const uint32_t e0 = a.offs[chunk], e1 = a.offs[chunk + 1];
-  const int lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gw = (blockIdx.x * SLOT_THREADS + threadIdx.x) >> 5;
   const int nw = (gridDim.x * SLOT_THREADS) >> 5;
   const int d4 = a.d_v / 4;
   const bool bf16 = a.v_bf16 != 0;
+  const unsigned lt = lanemask_lt();
   const uint32_t per_g = static_cast<uint32_t>(a.N);
+  float* ring = reinterpret_cast<float*>(smem + (size_t)warp * slot_warp_smem(NQ, PF));
+  uint32_t* heads = reinterpret_cast<uint32_t*>(ring + (size_t)PF * 128 * NQ);
 
-  for (uint32_t tile = e0 + 32u * gw; tile < e1; tile += 32u * nw) {
-    const uint32_t ei = tile + lane;
-    const uint32_t k = ei < e1 ? a.keys[ei] : EV_SENTINEL;
-    uint32_t kprev = __shfl_up_sync(FULL_MASK, k, 1);
-    if (lane == 0) kprev = tile > e0 ? a.keys[tile - 1] : EV_SENTINEL;
-    unsigned heads = __ballot_sync(FULL_MASK, ei < e1 && k != kprev);
-    while (heads) {
-      const int hl = __ffs(heads) - 1;
-      heads &= heads - 1;
-      const uint32_t K = __shfl_sync(FULL_MASK, k, hl);
+  auto row_of = [&](uint32_t K) -> float* {
+    const uint32_t g = K / per_g;
+    const uint32_t slot = K - g * per_g;
+    const uint32_t h = g % a.H;
+    const uint32_t b = (g / a.H) % a.B;
+    return a.M + (((size_t)b * a.H + h) * a.N + slot) * a.d_v;
+  };
+
+  for (uint32_t span = e0 + (uint32_t)SLOT_SPAN * gw; span < e1; span += (uint32_t)SLOT_SPAN * nw) {
+    const uint32_t span_end = min(e1, span + (uint32_t)SLOT_SPAN);
+    // segment heads of the span, in event order
+    int nh = 0;
+    for (uint32_t tile = span; tile < span_end; tile += 32) {
+      const uint32_t ei = tile + lane;
+      const uint32_t k = ei < span_end ? a.keys[ei] : EV_SENTINEL;
+      uint32_t kprev = __shfl_up_sync(FULL_MASK, k, 1);
+      if (lane == 0) kprev = tile > e0 ? a.keys[tile - 1] : EV_SENTINEL;
+      const bool head = ei < span_end && k != kprev;
+      const unsigned hm = __ballot_sync(FULL_MASK, head);
+      if (head) heads[nh + __popc(hm & lt)] = ei;
+      nh += __popc(hm);
+    }
+    __syncwarp();
+
+    auto issue = [&](int i) {
+      if (i < nh) {
+        const float* src = row_of(a.keys[heads[i]]);
+        float* dst = ring + (size_t)(i % PF) * 128 * NQ;
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          const int c = lane + 32 * q;
+          if (c < d4) cp_async16(dst + 4 * c, src + 4 * c);
+        }
+      }
+      cp_async_commit();
+    };
+#pragma unroll
+    for (int i = 0; i < PF - 1; ++i) issue(i);
+
+    for (int si = 0; si < nh; ++si) {
+      issue(si + PF - 1);
+      cp_async_wait<PF - 1>();
+      __syncwarp();
+      const uint32_t hpos = heads[si];
+      const uint32_t K = a.keys[hpos];
       const uint32_t g = K / per_g;
-      const int slot = static_cast<int>(K - g * per_g);
       const int h = static_cast<int>(g % a.H);
       const int b = static_cast<int>((g / a.H) % a.B);
-      float* row = a.M + (((size_t)b * a.H + h) * a.N + slot) * a.d_v;
+      float* row = row_of(K);
+      const float* slot_row = ring + (size_t)(si % PF) * 128 * NQ;
       float4 m[NQ];
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
         const int c = lane + 32 * q;
-        if (c < d4) m[q] = reinterpret_cast<const float4*>(row)[c];
+        if (c < d4) m[q] = reinterpret_cast<const float4*>(slot_row)[c];
       }
       bool dirty = false;
-      uint32_t e = tile + hl;
+      uint32_t e = hpos;
       while (true) {
         // next batch of up to 32 events of this slot
         const uint32_t ej = e + lane;
         const uint32_t kj = ej < e1 ? a.keys[ej] : EV_SENTINEL;
         const unsigned match = __ballot_sync(FULL_MASK, kj == K);
         const int cnt = match == FULL_MASK ? 32 : __ffs(~match) - 1;
-        uint2 pv = make_uint2(0u, 0u);
         float ca = 0.f, cb = 0.f;
         size_t rowoff = 0;
         int kind = 1;
         if (lane < cnt) {
-          pv = a.vals[ej];
+          const uint2 pv = a.vals[ej];
           const int t = static_cast<int>(pv.x >> 8);
           kind = (pv.x >> 7) & 1;
           const size_t r = ((size_t)b * a.T + t) * a.H + h;
@@ -315,18 +363,18 @@ __global__ void __launch_bounds__(SLOT_THREADS) slot_chunk_kernel(SlotArgs a, in
           float4 vv[G][NQ];
 #pragma unroll
           for (int i = 0; i < G; ++i) {
-            const int src = i0 + i;
-            const int kd = __shfl_sync(FULL_MASK, kind, src & 31);
-            const size_t ro = __shfl_sync(FULL_MASK, rowoff, src & 31);
+            const int src = (i0 + i) & 31;
+            const int kd = __shfl_sync(FULL_MASK, kind, src);
+            const size_t ro = __shfl_sync(FULL_MASK, rowoff, src);
             if (i < ng && kd == 0) load_v<NQ>(a.v, ro, bf16, lane, d4, vv[i]);
           }
 #pragma unroll
           for (int i = 0; i < G; ++i) {
-            const int src = i0 + i;
-            const int kd = __shfl_sync(FULL_MASK, kind, src & 31);
-            const size_t ro = __shfl_sync(FULL_MASK, rowoff, src & 31);
-            const float A = __shfl_sync(FULL_MASK, ca, src & 31);
-            const float Bc = __shfl_sync(FULL_MASK, cb, src & 31);
+            const int src = (i0 + i) & 31;
+            const int kd = __shfl_sync(FULL_MASK, kind, src);
+            const size_t ro = __shfl_sync(FULL_MASK, rowoff, src);
+            const float A = __shfl_sync(FULL_MASK, ca, src);
+            const float Bc = __shfl_sync(FULL_MASK, cb, src);
             if (i < ng) {
               if (kd == 0) {
 #pragma unroll
@@ -360,7 +408,10 @@ __global__ void __launch_bounds__(SLOT_THREADS) slot_chunk_kernel(SlotArgs a, in
           if (c < d4) reinterpret_cast<float4*>(row)[c] = m[q];
         }
       }
+      __syncwarp();  // the ring slot is refilled by the next iteration's issue()
     }
+    cp_async_wait<0>();
+    __syncwarp();
   }
 }
 

@@ -3,6 +3,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -12,12 +13,18 @@
 #include "scan_seq.cuh"
 #include "scan_slot.cuh"
 #include "select.cuh"
+#include "select_fast.cuh"
 
 using namespace sdm;
 
 namespace {
 
 constexpr int MAX_DEVICES = 64;
+
+// decode_kernel instantiations, cheapest first: (halves class R8, K class, float4 columns
+// per lane).  R8 == 0 is the general selection.
+#define SDM_DEC_VARIANTS(X) \
+  X(1, 32, 1) X(2, 64, 1) X(4, 64, 2) X(4, 128, 8) X(0, 128, 8)
 constexpr size_t WS_ALIGN = 256;
 
 #define SDM_CUDA_TRY(expr)                       \
@@ -27,6 +34,9 @@ constexpr size_t WS_ALIGN = 256;
       return SDM_ERR_CUDA;                       \
     }                                            \
   } while (0)
+
+// Kernels launched by this library in this process (all devices).
+std::atomic<unsigned long long> g_launches{0};
 
 struct DeviceInfo {
   int sms = 0;
@@ -49,12 +59,25 @@ sdm_status device_info(DeviceInfo** out) {
                                         cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
     const int m = d.max_smem_optin;
     SDM_CUDA_TRY(cudaFuncSetAttribute(sel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, m));
-    SDM_CUDA_TRY(cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+#define SDM_FAST_ATTR(R8, KC) \
+  SDM_CUDA_TRY(cudaFuncSetAttribute(sel_fast_kernel<R8, KC>, cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+    SDM_FAST_ATTR(1, 32) SDM_FAST_ATTR(1, 64) SDM_FAST_ATTR(1, 128)
+    SDM_FAST_ATTR(2, 32) SDM_FAST_ATTR(2, 64) SDM_FAST_ATTR(2, 128)
+    SDM_FAST_ATTR(4, 32) SDM_FAST_ATTR(4, 64) SDM_FAST_ATTR(4, 128)
+#undef SDM_FAST_ATTR
+#define SDM_DEC_ATTR(R8, KC, NQ) \
+  SDM_CUDA_TRY(cudaFuncSetAttribute(decode_kernel<R8, KC, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+    SDM_DEC_VARIANTS(SDM_DEC_ATTR)
+#undef SDM_DEC_ATTR
 #define SDM_SEQ_ATTR(CW, D) \
   SDM_CUDA_TRY(cudaFuncSetAttribute(seq_scan_kernel<CW, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, m));
     SDM_SEQ_ATTR(4, 4) SDM_SEQ_ATTR(4, 8) SDM_SEQ_ATTR(8, 4) SDM_SEQ_ATTR(8, 8)
     SDM_SEQ_ATTR(16, 4) SDM_SEQ_ATTR(16, 8) SDM_SEQ_ATTR(32, 4) SDM_SEQ_ATTR(32, 8)
 #undef SDM_SEQ_ATTR
+#define SDM_SLOT_ATTR(NQ, G, PF) \
+  SDM_CUDA_TRY(cudaFuncSetAttribute(slot_chunk_kernel<NQ, G, PF>, cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+    SDM_SLOT_ATTR(1, 8, 8) SDM_SLOT_ATTR(2, 4, 8) SDM_SLOT_ATTR(4, 4, 4) SDM_SLOT_ATTR(8, 2, 2)
+#undef SDM_SLOT_ATTR
     d.attrs_set = true;
   }
   *out = &d;
@@ -193,6 +216,47 @@ int pick_engine(const sdm_shape& s, int requested, int sms) {
   return (units < 2LL * sms && s.d_v >= 128) ? SDM_ENGINE_SLOT : SDM_ENGINE_SEQ;
 }
 
+int env_int(const char* name, int dflt) {
+  const char* v = getenv(name);
+  return v ? atoi(v) : dflt;
+}
+
+template <int R8, int KC>
+sdm_status launch_select_fast_t(const SelJob& j0, const SelJob* j1, long long rows, int S1, int S2,
+                                const DeviceInfo* di, cudaStream_t st) {
+  const int K1 = j1 ? j1->K : j0.K;
+  int warps = 8;
+  size_t smem = sel_fast_smem_bytes(S1, S2, j0.K, K1, warps);
+  if (smem > (size_t)di->max_smem_optin) return SDM_ERR_UNSUPPORTED;
+  int per_sm = 0;
+  SDM_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sel_fast_kernel<R8, KC>,
+                                                             warps * 32, smem));
+  if (per_sm < 1) return SDM_ERR_UNSUPPORTED;
+  const long long total_rows = rows * (j1 ? 2 : 1);
+  long long grid = (long long)di->sms * per_sm;
+  const long long need = (total_rows + warps - 1) / warps;
+  if (grid > need) grid = need;
+  sel_fast_kernel<R8, KC><<<(unsigned)grid, warps * 32, smem, st>>>(j0, j1 ? *j1 : j0, rows,
+                                                                    j1 ? 2 : 1, S1, S2);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  SDM_CUDA_TRY(cudaGetLastError());
+  return SDM_OK;
+}
+
+sdm_status launch_select_fast(const SelJob& j0, const SelJob* j1, long long rows, int S1, int S2,
+                              const DeviceInfo* di, cudaStream_t st) {
+  const int K1 = j1 ? j1->K : j0.K;
+  const int r8 = fast_r8(S1, S2);
+  const int kc = fast_kc(j0.K > K1 ? j0.K : K1);
+#define SDM_FAST_CASE(R8, KC) \
+  if (r8 == R8 && kc == KC) return launch_select_fast_t<R8, KC>(j0, j1, rows, S1, S2, di, st);
+  SDM_FAST_CASE(1, 32) SDM_FAST_CASE(1, 64) SDM_FAST_CASE(1, 128)
+  SDM_FAST_CASE(2, 32) SDM_FAST_CASE(2, 64) SDM_FAST_CASE(2, 128)
+  SDM_FAST_CASE(4, 32) SDM_FAST_CASE(4, 64) SDM_FAST_CASE(4, 128)
+#undef SDM_FAST_CASE
+  return SDM_ERR_UNSUPPORTED;
+}
+
 // Selection of one or two jobs over `rows` score rows.
 sdm_status launch_select(const SelJob& j0, const SelJob* j1, long long rows, int S1, int S2,
                          int bf16, cudaStream_t st) {
@@ -201,6 +265,9 @@ sdm_status launch_select(const SelJob& j0, const SelJob* j1, long long rows, int
   if (rc != SDM_OK) return rc;
   if (rows == 0) return SDM_OK;
   const int K1 = j1 ? j1->K : j0.K;
+  const int kmax_all = j0.K > K1 ? j0.K : K1;
+  if (fast_select_ok(bf16, S1, S2, kmax_all) && env_int("SDM_SELECT_SLOW", 0) == 0)
+    return launch_select_fast(j0, j1, rows, S1, S2, di, st);
   int warps = 8;
   size_t smem = sel_smem_bytes(S1, S2, j0.K, K1, warps);
   while (warps > 1 && smem > (size_t)di->max_smem_optin / 2) {
@@ -218,18 +285,15 @@ sdm_status launch_select(const SelJob& j0, const SelJob* j1, long long rows, int
   const int kmax = j0.K > K1 ? j0.K : K1;
   sel_kernel<<<(unsigned)grid, warps * 32, smem, st>>>(j0, j1 ? *j1 : j0, rows, j1 ? 2 : 1, S1,
                                                        S2, bf16, kmax);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   SDM_CUDA_TRY(cudaGetLastError());
   return SDM_OK;
-}
-
-int env_int(const char* name, int dflt) {
-  const char* v = getenv(name);
-  return v ? atoi(v) : dflt;
 }
 
 template <int CW, int D>
 sdm_status launch_seq_t(const SeqArgs& a, int grid, size_t smem, cudaStream_t st) {
   seq_scan_kernel<CW, D><<<grid, SEQ_THREADS, smem, st>>>(a);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   SDM_CUDA_TRY(cudaGetLastError());
   return SDM_OK;
 }
@@ -287,6 +351,7 @@ sdm_status launch_norm_gate(const float* y, const void* gate, int gate_bf16, con
   if (blocks > cap) blocks = cap;
   norm_gate_kernel<<<(unsigned)blocks, 256, 0, st>>>(y, gate, gate_bf16, gamma, eps, act, rows,
                                                      d_v, o);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   SDM_CUDA_TRY(cudaGetLastError());
   return SDM_OK;
 }
@@ -303,19 +368,22 @@ sdm_status launch_state_init(const float* M0, float* M, const sdm_shape& s, cuda
   state_init_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(M0),
                                                       reinterpret_cast<float4*>(M), s.B, s.H,
                                                       per_head4);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   SDM_CUDA_TRY(cudaGetLastError());
   return SDM_OK;
 }
 
-template <int NQ, int G>
+template <int NQ, int G, int PF>
 sdm_status launch_slot_chunks(const SlotArgs& a, int n_chunks, const DeviceInfo* di,
                               cudaStream_t st) {
+  const size_t smem = (SLOT_THREADS / 32) * slot_warp_smem(NQ, PF);
   int per_sm = 0;
-  SDM_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, slot_chunk_kernel<NQ, G>,
-                                                             SLOT_THREADS, 0));
+  SDM_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+      &per_sm, slot_chunk_kernel<NQ, G, PF>, SLOT_THREADS, smem));
   const int grid = di->sms * (per_sm > 0 ? per_sm : 1);
   for (int c = 0; c < n_chunks; ++c) {
-    slot_chunk_kernel<NQ, G><<<grid, SLOT_THREADS, 0, st>>>(a, c);
+    slot_chunk_kernel<NQ, G, PF><<<grid, SLOT_THREADS, smem, st>>>(a, c);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
     SDM_CUDA_TRY(cudaGetLastError());
   }
   return SDM_OK;
@@ -358,6 +426,7 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
     long long blocks = (E + 255) / 256;
     if (blocks > (long long)di->sms * 16) blocks = (long long)di->sms * 16;
     slot_events_kernel<<<(unsigned)blocks, 256, 0, st>>>(ea);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
     SDM_CUDA_TRY(cudaGetLastError());
     // LSD radix sort over the bits the keys use
     const unsigned long long maxkey =
@@ -366,9 +435,12 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
     while (bits < 32 && (maxkey >> bits) != 0ull) ++bits;
     for (int shift = 0; shift < bits; shift += 8) {
       radix_hist_kernel<<<WL.ntiles, RS_THREADS, 0, st>>>(k0, E, shift, hist, WL.ntiles);
+      g_launches.fetch_add(1, std::memory_order_relaxed);
       radix_scan_kernel<<<RS_BINS, 1024, 0, st>>>(hist, WL.ntiles, tot);
+      g_launches.fetch_add(1, std::memory_order_relaxed);
       radix_scatter_kernel<<<WL.ntiles, RS_THREADS, 0, st>>>(k0, v0, k1, v1, E, shift, hist, tot,
                                                             WL.ntiles);
+      g_launches.fetch_add(1, std::memory_order_relaxed);
       SDM_CUDA_TRY(cudaGetLastError());
       uint32_t* tk = k0;
       k0 = k1;
@@ -379,6 +451,7 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
     }
     slot_chunk_offsets_kernel<<<(WL.n_chunks + 1 + 127) / 128, 128, 0, st>>>(
         k0, E, WL.n_chunks, (uint32_t)((unsigned long long)s.B * s.H * N), offs);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
     SDM_CUDA_TRY(cudaGetLastError());
   }
   SlotArgs a;
@@ -398,10 +471,10 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
   a.v_bf16 = s.in_dtype == SDM_BF16;
   ProfScope ps(SDM_KERNEL_SCAN_SLOT, st);
   const int d4 = s.d_v / 4;
-  if (d4 <= 32) return launch_slot_chunks<1, 8>(a, WL.n_chunks, di, st);
-  if (d4 <= 64) return launch_slot_chunks<2, 8>(a, WL.n_chunks, di, st);
-  if (d4 <= 128) return launch_slot_chunks<4, 4>(a, WL.n_chunks, di, st);
-  return launch_slot_chunks<8, 2>(a, WL.n_chunks, di, st);
+  if (d4 <= 32) return launch_slot_chunks<1, 8, 8>(a, WL.n_chunks, di, st);
+  if (d4 <= 64) return launch_slot_chunks<2, 4, 8>(a, WL.n_chunks, di, st);
+  if (d4 <= 128) return launch_slot_chunks<4, 4, 4>(a, WL.n_chunks, di, st);
+  return launch_slot_chunks<8, 2, 2>(a, WL.n_chunks, di, st);
 }
 
 bool act_ok(int act) { return act >= SDM_GATE_SILU && act <= SDM_GATE_IDENTITY; }
@@ -598,7 +671,21 @@ sdm_status sdm_decode_step(const void* kp, const void* qp, const void* v, const 
   DeviceInfo* di;
   sdm_status rc = device_info(&di);
   if (rc != SDM_OK) return rc;
-  const DecLayout L = dec_layout(s.S1, s.S2, s.W, s.R, s.d_v);
+  const bool fast = fast_select_ok(s.in_dtype == SDM_BF16, s.S1, s.S2, s.W > s.R ? s.W : s.R);
+  const int need_r8 = fast ? fast_r8(s.S1, s.S2) : 0;
+  const int need_kc = fast_kc(s.W > s.R ? s.W : s.R);
+  const int need_nq = (s.d_v / 4 + 31) / 32;
+  int v_r8 = -1, v_kc = 0;
+#define SDM_DEC_PICK(R8, KC, NQ)                                                   \
+  if (v_r8 < 0 && (fast ? (R8 >= need_r8 && R8 > 0) : R8 == 0) && KC >= need_kc && \
+      NQ >= need_nq) {                                                              \
+    v_r8 = R8;                                                                      \
+    v_kc = KC;                                                                      \
+  }
+  SDM_DEC_VARIANTS(SDM_DEC_PICK)
+#undef SDM_DEC_PICK
+  if (v_r8 < 0) return SDM_ERR_UNSUPPORTED;
+  const DecLayout L = dec_layout(s.S1, s.S2, s.W, s.R, s.d_v, v_r8 > 0, v_kc);
   if (L.total > (size_t)di->max_smem_optin) return SDM_ERR_UNSUPPORTED;
   DecodeArgs a;
   a.kp = kp;
@@ -623,7 +710,17 @@ sdm_status sdm_decode_step(const void* kp, const void* qp, const void* v, const 
   a.d_v = s.d_v;
   a.in_bf16 = s.in_dtype == SDM_BF16;
   ProfScope ps(SDM_KERNEL_DECODE, static_cast<cudaStream_t>(stream));
-  decode_kernel<<<a.BH, DEC_THREADS, L.total, static_cast<cudaStream_t>(stream)>>>(a);
+  bool launched = false;
+#define SDM_DEC_LAUNCH(R8, KC, NQ)                                                        \
+  if (!launched && (fast ? (R8 >= need_r8 && R8 > 0) : R8 == 0) && KC >= need_kc &&        \
+      NQ >= need_nq) {                                                                     \
+    decode_kernel<R8, KC, NQ><<<a.BH, DEC_THREADS, L.total, static_cast<cudaStream_t>(stream)>>>(a); \
+    g_launches.fetch_add(1, std::memory_order_relaxed);                                    \
+    launched = true;                                                                       \
+  }
+  SDM_DEC_VARIANTS(SDM_DEC_LAUNCH)
+#undef SDM_DEC_LAUNCH
+  if (!launched) return SDM_ERR_UNSUPPORTED;
   SDM_CUDA_TRY(cudaGetLastError());
   return SDM_OK;
 }
@@ -637,6 +734,8 @@ sdm_status sdm_get_device_status(void* stream) {
   if (v & STATUS_BAD_INDEX) return SDM_ERR_DEVICE_CHECK;
   return SDM_OK;
 }
+
+uint64_t sdm_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 sdm_status sdm_profile_enable(int32_t on) {
   std::vector<ProfRec> drop;

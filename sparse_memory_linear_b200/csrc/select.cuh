@@ -25,13 +25,13 @@
 namespace sdm {
 
 // Number of rank pairs (r1, r2) with (r1 + 1) * (r2 + 1) <= K.
-__host__ __device__ inline int cand_count(int K) {
+__host__ __device__ constexpr inline int cand_count(int K) {
   int c = 0;
   for (int r = 1; r <= K; ++r) c += K / r;
   return c;
 }
 
-__host__ __device__ inline int pow2_at_least(int x) {
+__host__ __device__ constexpr inline int pow2_at_least(int x) {
   int p = 1;
   while (p < x) p <<= 1;
   return p;

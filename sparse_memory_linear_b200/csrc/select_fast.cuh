@@ -1,0 +1,404 @@
+// select_fast.cuh -- register-resident product-key selection for bf16 score halves of up to
+// 1024 values and K <= 128 (the selection of select.cuh, same order and same result).
+//
+// Method: "Sparse Delta Memory: Scaling the State of Linear RNNs through Sparsity"
+// (paper.rainbus.top summary), method step 1; ai-paper-analysis.pages.dev SDM write-up,
+// 步骤 1.  Per half, per warp:
+//   1. 16-byte loads; lane l holds elements r*256 + 8l + i as 16-bit order keys;
+//   2. every lane keeps its P = ceil(K/32) largest keys; the K-th largest key T lies between
+//      the smallest and the largest of the lanes' P-th largest keys (each lane then has at
+//      least P keys >= the smallest, and fewer than 32(P-1) < K keys exceed the largest);
+//   3. keys inside that bracket are compacted to shared memory in index order, T is found by
+//      binary search on counts, and the top K are the keys > T plus the lowest-index ties;
+//   4. a register bitonic sort (shuffles) orders them: (key desc, index asc).
+// Candidates: the rank pairs with (r1+1)(r2+1) <= K; their K-th largest sum is at least
+// max_p A[p-1] + B[ceil(K/p)-1] (p*ceil(K/p) >= K pairs reach that sum), which brackets the
+// same binary search; equal sums at the threshold take the lowest flat slot indices.
+#pragma once
+
+#include "select.cuh"
+
+namespace sdm {
+
+// 16-bit order key of a bf16 score from its raw bits; -0 and +0 share one key, and every
+// non-NaN value has a key >= 1.
+__device__ __forceinline__ uint32_t bf16_key16(uint32_t h) {
+  h &= 0xffffu;
+  if ((h & 0x7fffu) == 0u) h = 0u;
+  return (h & 0x8000u) ? (~h & 0xffffu) : (h | 0x8000u);
+}
+
+__device__ __forceinline__ float key16_value(uint32_t k) {
+  const uint32_t h = (k & 0x8000u) ? (k & 0x7fffu) : (~k & 0xffffu);
+  return __uint_as_float(h << 16);
+}
+
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(FULL_MASK, v, o);
+    if (lane >= o) v += t;
+  }
+  return v;
+}
+
+// Descending bitonic sort of 32*NPL values held NPL per lane (position q*32 + lane).
+template <typename V, int NPL>
+__device__ __forceinline__ void bitonic_desc_reg(V (&v)[NPL], int lane) {
+  constexpr int P2 = 32 * NPL;
+#pragma unroll
+  for (int size = 2; size <= P2; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride >= 32) {
+        const int qs = stride >> 5;
+#pragma unroll
+        for (int q = 0; q < NPL; ++q) {
+          if ((q & qs) == 0) {
+            const int q2 = q | qs;
+            const int p = q * 32 + lane;
+            const bool desc = (p & size) == 0;
+            const V a = v[q], b = v[q2];
+            const bool sw = desc ? (a < b) : (a > b);
+            v[q] = sw ? b : a;
+            v[q2] = sw ? a : b;
+          }
+        }
+      } else {
+        const bool lower = (lane & stride) == 0;
+#pragma unroll
+        for (int q = 0; q < NPL; ++q) {
+          const int p = q * 32 + lane;
+          const bool desc = (p & size) == 0;
+          const V o = __shfl_xor_sync(FULL_MASK, v[q], stride);
+          const bool take_max = lower == desc;
+          v[q] = take_max ? (v[q] > o ? v[q] : o) : (v[q] < o ? v[q] : o);
+        }
+      }
+    }
+  }
+}
+
+// Shared scratch of one warp of the fast path.
+struct FastScratch {
+  uint32_t* surv;   // [max(S1, S2)] bracket survivors of one half (composites)
+  uint32_t* a;      // [KMAX] first half: sorted composites key16 << 16 | (0xffff - idx)
+  uint32_t* b;      // [KMAX] second half
+  uint64_t* cbuf;   // [cand_count(KMAX)] candidate survivors
+  uint32_t* stage;  // [KMAX] unsorted winners of a half (u32) / of the candidates (u64)
+};
+
+__host__ __device__ inline size_t fast_scratch_bytes(int S1, int S2, int K) {
+  const int smax = S1 > S2 ? S1 : S2;
+  return ((size_t)smax * 4 + 15) / 16 * 16 + 2 * (size_t)KMAX * 4 +
+         (size_t)cand_count(K) * 8 + (size_t)KMAX * 8;
+}
+
+__device__ inline FastScratch carve_fast_scratch(unsigned char* p, int S1, int S2, int K) {
+  FastScratch s;
+  const int smax = S1 > S2 ? S1 : S2;
+  s.surv = reinterpret_cast<uint32_t*>(p);
+  p += ((size_t)smax * 4 + 15) / 16 * 16;
+  s.a = reinterpret_cast<uint32_t*>(p);
+  p += KMAX * 4;
+  s.b = reinterpret_cast<uint32_t*>(p);
+  p += KMAX * 4;
+  s.cbuf = reinterpret_cast<uint64_t*>(p);
+  p += (size_t)cand_count(K) * 8;
+  s.stage = reinterpret_cast<uint32_t*>(p);
+  return s;
+}
+
+// Top-K of one bf16 half of S values (S <= 256 * R8), written sorted to out[0..K).
+template <int R8, int KC>
+__device__ __forceinline__ void half_topk_bf16(const __nv_bfloat16* src, int S, int K, int lane,
+                                               uint32_t* surv, uint32_t* stage, uint32_t* out) {
+  constexpr int P = KC / 32;  // enough per-lane leaders for any K <= KC
+  const unsigned lt = lanemask_lt();
+  uint32_t k[R8][8];
+  const bool vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
+  const uint16_t* raw16 = reinterpret_cast<const uint16_t*>(src);
+#pragma unroll
+  for (int r = 0; r < R8; ++r) {
+    const int e0 = r * 256 + lane * 8;
+    if (vec && e0 + 8 <= S) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(src + e0);
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        k[r][2 * j] = bf16_key16(w[j]);
+        k[r][2 * j + 1] = bf16_key16(w[j] >> 16);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) k[r][i] = (e0 + i < S) ? bf16_key16(raw16[e0 + i]) : 0u;
+    }
+  }
+  // per-lane P largest keys (descending)
+  uint32_t t[P];
+#pragma unroll
+  for (int q = 0; q < P; ++q) t[q] = 0u;
+#pragma unroll
+  for (int r = 0; r < R8; ++r) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      uint32_t x = k[r][i];
+#pragma unroll
+      for (int q = 0; q < P; ++q) {
+        const uint32_t hi = max(t[q], x);
+        x = min(t[q], x);
+        t[q] = hi;
+      }
+    }
+  }
+  const int pe = (K + 31) / 32;  // leaders that bracket the K-th key
+  uint32_t lead = t[0];
+#pragma unroll
+  for (int q = 1; q < P; ++q)
+    if (q == pe - 1) lead = t[q];
+  const uint32_t lo = max(__reduce_min_sync(FULL_MASK, lead), 1u);
+  const uint32_t hi = __reduce_max_sync(FULL_MASK, lead);
+  // bracket survivors, index order, as composites
+  int base = 0;
+#pragma unroll
+  for (int r = 0; r < R8; ++r) {
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c += k[r][i] >= lo ? 1 : 0;
+    const int incl = warp_incl_scan(c, lane);
+    int pos = base + incl - c;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (k[r][i] >= lo) surv[pos++] = (k[r][i] << 16) | (0xffffu - (uint32_t)(r * 256 + lane * 8 + i));
+    }
+    base += __shfl_sync(FULL_MASK, incl, 31);
+  }
+  __syncwarp();
+  const int ns = base;
+  auto count_ge = [&](uint32_t x) {
+    int c = 0;
+    for (int s = lane; s < ns; s += 32) c += (surv[s] >> 16) >= x ? 1 : 0;
+    return __reduce_add_sync(FULL_MASK, c);
+  };
+  uint32_t a = lo, b = hi + 1u;
+  while (b - a > 1u) {
+    const uint32_t m = (a + b) >> 1;
+    if (count_ge(m) >= K) a = m;
+    else b = m;
+  }
+  const uint32_t T = a;
+  const int need = K - count_ge(T + 1u);
+  int tb = 0, ob = 0;
+  for (int s0 = 0; s0 < ns; s0 += 32) {
+    const int s = s0 + lane;
+    const uint32_t c = s < ns ? surv[s] : 0u;
+    const uint32_t key = c >> 16;
+    const bool tie = s < ns && key == T;
+    const bool gt = s < ns && key > T;
+    const unsigned tm = __ballot_sync(FULL_MASK, tie);
+    const bool take = gt || (tie && tb + __popc(tm & lt) < need);
+    const unsigned sm = __ballot_sync(FULL_MASK, take);
+    if (take) stage[ob + __popc(sm & lt)] = c;
+    ob += __popc(sm);
+    tb += __popc(tm);
+  }
+  __syncwarp();
+  constexpr int NPL = KC / 32;
+  uint32_t v[NPL];
+#pragma unroll
+  for (int q = 0; q < NPL; ++q) {
+    const int p = q * 32 + lane;
+    v[q] = p < K ? stage[p] : 0u;
+  }
+  bitonic_desc_reg<uint32_t, NPL>(v, lane);
+#pragma unroll
+  for (int q = 0; q < NPL; ++q) {
+    const int p = q * 32 + lane;
+    if (p < K) out[p] = v[q];
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ float comp16_value(uint32_t c) { return key16_value(c >> 16); }
+__device__ __forceinline__ int comp16_index(uint32_t c) { return (int)(0xffffu - (c & 0xffffu)); }
+
+// Top-K of the rank-pair candidate sums of two sorted halves A, B (composites), written as
+// slot indices and softmax weights in selection order.
+template <int KC>
+__device__ __forceinline__ void cand_topk_bf16(const uint32_t* A, const uint32_t* B, int K,
+                                               int S2, const uint16_t* ctab, int lane,
+                                               uint64_t* cbuf, uint64_t* stage,
+                                               int32_t* out_idx, float* out_wt) {
+  constexpr int CPL = (cand_count(KC) + 31) / 32;
+  const unsigned lt = lanemask_lt();
+  const int C = cand_count(K);
+  uint32_t ck[CPL];
+  uint32_t cf[CPL];
+#pragma unroll
+  for (int q = 0; q < CPL; ++q) {
+    const int c = lane + 32 * q;
+    ck[q] = 0u;
+    cf[q] = 0u;
+    if (c < C) {
+      const int e = ctab[c];
+      const uint32_t ca = A[e >> 7], cb = B[e & 127];
+      const float s = __fadd_rn(comp16_value(ca), comp16_value(cb));
+      ck[q] = score_key(s);
+      cf[q] = (uint32_t)(comp16_index(ca) * S2 + comp16_index(cb));
+    }
+  }
+  // bracket of the K-th largest sum
+  uint32_t lo = 0u;
+  for (int p = lane + 1; p <= K; p += 32) {
+    const int q = (K + p - 1) / p;
+    lo = max(lo, score_key(__fadd_rn(comp16_value(A[p - 1]), comp16_value(B[q - 1]))));
+  }
+  lo = max(__reduce_max_sync(FULL_MASK, lo), 1u);
+  const uint32_t hi = score_key(__fadd_rn(comp16_value(A[0]), comp16_value(B[0])));
+  // survivors
+  int cnt = 0;
+#pragma unroll
+  for (int q = 0; q < CPL; ++q) cnt += ck[q] >= lo ? 1 : 0;
+  const int incl = warp_incl_scan(cnt, lane);
+  int pos = incl - cnt;
+#pragma unroll
+  for (int q = 0; q < CPL; ++q) {
+    if (ck[q] >= lo) cbuf[pos++] = (static_cast<uint64_t>(ck[q]) << 32) | (0xffffffffu - cf[q]);
+  }
+  const int ns = __shfl_sync(FULL_MASK, incl, 31);
+  __syncwarp();
+  auto count_ge = [&](uint32_t x) {
+    int c = 0;
+    for (int s = lane; s < ns; s += 32) c += static_cast<uint32_t>(cbuf[s] >> 32) >= x ? 1 : 0;
+    return __reduce_add_sync(FULL_MASK, c);
+  };
+  uint32_t a = lo, b = hi + 1u;
+  if (hi == 0xffffffffu) b = hi;  // unreachable for non-NaN scores; keeps b > a well defined
+  while (b - a > 1u) {
+    const uint32_t m = a + ((b - a) >> 1);
+    if (count_ge(m) >= K) a = m;
+    else b = m;
+  }
+  const uint32_t T = a;
+  const int ngt = count_ge(T + 1u);
+  const int need = K - ngt;
+  const int nties = count_ge(T) - ngt;
+  int ob = 0;
+  for (int s0 = 0; s0 < ns; s0 += 32) {
+    const int s = s0 + lane;
+    const uint64_t c = s < ns ? cbuf[s] : 0ull;
+    const uint32_t key = static_cast<uint32_t>(c >> 32);
+    const bool take = s < ns && (key > T || (key == T && nties == need));
+    const unsigned sm = __ballot_sync(FULL_MASK, take);
+    if (take) stage[ob + __popc(sm & lt)] = c;
+    ob += __popc(sm);
+  }
+  if (nties != need) {
+    // equal sums at the threshold: the lowest flat indices (the largest composites) win
+    uint64_t floor_c = 0xffffffffffffffffull;
+    for (int r = 0; r < need; ++r) {
+      uint64_t best = 0ull;
+      for (int s = lane; s < ns; s += 32) {
+        const uint64_t c = cbuf[s];
+        if (static_cast<uint32_t>(c >> 32) == T && c < floor_c && c > best) best = c;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t t2 = __shfl_xor_sync(FULL_MASK, best, o);
+        best = t2 > best ? t2 : best;
+      }
+      if (lane == 0) stage[ob] = best;
+      floor_c = best;
+      ++ob;
+    }
+  }
+  __syncwarp();
+  constexpr int NPL = KC / 32;
+  uint64_t v[NPL];
+#pragma unroll
+  for (int q = 0; q < NPL; ++q) {
+    const int p = q * 32 + lane;
+    v[q] = p < K ? stage[p] : 0ull;
+  }
+  bitonic_desc_reg<uint64_t, NPL>(v, lane);
+  const float s0 = key_score(static_cast<uint32_t>(__shfl_sync(FULL_MASK, v[0], 0) >> 32));
+  float e[NPL];
+  float part = 0.0f;
+#pragma unroll
+  for (int q = 0; q < NPL; ++q) {
+    const int p = q * 32 + lane;
+    e[q] = p < K ? expf(key_score(static_cast<uint32_t>(v[q] >> 32)) - s0) : 0.0f;
+    part += e[q];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(FULL_MASK, part, o);
+  const float inv = 1.0f / part;
+#pragma unroll
+  for (int q = 0; q < NPL; ++q) {
+    const int p = q * 32 + lane;
+    if (p < K) {
+      out_idx[p] = static_cast<int32_t>(0xffffffffu - static_cast<uint32_t>(v[q]));
+      out_wt[p] = e[q] * inv;
+    }
+  }
+  __syncwarp();
+}
+
+// Full selection of one bf16 score row by one warp (fast path).
+template <int R8, int KC>
+__device__ __forceinline__ void select_row_fast(const __nv_bfloat16* row, int S1, int S2, int K,
+                                                const uint16_t* ctab, FastScratch& sc, int lane,
+                                                int32_t* out_idx, float* out_wt) {
+  half_topk_bf16<R8, KC>(row, S1, K, lane, sc.surv, sc.stage, sc.a);
+  half_topk_bf16<R8, KC>(row + S1, S2, K, lane, sc.surv, sc.stage, sc.b);
+  cand_topk_bf16<KC>(sc.a, sc.b, K, S2, ctab, lane, sc.cbuf,
+                     reinterpret_cast<uint64_t*>(sc.stage), out_idx, out_wt);
+}
+
+// Whether a row shape takes the fast path, and its template parameters.
+__host__ __device__ inline bool fast_select_ok(int bf16, int S1, int S2, int K) {
+  return bf16 && S1 <= 1024 && S2 <= 1024 && K <= 128;
+}
+__host__ __device__ inline int fast_r8(int S1, int S2) {
+  const int s = S1 > S2 ? S1 : S2;
+  return s <= 256 ? 1 : (s <= 512 ? 2 : 4);
+}
+__host__ __device__ inline int fast_kc(int K) { return K <= 32 ? 32 : (K <= 64 ? 64 : 128); }
+
+// Persistent fast selection kernel over rows of job0 followed by rows of job1.
+template <int R8, int KC>
+__global__ void __launch_bounds__(256) sel_fast_kernel(SelJob job0, SelJob job1, long long n_rows,
+                                                       int njobs, int S1, int S2) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int C0 = cand_count(job0.K);
+  const int C1 = njobs > 1 ? cand_count(job1.K) : 0;
+  uint16_t* tab0 = reinterpret_cast<uint16_t*>(smem);
+  uint16_t* tab1 = tab0 + ((C0 + 7) / 8) * 8;
+  unsigned char* scratch_base = reinterpret_cast<unsigned char*>(tab1 + ((C1 + 7) / 8) * 8);
+  build_cand_table(tab0, job0.K, threadIdx.x, blockDim.x);
+  if (njobs > 1) build_cand_table(tab1, job1.K, threadIdx.x, blockDim.x);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wpc = blockDim.x >> 5;
+  FastScratch sc = carve_fast_scratch(scratch_base + (size_t)warp * fast_scratch_bytes(S1, S2, KC),
+                                      S1, S2, KC);
+  const long long total = n_rows * njobs;
+  const int S = S1 + S2;
+  for (long long r = (long long)blockIdx.x * wpc + warp; r < total;
+       r += (long long)gridDim.x * wpc) {
+    const bool second = r >= n_rows;
+    const SelJob& J = second ? job1 : job0;
+    const long long row = second ? r - n_rows : r;
+    const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(J.halves) + (size_t)row * S;
+    select_row_fast<R8, KC>(src, S1, S2, J.K, second ? tab1 : tab0, sc, lane,
+                            J.idx + (size_t)row * J.ld, J.wt + (size_t)row * J.ld);
+  }
+}
+
+inline size_t sel_fast_smem_bytes(int S1, int S2, int K0, int K1, int warps) {
+  const int kc = fast_kc(K0 > K1 ? K0 : K1);
+  size_t tabs = (size_t)((cand_count(K0) + 7) / 8) * 16 + (size_t)((cand_count(K1) + 7) / 8) * 16;
+  return tabs + (size_t)warps * fast_scratch_bytes(S1, S2, kc);
+}
+
+}  // namespace sdm

@@ -52,7 +52,13 @@ def test_workspace_size(sdm):
     def r256(x):
         return (x + 255) // 256 * 256
     want = r256(rows * 8 * 4) * 2 + r256(rows * 8 * 4) * 2
-    assert sdm.sdm_workspace_size(s) == want
+    assert sdm.sdm_workspace_size(s, "seq") == want
+    # the slot engine adds double-buffered events (12 B each), the radix histogram and the
+    # chunk offsets; AUTO reserves room for either engine
+    events = rows * (6 + 8)
+    slot = sdm.sdm_workspace_size(s, "slot")
+    assert slot >= want + 2 * events * 12
+    assert sdm.sdm_workspace_size(s) == slot
     assert sdm.sdm_workspace_size(good_shape(sdm, W=40)) == 0  # W > S
     assert sdm.sdm_workspace_size(good_shape(sdm, d_v=12)) == 0  # bf16 needs d_v % 8 == 0
 

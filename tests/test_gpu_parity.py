@@ -55,6 +55,20 @@ def test_select_matches_oracle(sdm, S1, S2, K, dt):
         np.testing.assert_array_equal(idx.cpu().numpy(), bf_idx)
 
 
+@pytest.mark.parametrize("S1,S2,K", [(1024, 1024, 64), (512, 512, 64), (256, 200, 33),
+                                     (1000, 24, 17), (8, 8, 8), (128, 130, 128)])
+def test_select_fast_path_equals_general_path(sdm, S1, S2, K, monkeypatch):
+    """bf16 rows take the register-resident path; forcing the general path must give the
+    same slots bit for bit and the same weights."""
+    x = sdm_synth.draw(5 + S1 + K, 1, (300, S1 + S2), BF16).to(DEV)
+    idx_f, wt_f = sdm.sdm_select(x, K, S1=S1)
+    monkeypatch.setenv("SDM_SELECT_SLOW", "1")
+    idx_g, wt_g = sdm.sdm_select(x, K, S1=S1)
+    torch.cuda.synchronize()
+    assert torch.equal(idx_f, idx_g)
+    assert_close(wt_f.cpu().numpy(), wt_g.cpu().numpy(), "weights", atol=1e-7, rtol=1e-6)
+
+
 @pytest.mark.parametrize("dt", [F32, BF16])
 @pytest.mark.parametrize("S1,S2,K", [(8, 8, 8), (16, 12, 5), (64, 64, 64), (40, 40, 9)])
 def test_select_ties_and_signed_zeros(sdm, S1, S2, K, dt):

@@ -121,6 +121,34 @@ sdm_status sdm_scan_forward(const void *kp, const void *qp, const void *v, const
                             int32_t act, float *o, int32_t *sel_out, int32_t engine, void *ws,
                             size_t ws_bytes, sdm_shape shape, void *stream);
 
+/* Size of the fixed scratch of sdm_scan_forward_noalloc (16 MiB per device). */
+#define SDM_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * Prefill that allocates nothing (no paper counterpart: a deployment variant of
+ * sdm_scan_forward).  It is for callers that cannot allocate device memory while the pass
+ * runs: a host engine that owns all device memory in its own pool, a plugin interface
+ * without a workspace argument, or a loop that must not call the CUDA allocator once
+ * running.  The arguments and results are those of sdm_scan_forward with the sequential
+ * engine; the scratch is a fixed device array of SDM_NOALLOC_SCRATCH_BYTES that the library
+ * holds on every device that loads it, until the process exits.
+ *  - The shape's scratch, sdm_workspace_size(shape, SDM_ENGINE_SEQ), must not exceed
+ *    SDM_NOALLOC_SCRATCH_BYTES; a larger shape returns SDM_ERR_INVALID_ARG and launches
+ *    nothing (for W = R = 64 that is up to 16384 (sequence, token, head) rows per call).
+ *  - The first call on a device looks up the array's device address (once per device);
+ *    make that first call before capturing any stream into a CUDA graph.
+ *  - Every call on a device shares the one array, which keeps the last call's contents.
+ *    Nothing in it needs to start at zero (each call rewrites what it reads), but calls
+ *    that overlap on the GPU (different streams, or host threads, at the same time) race
+ *    on it: serialise them.
+ *  - Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+sdm_status sdm_scan_forward_noalloc(const void *kp, const void *qp, const void *v,
+                                    const float *alpha, const float *beta, const float *M0,
+                                    float *M, int32_t init, float *y, const void *gate,
+                                    const float *gamma, float eps, int32_t act, float *o,
+                                    int32_t *sel_out, sdm_shape shape, void *stream);
+
 /*
  * Decode: steps 1-4 for ONE token of each of B sequences and H heads, in one fused
  * launch [paper.rainbus.top summary, method steps 1-4; m.163.com article, section 八,

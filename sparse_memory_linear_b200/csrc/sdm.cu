@@ -781,3 +781,58 @@ sdm_status sdm_profile_read(double* ms, int64_t* launches) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------
+// Prefill without any allocation.
+//
+// Some callers cannot allocate device memory at the time they run the pass: a host engine
+// that hands all device memory to its own pool at start-up, a plugin interface that
+// offers no workspace argument, or a real-time loop that must not call the CUDA allocator
+// (cudaMalloc and cudaFree can synchronise the device) once it is running.  For them,
+// sdm_scan_forward_noalloc takes the scratch of the sequential engine from a fixed
+// file-scope device array instead of from a caller buffer.  The array exists once per
+// device that loads this library and stays allocated until the process exits.
+__device__ __align__(256) unsigned char g_noalloc_scratch[SDM_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[MAX_DEVICES];  // device address of g_noalloc_scratch, per device
+
+// The device address of the array on the current device.  In host code the array's name
+// is only a host-side stand-in, so the address comes from cudaGetSymbolAddress, once per
+// device, with that device current.
+sdm_status noalloc_scratch(void** out) {
+  int dev = 0;
+  SDM_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= MAX_DEVICES) return SDM_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      (void)cudaGetLastError();
+      return SDM_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SDM_OK;
+}
+}  // namespace
+
+extern "C" sdm_status sdm_scan_forward_noalloc(const void* kp, const void* qp, const void* v,
+                                               const float* alpha, const float* beta,
+                                               const float* M0, float* M, int32_t init,
+                                               float* y, const void* gate, const float* gamma,
+                                               float eps, int32_t act, float* o,
+                                               int32_t* sel_out, sdm_shape shape,
+                                               void* stream) {
+  if (!shape_ok(shape, true)) return SDM_ERR_INVALID_ARG;
+  if (sdm_workspace_size(shape, SDM_ENGINE_SEQ) > (size_t)SDM_NOALLOC_SCRATCH_BYTES)
+    return SDM_ERR_INVALID_ARG;
+  void* ws = nullptr;
+  const sdm_status rc = noalloc_scratch(&ws);
+  if (rc != SDM_OK) return rc;
+  return sdm_scan_forward(kp, qp, v, alpha, beta, M0, M, init, y, gate, gamma, eps, act, o,
+                          sel_out, SDM_ENGINE_SEQ, ws, SDM_NOALLOC_SCRATCH_BYTES, shape,
+                          stream);
+}

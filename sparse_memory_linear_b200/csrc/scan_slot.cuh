@@ -7,14 +7,19 @@
 // and a read of slot i at token t needs M[i] after the writes of tokens <= t.
 //
 // Design.  The selections of every token are turned into events (slot, token, kind,
-// weight) and sorted, stably, by (time chunk, sequence, head, slot) with an LSD radix
-// sort; events of one slot inside one chunk are then contiguous and in token order,
-// writes before reads at equal tokens.  Chunks run one after another (a slot's state
-// carries over); inside a chunk every slot is independent.  A warp takes the events of
-// one slot, loads the row once, applies the writes in registers (v rows of the chunk are
-// L2 resident), adds q * row into y for every read (y rows of the chunk are L2
-// resident), and stores the row once.  Rows hit by many tokens (skewed access) cost one
-// HBM round trip per chunk instead of one per token.
+// weight) and sorted, stably, by (time chunk, sequence, head, slot) -- bit fields of a
+// 32-bit key -- with an LSD radix sort; events of one slot inside one chunk are then
+// contiguous and in token order, writes before reads at equal tokens.  Chunks run one
+// after another (a slot's state carries over); inside a chunk every slot is independent.
+//   * A warp takes the events of one slot ("segment"): the row is loaded once (a cp.async
+//     ring keeps PF rows in flight per warp), the writes are applied in registers (the v
+//     rows of a chunk are L2 resident), every read adds q * row into y with vector atomics
+//     (the y rows of a chunk are L2 resident), and the row is stored once.
+//   * A segment of at least SLOT_LONG events (a hot slot under skewed access) is taken by a
+//     whole CTA: each warp composes the affine map of its slice of the events
+//     (s -> A s + B), the maps are chained to give every slice its exact start state, and
+//     each warp then re-walks its slice to produce the reads.
+// Rows hit by many tokens cost one HBM round trip per chunk instead of one per token.
 #pragma once
 
 #include "common.cuh"
@@ -27,6 +32,20 @@ constexpr int RS_IPT = 16;                       // items per thread
 constexpr int RS_TILE = RS_THREADS * RS_IPT;     // 4096 items per tile
 constexpr int RS_BINS = 256;
 constexpr uint32_t EV_SENTINEL = 0xffffffffu;
+constexpr int SLOT_LONG = 256;  // events of a segment taken by a whole CTA
+
+// Bit layout of an event key: chunk | sequence | head | slot (most significant first).
+struct KeyBits {
+  int nbits, hbits, bbits, cbits;
+  __host__ __device__ int total() const { return nbits + hbits + bbits + cbits; }
+  __host__ __device__ int chunk_shift() const { return nbits + hbits + bbits; }
+};
+
+__host__ __device__ inline int bits_for(long long n) {
+  int b = 0;
+  while ((1LL << b) < n) ++b;
+  return b;
+}
 
 // ---------------------------------------------------------------- event construction
 struct EventArgs {
@@ -37,17 +56,20 @@ struct EventArgs {
   uint32_t* keys;        // [rows * (W + R)]
   uint2* vals;
   float* y;              // [rows, d_v], zeroed here
-  int B, T, H, N, W, R, ldw, ldr, d_v, chunk;
+  uint32_t* counters;    // [2 * n_chunks], zeroed here
+  int B, T, H, N, W, R, ldw, ldr, d_v, chunk, n_chunks;
+  KeyBits kb;
 };
 
 // Event e = row * (W + R) + j: j < W is write j of the row, else read j - W.
-// key = ((chunk * B + b) * H + h) * N + slot; val = {t << 8 | kind << 7 | j, weight bits}.
+// val = {t << 8 | kind << 7 | j, weight bits}.
 __global__ void __launch_bounds__(256) slot_events_kernel(EventArgs a) {
   const long long rows = (long long)a.B * a.T * a.H;
   const int per = a.W + a.R;
   const long long n = rows * per;
   const long long stride = (long long)gridDim.x * blockDim.x;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += stride) {
+  const long long tid0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  for (long long e = tid0; e < n; e += stride) {
     const long long row = e / per;
     const int j = static_cast<int>(e - row * per);
     const int h = static_cast<int>(row % a.H);
@@ -62,16 +84,18 @@ __global__ void __launch_bounds__(256) slot_events_kernel(EventArgs a) {
       record_status(STATUS_BAD_INDEX);
       slot = 0;
     }
-    const int c = t / a.chunk;
-    const uint32_t g = static_cast<uint32_t>((c * a.B + b) * a.H + h);
-    a.keys[e] = g * static_cast<uint32_t>(a.N) + static_cast<uint32_t>(slot);
+    const uint32_t c = static_cast<uint32_t>(t / a.chunk);
+    const uint32_t key = (((((c << a.kb.bbits) | (uint32_t)b) << a.kb.hbits) | (uint32_t)h)
+                          << a.kb.nbits) |
+                         (uint32_t)slot;
+    a.keys[e] = key;
     a.vals[e] = make_uint2((static_cast<uint32_t>(t) << 8) | (rd ? 128u : 0u) | jj,
                            __float_as_uint(w));
   }
   const long long ny = rows * a.d_v / 4;
   float4* y4 = reinterpret_cast<float4*>(a.y);
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < ny; i += stride)
-    y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (long long i = tid0; i < ny; i += stride) y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (long long i = tid0; i < 2LL * a.n_chunks; i += stride) a.counters[i] = 0u;
 }
 
 // --------------------------------------------------------------------- radix sort
@@ -195,7 +219,7 @@ __global__ void __launch_bounds__(RS_THREADS) radix_scatter_kernel(
 
 // First event of every chunk in the sorted keys (binary search); offs[n_chunks] = n.
 __global__ void slot_chunk_offsets_kernel(const uint32_t* __restrict__ keys, long long n,
-                                          int n_chunks, uint32_t per_chunk_keys,
+                                          int n_chunks, int chunk_shift,
                                           uint32_t* __restrict__ offs) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c > n_chunks) return;
@@ -203,7 +227,7 @@ __global__ void slot_chunk_offsets_kernel(const uint32_t* __restrict__ keys, lon
     offs[c] = static_cast<uint32_t>(n);
     return;
   }
-  const unsigned long long target = (unsigned long long)c * per_chunk_keys;
+  const unsigned long long target = (unsigned long long)c << chunk_shift;
   long long lo = 0, hi = n;
   while (lo < hi) {
     const long long mid = (lo + hi) >> 1;
@@ -211,6 +235,49 @@ __global__ void slot_chunk_offsets_kernel(const uint32_t* __restrict__ keys, lon
     else hi = mid;
   }
   offs[c] = static_cast<uint32_t>(lo);
+}
+
+// Segments of at least SLOT_LONG events: listed per chunk as {first event, length}.
+__global__ void __launch_bounds__(256) slot_long_segments_kernel(
+    const uint32_t* __restrict__ keys, long long n, int chunk_shift, uint32_t* hot_count,
+    uint2* hot_list, int hot_cap) {
+  const int lane = threadIdx.x & 31;
+  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long tile = gw * 32; tile < n; tile += nw * 32) {
+    const long long e = tile + lane;
+    const uint32_t k = e < n ? keys[e] : EV_SENTINEL;
+    uint32_t kprev = __shfl_up_sync(FULL_MASK, k, 1);
+    if (lane == 0) kprev = tile > 0 ? keys[tile - 1] : EV_SENTINEL;
+    const bool head = e < n && k != kprev;
+    const bool is_long = head && e + SLOT_LONG - 1 < n && keys[e + SLOT_LONG - 1] == k;
+    unsigned lm = __ballot_sync(FULL_MASK, is_long);
+    while (lm) {
+      const int hl = __ffs(lm) - 1;
+      lm &= lm - 1;
+      const long long first = tile + hl;
+      const uint32_t K = __shfl_sync(FULL_MASK, k, hl);
+      long long end = first + SLOT_LONG;
+      while (true) {
+        const long long ej = end + lane;
+        const bool same = ej < n && keys[ej] == K;
+        const unsigned m = __ballot_sync(FULL_MASK, same);
+        if (m == FULL_MASK) {
+          end += 32;
+          continue;
+        }
+        end += __ffs(~m) - 1;
+        break;
+      }
+      if (lane == 0) {
+        const uint32_t c = K >> chunk_shift;
+        const uint32_t pos = atomicAdd(&hot_count[c], 1u);
+        if (pos < (uint32_t)hot_cap)
+          hot_list[(size_t)c * hot_cap + pos] =
+              make_uint2(static_cast<uint32_t>(first), static_cast<uint32_t>(end - first));
+      }
+    }
+  }
 }
 
 // ------------------------------------------------------------- chunk processing
@@ -223,10 +290,17 @@ struct SlotArgs {
   const void* v;         // [rows, d_v]
   float* M;              // [B*H, N, d_v]
   float* y;              // [rows, d_v]
+  const uint32_t* hot_count;  // [n_chunks]
+  const uint2* hot_list;      // [n_chunks, hot_cap]
+  uint32_t* span_next;        // [n_chunks] dynamic span queue
+  int hot_cap;
   int B, T, H, N, d_v, v_bf16;
+  KeyBits kb;
 };
 
 constexpr int SLOT_THREADS = 256;
+constexpr int SLOT_WARPS = SLOT_THREADS / 32;
+constexpr int SLOT_SPAN = 256;
 
 // Loads lane's part of a v row (NQ chunks of 4 values) as fp32.
 template <int NQ>
@@ -249,51 +323,181 @@ __device__ __forceinline__ void load_v(const void* v, size_t off, bool bf16, int
   }
 }
 
-// Per-warp shared memory of slot_chunk_kernel: a ring of PF state rows (128*NQ floats each)
-// and the segment heads of one span of events.
-constexpr int SLOT_SPAN = 256;
+// Applies the events [first, last) of one slot of sequence b, head h to the lane's part of
+// the row, m.  compose == false: writes update m, reads add q * m into y.  compose == true:
+// m starts at 0 and accumulates the affine map's additive part, A_acc its multiplicative
+// part; reads are skipped.  Returns whether any write was applied.
+template <int NQ, int G>
+__device__ __forceinline__ bool walk_events(const SlotArgs& a, uint32_t first, uint32_t last, int b,
+                                            int h, int lane, float4 (&m)[NQ], bool compose,
+                                            float& A_acc) {
+  const int d4 = a.d_v / 4;
+  const bool bf16 = a.v_bf16 != 0;
+  bool wrote = false;
+  for (uint32_t e = first; e < last; e += 32) {
+    const int cnt = static_cast<int>(min(32u, last - e));
+    uint32_t r32 = 0u;
+    float ca = 0.f, cb = 0.f;
+    if (lane < cnt) {
+      const uint2 pv = a.vals[e + lane];
+      const uint32_t t = pv.x >> 8;
+      const uint32_t kind = (pv.x >> 7) & 1u;
+      const uint32_t r = ((uint32_t)b * a.T + t) * a.H + (uint32_t)h;
+      const float w = __uint_as_float(pv.y);
+      if (kind == 0u) {
+        const float kb = a.beta[r] * w;
+        ca = a.alpha[r] * (1.0f - kb);
+        cb = kb;
+      } else {
+        ca = w;
+      }
+      r32 = r | (kind << 31);
+    }
+    for (int i0 = 0; i0 < cnt; i0 += G) {
+      float4 vv[G][NQ];
+      uint32_t rr[G];
+#pragma unroll
+      for (int i = 0; i < G; ++i) {
+        rr[i] = __shfl_sync(FULL_MASK, r32, (i0 + i) & 31);
+        if (i0 + i < cnt && (rr[i] >> 31) == 0u)
+          load_v<NQ>(a.v, (size_t)(rr[i] & 0x7fffffffu) * a.d_v, bf16, lane, d4, vv[i]);
+      }
+#pragma unroll
+      for (int i = 0; i < G; ++i) {
+        const float A = __shfl_sync(FULL_MASK, ca, (i0 + i) & 31);
+        const float Bc = __shfl_sync(FULL_MASK, cb, (i0 + i) & 31);
+        if (i0 + i < cnt) {
+          if ((rr[i] >> 31) == 0u) {
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+              m[q].x = fmaf(A, m[q].x, Bc * vv[i][q].x);
+              m[q].y = fmaf(A, m[q].y, Bc * vv[i][q].y);
+              m[q].z = fmaf(A, m[q].z, Bc * vv[i][q].z);
+              m[q].w = fmaf(A, m[q].w, Bc * vv[i][q].w);
+            }
+            A_acc *= A;
+            wrote = true;
+          } else if (!compose) {
+            float* yrow = a.y + (size_t)(rr[i] & 0x7fffffffu) * a.d_v;
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+              const int c = lane + 32 * q;
+              if (c < d4)
+                atomicAdd(reinterpret_cast<float4*>(yrow) + c,
+                          make_float4(A * m[q].x, A * m[q].y, A * m[q].z, A * m[q].w));
+            }
+          }
+        }
+      }
+    }
+  }
+  return wrote;
+}
 
 __host__ __device__ constexpr inline size_t slot_warp_smem(int NQ, int PF) {
   return (size_t)PF * 128 * NQ * 4 + (size_t)SLOT_SPAN * 4;
 }
 
-// One chunk.  Warps take spans of SLOT_SPAN sorted events; a warp handles every slot segment
-// that starts in its span, to the segment's end.  It first lists the span's segment heads,
-// then streams the segments' state rows into a ring of PF shared-memory rows with cp.async,
-// PF - 1 segments ahead of the one it applies, so that every warp keeps several HBM row
-// reads in flight.  G write events have their v rows (L2 resident) loaded together.
+// One chunk.  CTAs first take the chunk's long segments, one CTA each (see the file
+// comment); then every warp takes spans of SLOT_SPAN sorted events from a queue and handles
+// each shorter segment that starts in its span, streaming the segments' state rows through
+// a ring of PF shared-memory rows with cp.async.
 template <int NQ, int G, int PF>
 __global__ void __launch_bounds__(SLOT_THREADS) slot_chunk_kernel(SlotArgs a, int chunk) {
   extern __shared__ __align__(16) unsigned char smem[];
   const uint32_t e0 = a.offs[chunk], e1 = a.offs[chunk + 1];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int gw = (blockIdx.x * SLOT_THREADS + threadIdx.x) >> 5;
-  const int nw = (gridDim.x * SLOT_THREADS) >> 5;
   const int d4 = a.d_v / 4;
-  const bool bf16 = a.v_bf16 != 0;
   const unsigned lt = lanemask_lt();
-  const uint32_t per_g = static_cast<uint32_t>(a.N);
-  float* ring = reinterpret_cast<float*>(smem + (size_t)warp * slot_warp_smem(NQ, PF));
-  uint32_t* heads = reinterpret_cast<uint32_t*>(ring + (size_t)PF * 128 * NQ);
-
-  auto row_of = [&](uint32_t K) -> float* {
-    const uint32_t g = K / per_g;
-    const uint32_t slot = K - g * per_g;
-    const uint32_t h = g % a.H;
-    const uint32_t b = (g / a.H) % a.B;
+  const uint32_t nmask = (1u << a.kb.nbits) - 1u;
+  const uint32_t hmask = (1u << a.kb.hbits) - 1u;
+  const uint32_t bmask = (1u << a.kb.bbits) - 1u;
+  auto row_of = [&](uint32_t K, int& b, int& h) -> float* {
+    const uint32_t slot = K & nmask;
+    h = static_cast<int>((K >> a.kb.nbits) & hmask);
+    b = static_cast<int>((K >> (a.kb.nbits + a.kb.hbits)) & bmask);
     return a.M + (((size_t)b * a.H + h) * a.N + slot) * a.d_v;
   };
 
-  for (uint32_t span = e0 + (uint32_t)SLOT_SPAN * gw; span < e1; span += (uint32_t)SLOT_SPAN * nw) {
+  // ---- long segments: one CTA per segment
+  {
+    float* coefA = reinterpret_cast<float*>(smem);  // [SLOT_WARPS] (32 reserved)
+    float* coefB = coefA + 32;                      // [SLOT_WARPS][128 * NQ]
+    const uint32_t nh = min(a.hot_count[chunk], (uint32_t)a.hot_cap);
+    for (uint32_t hs = blockIdx.x; hs < nh; hs += gridDim.x) {
+      const uint2 seg = a.hot_list[(size_t)chunk * a.hot_cap + hs];
+      const uint32_t first = seg.x, n = seg.y;
+      int b, h;
+      float* row = row_of(a.keys[first], b, h);
+      const uint32_t per = (n + SLOT_WARPS - 1) / SLOT_WARPS;
+      const uint32_t s0 = first + min(n, per * warp), s1 = first + min(n, per * (warp + 1));
+      // 1. this slice's affine map s -> A s + m
+      float4 m[NQ];
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) m[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      float A = 1.0f;
+      walk_events<NQ, G>(a, s0, s1, b, h, lane, m, true, A);
+      if (lane == 0) coefA[warp] = A;
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        const int c = lane + 32 * q;
+        if (c < d4) reinterpret_cast<float4*>(coefB + warp * 128 * NQ)[c] = m[q];
+      }
+      __syncthreads();
+      // 2. start state of this slice: the row after the slices before it
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        const int c = lane + 32 * q;
+        if (c < d4) m[q] = reinterpret_cast<const float4*>(row)[c];
+      }
+      for (int k = 0; k < warp; ++k) {
+        const float Ak = coefA[k];
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          const int c = lane + 32 * q;
+          if (c < d4) {
+            const float4 Bk = reinterpret_cast<const float4*>(coefB + k * 128 * NQ)[c];
+            m[q].x = fmaf(Ak, m[q].x, Bk.x);
+            m[q].y = fmaf(Ak, m[q].y, Bk.y);
+            m[q].z = fmaf(Ak, m[q].z, Bk.z);
+            m[q].w = fmaf(Ak, m[q].w, Bk.w);
+          }
+        }
+      }
+      __syncthreads();  // every warp has read the row before the last one rewrites it
+      // 3. re-walk the slice from its exact start state: the reads, and the final row
+      float unused = 1.0f;
+      walk_events<NQ, G>(a, s0, s1, b, h, lane, m, false, unused);
+      if (warp == SLOT_WARPS - 1) {
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          const int c = lane + 32 * q;
+          if (c < d4) reinterpret_cast<float4*>(row)[c] = m[q];
+        }
+      }
+      __syncthreads();  // coefficients are reused by the next long segment
+    }
+  }
+
+  // ---- the other segments, span by span
+  float* ring = reinterpret_cast<float*>(smem + (size_t)warp * slot_warp_smem(NQ, PF));
+  uint32_t* heads = reinterpret_cast<uint32_t*>(ring + (size_t)PF * 128 * NQ);
+  while (true) {
+    uint32_t span_id = 0;
+    if (lane == 0) span_id = atomicAdd(&a.span_next[chunk], 1u);
+    span_id = __shfl_sync(FULL_MASK, span_id, 0);
+    if (span_id >= (e1 - e0 + SLOT_SPAN - 1) / SLOT_SPAN) break;
+    const uint32_t span = e0 + span_id * (uint32_t)SLOT_SPAN;
     const uint32_t span_end = min(e1, span + (uint32_t)SLOT_SPAN);
-    // segment heads of the span, in event order
+    // heads of the short segments starting in the span, in event order
     int nh = 0;
     for (uint32_t tile = span; tile < span_end; tile += 32) {
       const uint32_t ei = tile + lane;
       const uint32_t k = ei < span_end ? a.keys[ei] : EV_SENTINEL;
       uint32_t kprev = __shfl_up_sync(FULL_MASK, k, 1);
       if (lane == 0) kprev = tile > e0 ? a.keys[tile - 1] : EV_SENTINEL;
-      const bool head = ei < span_end && k != kprev;
+      bool head = ei < span_end && k != kprev;
+      if (head && ei + SLOT_LONG - 1 < e1 && a.keys[ei + SLOT_LONG - 1] == k) head = false;
       const unsigned hm = __ballot_sync(FULL_MASK, head);
       if (head) heads[nh + __popc(hm & lt)] = ei;
       nh += __popc(hm);
@@ -302,7 +506,8 @@ __global__ void __launch_bounds__(SLOT_THREADS) slot_chunk_kernel(SlotArgs a, in
 
     auto issue = [&](int i) {
       if (i < nh) {
-        const float* src = row_of(a.keys[heads[i]]);
+        int bb, hh;
+        const float* src = row_of(a.keys[heads[i]], bb, hh);
         float* dst = ring + (size_t)(i % PF) * 128 * NQ;
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
@@ -319,12 +524,22 @@ __global__ void __launch_bounds__(SLOT_THREADS) slot_chunk_kernel(SlotArgs a, in
       issue(si + PF - 1);
       cp_async_wait<PF - 1>();
       __syncwarp();
-      const uint32_t hpos = heads[si];
-      const uint32_t K = a.keys[hpos];
-      const uint32_t g = K / per_g;
-      const int h = static_cast<int>(g % a.H);
-      const int b = static_cast<int>((g / a.H) % a.B);
-      float* row = row_of(K);
+      const uint32_t first = heads[si];
+      const uint32_t K = a.keys[first];
+      int b, h;
+      float* row = row_of(K, b, h);
+      // the segment's end (it is shorter than SLOT_LONG)
+      uint32_t last = first;
+      while (true) {
+        const uint32_t ek = last + lane;
+        const unsigned m2 = __ballot_sync(FULL_MASK, ek < e1 && a.keys[ek] == K);
+        if (m2 == FULL_MASK) {
+          last += 32;
+          continue;
+        }
+        last += __ffs(~m2) - 1;
+        break;
+      }
       const float* slot_row = ring + (size_t)(si % PF) * 128 * NQ;
       float4 m[NQ];
 #pragma unroll
@@ -332,75 +547,8 @@ __global__ void __launch_bounds__(SLOT_THREADS) slot_chunk_kernel(SlotArgs a, in
         const int c = lane + 32 * q;
         if (c < d4) m[q] = reinterpret_cast<const float4*>(slot_row)[c];
       }
-      bool dirty = false;
-      uint32_t e = hpos;
-      while (true) {
-        // next batch of up to 32 events of this slot
-        const uint32_t ej = e + lane;
-        const uint32_t kj = ej < e1 ? a.keys[ej] : EV_SENTINEL;
-        const unsigned match = __ballot_sync(FULL_MASK, kj == K);
-        const int cnt = match == FULL_MASK ? 32 : __ffs(~match) - 1;
-        float ca = 0.f, cb = 0.f;
-        size_t rowoff = 0;
-        int kind = 1;
-        if (lane < cnt) {
-          const uint2 pv = a.vals[ej];
-          const int t = static_cast<int>(pv.x >> 8);
-          kind = (pv.x >> 7) & 1;
-          const size_t r = ((size_t)b * a.T + t) * a.H + h;
-          rowoff = r * a.d_v;
-          const float w = __uint_as_float(pv.y);
-          if (kind == 0) {
-            const float kb = a.beta[r] * w;
-            ca = a.alpha[r] * (1.0f - kb);
-            cb = kb;
-          } else {
-            ca = w;
-          }
-        }
-        for (int i0 = 0; i0 < cnt; i0 += G) {
-          const int ng = min(G, cnt - i0);
-          float4 vv[G][NQ];
-#pragma unroll
-          for (int i = 0; i < G; ++i) {
-            const int src = (i0 + i) & 31;
-            const int kd = __shfl_sync(FULL_MASK, kind, src);
-            const size_t ro = __shfl_sync(FULL_MASK, rowoff, src);
-            if (i < ng && kd == 0) load_v<NQ>(a.v, ro, bf16, lane, d4, vv[i]);
-          }
-#pragma unroll
-          for (int i = 0; i < G; ++i) {
-            const int src = (i0 + i) & 31;
-            const int kd = __shfl_sync(FULL_MASK, kind, src);
-            const size_t ro = __shfl_sync(FULL_MASK, rowoff, src);
-            const float A = __shfl_sync(FULL_MASK, ca, src);
-            const float Bc = __shfl_sync(FULL_MASK, cb, src);
-            if (i < ng) {
-              if (kd == 0) {
-#pragma unroll
-                for (int q = 0; q < NQ; ++q) {
-                  m[q].x = fmaf(A, m[q].x, Bc * vv[i][q].x);
-                  m[q].y = fmaf(A, m[q].y, Bc * vv[i][q].y);
-                  m[q].z = fmaf(A, m[q].z, Bc * vv[i][q].z);
-                  m[q].w = fmaf(A, m[q].w, Bc * vv[i][q].w);
-                }
-                dirty = true;
-              } else {
-#pragma unroll
-                for (int q = 0; q < NQ; ++q) {
-                  const int c = lane + 32 * q;
-                  if (c < d4) {
-                    float4* dst = reinterpret_cast<float4*>(a.y + ro) + c;
-                    atomicAdd(dst, make_float4(A * m[q].x, A * m[q].y, A * m[q].z, A * m[q].w));
-                  }
-                }
-              }
-            }
-          }
-        }
-        e += cnt;
-        if (cnt < 32) break;
-      }
+      float unused = 1.0f;
+      const bool dirty = walk_events<NQ, G>(a, first, last, b, h, lane, m, false, unused);
       if (dirty) {
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {

@@ -146,9 +146,10 @@ struct WsLayout {
   int ldw, ldr;
   size_t off_idx_w, off_wt_w, off_idx_r, off_wt_r;
   // slot engine
-  int chunk, n_chunks, ntiles;
+  int chunk, n_chunks, ntiles, hot_cap;
   long long events;
-  size_t off_k0, off_k1, off_v0, off_v1, off_hist, off_tot, off_offs;
+  KeyBits kb;
+  size_t off_k0, off_k1, off_v0, off_v1, off_hist, off_tot, off_offs, off_cnt, off_hot;
   size_t total;
 };
 
@@ -177,7 +178,14 @@ WsLayout ws_layout(const sdm_shape& s, int engine) {
   L.n_chunks = s.T > 0 ? (s.T + L.chunk - 1) / L.chunk : 0;
   L.events = (long long)rows * (s.W + s.R);
   L.ntiles = (int)((L.events + RS_TILE - 1) / RS_TILE);
+  L.kb.nbits = bits_for((long long)s.S1 * s.S2);
+  L.kb.hbits = bits_for(s.H);
+  L.kb.bbits = bits_for(s.B);
+  L.kb.cbits = bits_for(L.n_chunks > 0 ? L.n_chunks : 1);
+  const long long chunk_events = (long long)L.chunk * s.B * s.H * (s.W + s.R);
+  L.hot_cap = (int)(chunk_events / SLOT_LONG + 1);
   L.off_k0 = L.off_k1 = L.off_v0 = L.off_v1 = L.off_hist = L.off_tot = L.off_offs = 0;
+  L.off_cnt = L.off_hot = 0;
   if (engine == SDM_ENGINE_SLOT) {
     const size_t E = (size_t)L.events;
     L.off_k0 = L.total;
@@ -187,18 +195,20 @@ WsLayout ws_layout(const sdm_shape& s, int engine) {
     L.off_hist = round_up(L.off_v1 + E * 8, WS_ALIGN);
     L.off_tot = round_up(L.off_hist + (size_t)RS_BINS * L.ntiles * 4, WS_ALIGN);
     L.off_offs = round_up(L.off_tot + RS_BINS * 4, WS_ALIGN);
-    L.total = round_up(L.off_offs + ((size_t)L.n_chunks + 1) * 4, WS_ALIGN);
+    L.off_cnt = round_up(L.off_offs + ((size_t)L.n_chunks + 1) * 4, WS_ALIGN);
+    L.off_hot = round_up(L.off_cnt + (size_t)2 * L.n_chunks * 4, WS_ALIGN);
+    L.total = round_up(L.off_hot + (size_t)L.n_chunks * L.hot_cap * 8, WS_ALIGN);
   }
   return L;
 }
 
-// The slot engine needs every event key below 2^32 - 1 and the event count below 2^32.
+// The slot engine packs (chunk, sequence, head, slot) into 31 bits of a key and counts
+// events and state rows in 32 bits.
 bool slot_engine_fits(const sdm_shape& s) {
   const WsLayout L = ws_layout(s, SDM_ENGINE_SEQ);
-  const unsigned long long keys =
-      (unsigned long long)L.n_chunks * s.B * s.H * (unsigned long long)s.S1 * s.S2;
-  return keys < 0xffffffffull && (unsigned long long)L.events < 0xffffffffull &&
-         s.T < (1 << 24);
+  const long long rows = (long long)s.B * s.T * s.H;
+  return L.kb.total() <= 31 && (unsigned long long)L.events < 0xffffffffull &&
+         rows < (1LL << 31) && s.T < (1 << 24);
 }
 
 // Engine of an AUTO request: the sequential engine needs enough (sequence, head, column
@@ -376,7 +386,7 @@ sdm_status launch_state_init(const float* M0, float* M, const sdm_shape& s, cuda
 template <int NQ, int G, int PF>
 sdm_status launch_slot_chunks(const SlotArgs& a, int n_chunks, const DeviceInfo* di,
                               cudaStream_t st) {
-  const size_t smem = (SLOT_THREADS / 32) * slot_warp_smem(NQ, PF);
+  const size_t smem = SLOT_WARPS * slot_warp_smem(NQ, PF);
   int per_sm = 0;
   SDM_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
       &per_sm, slot_chunk_kernel<NQ, G, PF>, SLOT_THREADS, smem));
@@ -389,8 +399,8 @@ sdm_status launch_slot_chunks(const SlotArgs& a, int n_chunks, const DeviceInfo*
   return SDM_OK;
 }
 
-// Steps 2-3 with the slot-parallel engine: events, radix sort, chunk offsets, then one
-// launch per time chunk.
+// Steps 2-3 with the slot-parallel engine: events, radix sort, chunk offsets, long segments,
+// then one launch per time chunk.
 sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
                        const float* alpha, const float* beta, const void* v, float* M, float* y,
                        const DeviceInfo* di, cudaStream_t st) {
@@ -401,6 +411,8 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
   uint32_t* hist = reinterpret_cast<uint32_t*>(w + WL.off_hist);
   uint32_t* tot = reinterpret_cast<uint32_t*>(w + WL.off_tot);
   uint32_t* offs = reinterpret_cast<uint32_t*>(w + WL.off_offs);
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(w + WL.off_cnt);  // hot counts | span queues
+  uint2* hot = reinterpret_cast<uint2*>(w + WL.off_hot);
   const long long E = WL.events;
   const int N = s.S1 * s.S2;
   {
@@ -413,6 +425,7 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
     ea.keys = k0;
     ea.vals = v0;
     ea.y = y;
+    ea.counters = cnt;
     ea.B = s.B;
     ea.T = s.T;
     ea.H = s.H;
@@ -423,24 +436,21 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
     ea.ldr = WL.ldr;
     ea.d_v = s.d_v;
     ea.chunk = WL.chunk;
+    ea.n_chunks = WL.n_chunks;
+    ea.kb = WL.kb;
     long long blocks = (E + 255) / 256;
     if (blocks > (long long)di->sms * 16) blocks = (long long)di->sms * 16;
     slot_events_kernel<<<(unsigned)blocks, 256, 0, st>>>(ea);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     SDM_CUDA_TRY(cudaGetLastError());
-    // LSD radix sort over the bits the keys use
-    const unsigned long long maxkey =
-        (unsigned long long)WL.n_chunks * s.B * s.H * (unsigned long long)N - 1ull;
-    int bits = 0;
-    while (bits < 32 && (maxkey >> bits) != 0ull) ++bits;
+    // LSD radix sort over the key bits in use
+    const int bits = WL.kb.total();
     for (int shift = 0; shift < bits; shift += 8) {
       radix_hist_kernel<<<WL.ntiles, RS_THREADS, 0, st>>>(k0, E, shift, hist, WL.ntiles);
-      g_launches.fetch_add(1, std::memory_order_relaxed);
       radix_scan_kernel<<<RS_BINS, 1024, 0, st>>>(hist, WL.ntiles, tot);
-      g_launches.fetch_add(1, std::memory_order_relaxed);
       radix_scatter_kernel<<<WL.ntiles, RS_THREADS, 0, st>>>(k0, v0, k1, v1, E, shift, hist, tot,
                                                             WL.ntiles);
-      g_launches.fetch_add(1, std::memory_order_relaxed);
+      g_launches.fetch_add(3, std::memory_order_relaxed);
       SDM_CUDA_TRY(cudaGetLastError());
       uint32_t* tk = k0;
       k0 = k1;
@@ -450,8 +460,13 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
       v1 = tv;
     }
     slot_chunk_offsets_kernel<<<(WL.n_chunks + 1 + 127) / 128, 128, 0, st>>>(
-        k0, E, WL.n_chunks, (uint32_t)((unsigned long long)s.B * s.H * N), offs);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
+        k0, E, WL.n_chunks, WL.kb.chunk_shift(), offs);
+    long long lblocks = (E / 32 + 7) / 8;
+    if (lblocks > (long long)di->sms * 8) lblocks = (long long)di->sms * 8;
+    if (lblocks < 1) lblocks = 1;
+    slot_long_segments_kernel<<<(unsigned)lblocks, 256, 0, st>>>(k0, E, WL.kb.chunk_shift(), cnt,
+                                                                 hot, WL.hot_cap);
+    g_launches.fetch_add(2, std::memory_order_relaxed);
     SDM_CUDA_TRY(cudaGetLastError());
   }
   SlotArgs a;
@@ -463,12 +478,17 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
   a.v = v;
   a.M = M;
   a.y = y;
+  a.hot_count = cnt;
+  a.hot_list = hot;
+  a.span_next = cnt + WL.n_chunks;
+  a.hot_cap = WL.hot_cap;
   a.B = s.B;
   a.T = s.T;
   a.H = s.H;
   a.N = N;
   a.d_v = s.d_v;
   a.v_bf16 = s.in_dtype == SDM_BF16;
+  a.kb = WL.kb;
   ProfScope ps(SDM_KERNEL_SCAN_SLOT, st);
   const int d4 = s.d_v / 4;
   if (d4 <= 32) return launch_slot_chunks<1, 8, 8>(a, WL.n_chunks, di, st);

@@ -94,7 +94,7 @@ __device__ __forceinline__ void decode_select_fast(const DecodeArgs& a, const De
     FastScratch pair = carve_fast_scratch(smem + L.off_sel + warp * L.sel_stride, a.S1, a.S2, KC);
     cand_topk_bf16<KC>(pair.a, pair.b, rd ? a.R : a.W, a.S2,
                        reinterpret_cast<const uint16_t*>(smem + (rd ? L.off_tab_r : L.off_tab_w)),
-                       lane, pair.cbuf, reinterpret_cast<uint64_t*>(pair.stage),
+                       lane, pair.pv, reinterpret_cast<uint64_t*>(pair.stage),
                        rd ? idx_r : idx_w, rd ? wt_r : wt_w);
   }
 }

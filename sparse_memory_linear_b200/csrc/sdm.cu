@@ -47,6 +47,16 @@ struct DeviceInfo {
 std::mutex g_dev_mu;
 DeviceInfo g_dev[MAX_DEVICES];
 
+// Lets `kernel` use all the opt-in shared memory that its static shared memory leaves.
+template <typename Kernel>
+cudaError_t allow_max_dynamic_smem(Kernel kernel, int optin) {
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              optin - (int)fa.sharedSizeBytes);
+}
+
 sdm_status device_info(DeviceInfo** out) {
   int dev = 0;
   SDM_CUDA_TRY(cudaGetDevice(&dev));
@@ -58,25 +68,25 @@ sdm_status device_info(DeviceInfo** out) {
     SDM_CUDA_TRY(cudaDeviceGetAttribute(&d.max_smem_optin,
                                         cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
     const int m = d.max_smem_optin;
-    SDM_CUDA_TRY(cudaFuncSetAttribute(sel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+    SDM_CUDA_TRY(allow_max_dynamic_smem(sel_kernel, m));
 #define SDM_FAST_ATTR(R8, KC) \
-  SDM_CUDA_TRY(cudaFuncSetAttribute(sel_fast_kernel<R8, KC>, cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+  SDM_CUDA_TRY(allow_max_dynamic_smem(sel_fast_kernel<R8, KC>, m));
     SDM_FAST_ATTR(1, 32) SDM_FAST_ATTR(1, 64) SDM_FAST_ATTR(1, 128)
     SDM_FAST_ATTR(2, 32) SDM_FAST_ATTR(2, 64) SDM_FAST_ATTR(2, 128)
     SDM_FAST_ATTR(4, 32) SDM_FAST_ATTR(4, 64) SDM_FAST_ATTR(4, 128)
 #undef SDM_FAST_ATTR
 #define SDM_DEC_ATTR(R8, KC, NQ) \
-  SDM_CUDA_TRY(cudaFuncSetAttribute(decode_kernel<R8, KC, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+  SDM_CUDA_TRY(allow_max_dynamic_smem(decode_kernel<R8, KC, NQ>, m));
     SDM_DEC_VARIANTS(SDM_DEC_ATTR)
 #undef SDM_DEC_ATTR
 #define SDM_SEQ_ATTR(CW, D) \
-  SDM_CUDA_TRY(cudaFuncSetAttribute(seq_scan_kernel<CW, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+  SDM_CUDA_TRY(allow_max_dynamic_smem(seq_scan_kernel<CW, D>, m));
     SDM_SEQ_ATTR(4, 4) SDM_SEQ_ATTR(4, 8) SDM_SEQ_ATTR(8, 4) SDM_SEQ_ATTR(8, 8)
     SDM_SEQ_ATTR(16, 4) SDM_SEQ_ATTR(16, 8) SDM_SEQ_ATTR(32, 4) SDM_SEQ_ATTR(32, 8)
 #undef SDM_SEQ_ATTR
 #define SDM_SLOT_ATTR(NQ, G, PF) \
-  SDM_CUDA_TRY(cudaFuncSetAttribute(slot_chunk_kernel<NQ, G, PF>, cudaFuncAttributeMaxDynamicSharedMemorySize, m));
-    SDM_SLOT_ATTR(1, 8, 8) SDM_SLOT_ATTR(2, 4, 8) SDM_SLOT_ATTR(4, 4, 4) SDM_SLOT_ATTR(8, 2, 2)
+  SDM_CUDA_TRY(allow_max_dynamic_smem(slot_chunk_kernel<NQ, G, PF>, m));
+    SDM_SLOT_ATTR(1, 8, 8) SDM_SLOT_ATTR(2, 2, 8) SDM_SLOT_ATTR(4, 4, 4) SDM_SLOT_ATTR(8, 2, 2)
 #undef SDM_SLOT_ATTR
     d.attrs_set = true;
   }
@@ -492,7 +502,7 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
   ProfScope ps(SDM_KERNEL_SCAN_SLOT, st);
   const int d4 = s.d_v / 4;
   if (d4 <= 32) return launch_slot_chunks<1, 8, 8>(a, WL.n_chunks, di, st);
-  if (d4 <= 64) return launch_slot_chunks<2, 4, 8>(a, WL.n_chunks, di, st);
+  if (d4 <= 64) return launch_slot_chunks<2, 2, 8>(a, WL.n_chunks, di, st);
   if (d4 <= 128) return launch_slot_chunks<4, 4, 4>(a, WL.n_chunks, di, st);
   return launch_slot_chunks<8, 2, 2>(a, WL.n_chunks, di, st);
 }

@@ -37,14 +37,28 @@ __host__ __device__ constexpr inline int pow2_at_least(int x) {
   return p;
 }
 
-// Fills tab[0 .. cand_count(K)) with the rank pairs, packed as r1 << 7 | r2.
+// Fills tab[0 .. cand_count(K)) with the rank pairs, packed as r1 << 7 | r2: one division
+// per row, a prefix sum of the row lengths, then every row written by its own thread.  Every
+// thread of the block must call it (it synchronises the block).
 __device__ inline void build_cand_table(uint16_t* tab, int K, int tid, int nthreads) {
+  __shared__ int start[KMAX + 1];
+  for (int r = tid; r < K; r += nthreads) start[r] = K / (r + 1);
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int r = 0; r < K; ++r) {
+      const int len = start[r];
+      start[r] = run;
+      run += len;
+    }
+    start[K] = run;
+  }
+  __syncthreads();
   for (int r1 = tid; r1 < K; r1 += nthreads) {
-    int off = 0;
-    for (int r = 0; r < r1; ++r) off += K / (r + 1);
-    const int len = K / (r1 + 1);
+    const int off = start[r1], len = start[r1 + 1] - off;
     for (int r2 = 0; r2 < len; ++r2) tab[off + r2] = static_cast<uint16_t>((r1 << 7) | r2);
   }
+  __syncthreads();
 }
 
 // Shared scratch of one selecting warp.

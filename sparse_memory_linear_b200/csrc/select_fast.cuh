@@ -42,13 +42,14 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
   return v;
 }
 
-// Descending bitonic sort of 32*NPL values held NPL per lane (position q*32 + lane).
+// Descending bitonic sort of 32*NPL values held NPL per lane (position q*32 + lane).  The
+// stage loops stay rolled (small code); the per-lane element loops are unrolled.
 template <typename V, int NPL>
 __device__ __forceinline__ void bitonic_desc_reg(V (&v)[NPL], int lane) {
   constexpr int P2 = 32 * NPL;
-#pragma unroll
+#pragma unroll 1
   for (int size = 2; size <= P2; size <<= 1) {
-#pragma unroll
+#pragma unroll 1
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
       if (stride >= 32) {
         const int qs = stride >> 5;
@@ -84,14 +85,15 @@ struct FastScratch {
   uint32_t* surv;   // [max(S1, S2)] bracket survivors of one half (composites)
   uint32_t* a;      // [KMAX] first half: sorted composites key16 << 16 | (0xffff - idx)
   uint32_t* b;      // [KMAX] second half
-  uint64_t* cbuf;   // [cand_count(KMAX)] candidate survivors
+  float* pv;        // [4 * KMAX] candidate phase: half values and scaled indices
   uint32_t* stage;  // [KMAX] unsorted winners of a half (u32) / of the candidates (u64)
 };
 
 __host__ __device__ inline size_t fast_scratch_bytes(int S1, int S2, int K) {
   const int smax = S1 > S2 ? S1 : S2;
-  return ((size_t)smax * 4 + 15) / 16 * 16 + 2 * (size_t)KMAX * 4 +
-         (size_t)cand_count(K) * 8 + (size_t)KMAX * 8;
+  (void)K;
+  return ((size_t)smax * 4 + 15) / 16 * 16 + 2 * (size_t)KMAX * 4 + 4 * (size_t)KMAX * 4 +
+         (size_t)KMAX * 8;
 }
 
 __device__ inline FastScratch carve_fast_scratch(unsigned char* p, int S1, int S2, int K) {
@@ -103,8 +105,8 @@ __device__ inline FastScratch carve_fast_scratch(unsigned char* p, int S1, int S
   p += KMAX * 4;
   s.b = reinterpret_cast<uint32_t*>(p);
   p += KMAX * 4;
-  s.cbuf = reinterpret_cast<uint64_t*>(p);
-  p += (size_t)cand_count(K) * 8;
+  s.pv = reinterpret_cast<float*>(p);
+  p += 4 * (size_t)KMAX * 4;
   s.stage = reinterpret_cast<uint32_t*>(p);
   return s;
 }
@@ -112,7 +114,8 @@ __device__ inline FastScratch carve_fast_scratch(unsigned char* p, int S1, int S
 // Top-K of one bf16 half of S values (S <= 256 * R8), written sorted to out[0..K).
 template <int R8, int KC>
 __device__ __forceinline__ void half_topk_bf16(const __nv_bfloat16* src, int S, int K, int lane,
-                                               uint32_t* surv, uint32_t* stage, uint32_t* out) {
+                                               uint32_t* surv, uint32_t* stage, uint32_t* out,
+                                               int idx_base = 0) {
   constexpr int P = KC / 32;  // enough per-lane leaders for any K <= KC
   const unsigned lt = lanemask_lt();
   uint32_t k[R8][8];
@@ -169,7 +172,8 @@ __device__ __forceinline__ void half_topk_bf16(const __nv_bfloat16* src, int S, 
     int pos = base + incl - c;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      if (k[r][i] >= lo) surv[pos++] = (k[r][i] << 16) | (0xffffu - (uint32_t)(r * 256 + lane * 8 + i));
+      if (k[r][i] >= lo)
+        surv[pos++] = (k[r][i] << 16) | (0xffffu - (uint32_t)(idx_base + r * 256 + lane * 8 + i));
     }
     base += __shfl_sync(FULL_MASK, incl, 31);
   }
@@ -219,78 +223,130 @@ __device__ __forceinline__ void half_topk_bf16(const __nv_bfloat16* src, int S, 
   __syncwarp();
 }
 
+// Top-K of two sorted (descending) lists of K composites, a and b, written sorted to out:
+// the element-wise larger of a[i] and b[K-1-i] forms a bitonic sequence holding the K
+// largest, which half-cleaner stages then sort.  K <= 32*NPL.
+template <int NPL>
+__device__ __forceinline__ void merge_top_sorted(const uint32_t* a, const uint32_t* b, int K,
+                                                 int lane, uint32_t* out) {
+  constexpr int P2 = 32 * NPL;
+  uint32_t v[NPL];
+#pragma unroll
+  for (int q = 0; q < NPL; ++q) {
+    const int p = q * 32 + lane;
+    // pad to P2 with the smallest composite; b reversed within the padded length
+    const uint32_t x = p < K ? a[p] : 0u;
+    const int pr = P2 - 1 - p;
+    const uint32_t y = pr < K ? b[pr] : 0u;
+    v[q] = x > y ? x : y;
+  }
+  // the sequence is bitonic over P2 positions: sort it descending with half-cleaners
+#pragma unroll 1
+  for (int stride = P2 >> 1; stride > 0; stride >>= 1) {
+    if (stride >= 32) {
+      const int qs = stride >> 5;
+#pragma unroll
+      for (int q = 0; q < NPL; ++q) {
+        if ((q & qs) == 0) {
+          const int q2 = q | qs;
+          const uint32_t x = v[q], y = v[q2];
+          v[q] = x > y ? x : y;
+          v[q2] = x > y ? y : x;
+        }
+      }
+    } else {
+      const bool lower = (lane & stride) == 0;
+#pragma unroll
+      for (int q = 0; q < NPL; ++q) {
+        const uint32_t o = __shfl_xor_sync(FULL_MASK, v[q], stride);
+        v[q] = lower ? (v[q] > o ? v[q] : o) : (v[q] < o ? v[q] : o);
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < NPL; ++q) {
+    const int p = q * 32 + lane;
+    if (p < K) out[p] = v[q];
+  }
+  __syncwarp();
+}
+
 __device__ __forceinline__ float comp16_value(uint32_t c) { return key16_value(c >> 16); }
 __device__ __forceinline__ int comp16_index(uint32_t c) { return (int)(0xffffu - (c & 0xffffu)); }
 
 // Top-K of the rank-pair candidate sums of two sorted halves A, B (composites), written as
-// slot indices and softmax weights in selection order.
+// slot indices and softmax weights in selection order.  The candidates stay in registers;
+// sums of bf16 halves leave the low bits of their fp32 patterns zero, so the threshold
+// search runs on keys shifted right by the bits every candidate has clear.
 template <int KC>
 __device__ __forceinline__ void cand_topk_bf16(const uint32_t* A, const uint32_t* B, int K,
                                                int S2, const uint16_t* ctab, int lane,
-                                               uint64_t* cbuf, uint64_t* stage,
-                                               int32_t* out_idx, float* out_wt) {
+                                               float* pv, uint64_t* stage, int32_t* out_idx,
+                                               float* out_wt) {
   constexpr int CPL = (cand_count(KC) + 31) / 32;
   const unsigned lt = lanemask_lt();
   const int C = cand_count(K);
+  float* av = pv;                                   // [KMAX] first-half values
+  float* bv = pv + KMAX;                            // [KMAX] second-half values
+  int* ai = reinterpret_cast<int*>(pv + 2 * KMAX);  // [KMAX] first-half index * S2
+  int* bi = reinterpret_cast<int*>(pv + 3 * KMAX);  // [KMAX] second-half index
+  for (int j = lane; j < K; j += 32) {
+    av[j] = comp16_value(A[j]);
+    ai[j] = comp16_index(A[j]) * S2;
+    bv[j] = comp16_value(B[j]);
+    bi[j] = comp16_index(B[j]);
+  }
+  __syncwarp();
   uint32_t ck[CPL];
   uint32_t cf[CPL];
+  uint32_t orbits = 0u;
 #pragma unroll
   for (int q = 0; q < CPL; ++q) {
     const int c = lane + 32 * q;
-    ck[q] = 0u;
+    ck[q] = 0u;  // no candidate (every real score has a key >= 1)
     cf[q] = 0u;
     if (c < C) {
       const int e = ctab[c];
-      const uint32_t ca = A[e >> 7], cb = B[e & 127];
-      const float s = __fadd_rn(comp16_value(ca), comp16_value(cb));
+      const int r1 = e >> 7, r2 = e & 127;
+      const float s = __fadd_rn(av[r1], bv[r2]);
+      orbits |= __float_as_uint(s) & 0x7fffffffu;
       ck[q] = score_key(s);
-      cf[q] = (uint32_t)(comp16_index(ca) * S2 + comp16_index(cb));
+      cf[q] = (uint32_t)(ai[r1] + bi[r2]);
     }
   }
   // bracket of the K-th largest sum
   uint32_t lo = 0u;
   for (int p = lane + 1; p <= K; p += 32) {
     const int q = (K + p - 1) / p;
-    lo = max(lo, score_key(__fadd_rn(comp16_value(A[p - 1]), comp16_value(B[q - 1]))));
+    lo = max(lo, score_key(__fadd_rn(av[p - 1], bv[q - 1])));
   }
   lo = max(__reduce_max_sync(FULL_MASK, lo), 1u);
-  const uint32_t hi = score_key(__fadd_rn(comp16_value(A[0]), comp16_value(B[0])));
-  // survivors
-  int cnt = 0;
-#pragma unroll
-  for (int q = 0; q < CPL; ++q) cnt += ck[q] >= lo ? 1 : 0;
-  const int incl = warp_incl_scan(cnt, lane);
-  int pos = incl - cnt;
-#pragma unroll
-  for (int q = 0; q < CPL; ++q) {
-    if (ck[q] >= lo) cbuf[pos++] = (static_cast<uint64_t>(ck[q]) << 32) | (0xffffffffu - cf[q]);
-  }
-  const int ns = __shfl_sync(FULL_MASK, incl, 31);
-  __syncwarp();
+  const uint32_t hi = score_key(__fadd_rn(av[0], bv[0]));
+  orbits = __reduce_or_sync(FULL_MASK, orbits);
+  const int tz = orbits ? __ffs(orbits) - 1 : 0;
   auto count_ge = [&](uint32_t x) {
     int c = 0;
-    for (int s = lane; s < ns; s += 32) c += static_cast<uint32_t>(cbuf[s] >> 32) >= x ? 1 : 0;
+#pragma unroll
+    for (int q = 0; q < CPL; ++q) c += (ck[q] != 0u && (ck[q] >> tz) >= x) ? 1 : 0;
     return __reduce_add_sync(FULL_MASK, c);
   };
-  uint32_t a = lo, b = hi + 1u;
-  if (hi == 0xffffffffu) b = hi;  // unreachable for non-NaN scores; keeps b > a well defined
+  uint32_t a = lo >> tz, b = (hi >> tz) + 1u;
   while (b - a > 1u) {
     const uint32_t m = a + ((b - a) >> 1);
     if (count_ge(m) >= K) a = m;
     else b = m;
   }
-  const uint32_t T = a;
+  const uint32_t T = a;  // shifted key of the K-th largest sum
   const int ngt = count_ge(T + 1u);
   const int need = K - ngt;
   const int nties = count_ge(T) - ngt;
   int ob = 0;
-  for (int s0 = 0; s0 < ns; s0 += 32) {
-    const int s = s0 + lane;
-    const uint64_t c = s < ns ? cbuf[s] : 0ull;
-    const uint32_t key = static_cast<uint32_t>(c >> 32);
-    const bool take = s < ns && (key > T || (key == T && nties == need));
+#pragma unroll
+  for (int q = 0; q < CPL; ++q) {
+    const uint32_t sk = ck[q] >> tz;
+    const bool take = ck[q] != 0u && (sk > T || (sk == T && nties == need));
     const unsigned sm = __ballot_sync(FULL_MASK, take);
-    if (take) stage[ob + __popc(sm & lt)] = c;
+    if (take) stage[ob + __popc(sm & lt)] = (static_cast<uint64_t>(ck[q]) << 32) | (0xffffffffu - cf[q]);
     ob += __popc(sm);
   }
   if (nties != need) {
@@ -298,9 +354,10 @@ __device__ __forceinline__ void cand_topk_bf16(const uint32_t* A, const uint32_t
     uint64_t floor_c = 0xffffffffffffffffull;
     for (int r = 0; r < need; ++r) {
       uint64_t best = 0ull;
-      for (int s = lane; s < ns; s += 32) {
-        const uint64_t c = cbuf[s];
-        if (static_cast<uint32_t>(c >> 32) == T && c < floor_c && c > best) best = c;
+#pragma unroll
+      for (int q = 0; q < CPL; ++q) {
+        const uint64_t c = (static_cast<uint64_t>(ck[q]) << 32) | (0xffffffffu - cf[q]);
+        if (ck[q] != 0u && (ck[q] >> tz) == T && c < floor_c && c > best) best = c;
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
@@ -351,7 +408,7 @@ __device__ __forceinline__ void select_row_fast(const __nv_bfloat16* row, int S1
                                                 int32_t* out_idx, float* out_wt) {
   half_topk_bf16<R8, KC>(row, S1, K, lane, sc.surv, sc.stage, sc.a);
   half_topk_bf16<R8, KC>(row + S1, S2, K, lane, sc.surv, sc.stage, sc.b);
-  cand_topk_bf16<KC>(sc.a, sc.b, K, S2, ctab, lane, sc.cbuf,
+  cand_topk_bf16<KC>(sc.a, sc.b, K, S2, ctab, lane, sc.pv,
                      reinterpret_cast<uint64_t*>(sc.stage), out_idx, out_wt);
 }
 
@@ -367,7 +424,7 @@ __host__ __device__ inline int fast_kc(int K) { return K <= 32 ? 32 : (K <= 64 ?
 
 // Persistent fast selection kernel over rows of job0 followed by rows of job1.
 template <int R8, int KC>
-__global__ void __launch_bounds__(256) sel_fast_kernel(SelJob job0, SelJob job1, long long n_rows,
+__global__ void __launch_bounds__(256, 3) sel_fast_kernel(SelJob job0, SelJob job1, long long n_rows,
                                                        int njobs, int S1, int S2) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int C0 = cand_count(job0.K);

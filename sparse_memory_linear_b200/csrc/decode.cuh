@@ -3,20 +3,24 @@
 // Method: "Sparse Delta Memory: Scaling the State of Linear RNNs through Sparsity"
 // (paper.rainbus.top summary), method steps 1-4, applied to a single token; the m.163.com
 // article on SDM (section 八) reports decode as the setting where the HBM-resident
-// memory costs most.  One CTA per (b, h):
-//   four warps select the four score halves (write and read, first and second half) and
-//   two of them then combine the candidate sums (step 1), while the other warps stage v,
-//   alpha, beta and the gate;
-//   every warp then rewrites its share of the W write rows (step 2) and, in the same
-//   pass, reads the read rows that this token does not write; after a barrier the read
-//   rows inside the write set are read back (this CTA's own stores) (step 3);
-//   the CTA sums the R weighted rows, then normalises and gates them (step 4).
-// About 33 KB of shared memory per CTA keeps a 64 x 8 batch in one wave.
+// memory costs most.  One CTA of 8 warps per (b, h), in one wave for a 64 x 8 batch:
+//   step 1 (bf16 halves of up to 1024 scores, K <= 128): two warps per score half (write
+//   and read selection, first and second half) find the half's top K with the group
+//   selection of select_group.cuh; four warps per selection then take the top K of the
+//   rank-pair candidate sums the same way and write slot indices and softmax weights.
+//   Other shapes: warps 0 and 1 run the warp-per-row selection of select.cuh;
+//   step 2: every warp rewrites its share of the W write rows; a write row that the token
+//   also reads is added to the warp's read sum straight from the registers that hold its
+//   new value;
+//   step 3: the read rows that the token does not write were prefetched into L2 when the
+//   selection ended; every warp adds its share;
+//   step 4: warp 0 sums the eight partial reads, normalises and gates them.
 #pragma once
 
 #include "common.cuh"
 #include "select.cuh"
 #include "select_fast.cuh"
+#include "select_group.cuh"
 
 namespace sdm {
 
@@ -41,117 +45,301 @@ constexpr int DEC_THREADS = 256;
 constexpr int DEC_WARPS = DEC_THREADS / 32;
 
 struct DecLayout {
-  size_t off_tab_w, off_tab_r, off_sel, sel_stride, off_list, off_vec, off_part, total;
-  bool fast;
+  uint32_t off_tab_w, off_tab_r, off_lists, off_vec, off_part;
+  // group selection
+  uint32_t off_hist, off_ctl, off_list, list_stride, off_clist, clist_stride, off_sorted, off_ev;
+  // warp-per-row selection
+  uint32_t off_sel, sel_stride;
+  uint32_t total;
+  int C_w, C_r;  // candidate counts of W and R
 };
 
-// Shared-memory plan: the two candidate tables, four selection scratch areas (fast path:
-// one per score half; general path: one per selection), the selected lists, v / gate /
-// gates and the per-warp partial reads.
-__host__ __device__ inline DecLayout dec_layout(int S1, int S2, int W, int R, int d_v, bool fast,
-                                                int kc) {
-  DecLayout L;
+// Shared-memory plan.  `group` selects the group selection (histograms, control words, four
+// half lists, two candidate lists, the sorted halves, softmax numerators); otherwise two
+// warp selection scratch areas.
+inline DecLayout dec_layout(int S1, int S2, int W, int R, int d_v, bool group) {
+  DecLayout L{};
+  size_t p = 0;
+  auto take = [&p](size_t bytes) {
+    const size_t o = p;
+    p += (bytes + 15) / 16 * 16;
+    return static_cast<uint32_t>(o);
+  };
+  L.C_w = cand_count(W);
+  L.C_r = cand_count(R);
   const int kmax = W > R ? W : R;
-  L.fast = fast;
-  L.off_tab_w = 0;
-  L.off_tab_r = L.off_tab_w + (size_t)((cand_count(W) + 7) / 8) * 16;
-  L.off_sel = L.off_tab_r + (size_t)((cand_count(R) + 7) / 8) * 16;
-  L.sel_stride = fast ? fast_scratch_bytes(S1, S2, kc) : sel_scratch_bytes(S1, S2, kmax);
-  L.sel_stride = (L.sel_stride + 15) / 16 * 16;
-  L.off_list = L.off_sel + (L.fast ? 4 : 2) * L.sel_stride;
-  // idx_w[KMAX], wt_w[KMAX], idx_r[KMAX], wt_r[KMAX]
-  L.off_vec = L.off_list + 4 * (size_t)KMAX * 4;
-  // v[d_v], act(gate)[d_v], alpha, beta, ssq partials
-  L.off_part = L.off_vec + ((size_t)(2 * d_v + 16 + DEC_WARPS) * 4 + 15) / 16 * 16;
-  L.total = L.off_part + (size_t)DEC_WARPS * d_v * 4;
+  const int smax = S1 > S2 ? S1 : S2;
+  L.off_tab_w = take((size_t)cand_count(W) * 2);
+  L.off_tab_r = take((size_t)cand_count(R) * 2);
+  L.off_lists = take(4 * (size_t)KMAX * 4);  // idx_w, wt_w, idx_r, wt_r
+  L.off_vec = take((2 * (size_t)d_v + 4) * 4);  // v, act(gate), alpha, beta
+  L.off_part = take((size_t)DEC_WARPS * d_v * 4);
+  if (group) {
+    L.off_hist = take(4 * 256 * 4);
+    L.off_ctl = take(6 * sizeof(GroupCtl));
+    L.list_stride = ((size_t)(smax + 4) * 4 + 15) / 16 * 16;
+    L.off_list = take(4 * L.list_stride);
+    L.clist_stride = ((size_t)(cand_count(kmax) + 2) * 8 + 15) / 16 * 16;
+    L.off_clist = take(2 * L.clist_stride);
+    L.off_sorted = take(4 * (size_t)KMAX * 4);
+    L.off_ev = take(2 * (size_t)KMAX * 4);
+  } else {
+    L.sel_stride = (sel_scratch_bytes(S1, S2, kmax) + 15) / 16 * 16;
+    L.off_sel = take(2 * L.sel_stride);
+  }
+  L.total = static_cast<uint32_t>(p);
   return L;
 }
 
-// Step 1 of one token on the CTA's warps.  Fast path: warps 0-3 take the four score halves
-// (write first, write second, read first, read second), then warps 0 and 2 combine the
-// candidates of the write and the read selection.  General path: warps 0 and 1.
-template <int R8, int KC>
-__device__ __forceinline__ void decode_select_fast(const DecodeArgs& a, const DecLayout& L,
-                                                   unsigned char* smem, int warp, int lane,
-                                                   int32_t* idx_w, float* wt_w, int32_t* idx_r,
-                                                   float* wt_r) {
-  const int S = a.S1 + a.S2;
-  if (warp < 4) {
-    const bool rd = warp >= 2;
-    const bool second = warp & 1;
-    const __nv_bfloat16* row =
-        reinterpret_cast<const __nv_bfloat16*>(rd ? a.qp : a.kp) + (size_t)blockIdx.x * S;
-    const int K = rd ? a.R : a.W;
-    FastScratch own = carve_fast_scratch(smem + L.off_sel + warp * L.sel_stride, a.S1, a.S2, KC);
-    FastScratch pair =
-        carve_fast_scratch(smem + L.off_sel + (rd ? 2 : 0) * L.sel_stride, a.S1, a.S2, KC);
-    half_topk_bf16<R8, KC>(second ? row + a.S1 : row, second ? a.S2 : a.S1, K, lane, own.surv,
-                           own.stage, second ? pair.b : pair.a);
+// floor(a / b) for 0 <= a, b <= 128: the approximate quotient is within 2^-15 of a / b, and a
+// non-integer a / b is at least 1/128 below the next integer, so adding 2^-10 before the
+// floor recovers the exact quotient.
+__device__ __forceinline__ int quot_small(int a, int b) {
+  return static_cast<int>(__fdividef(static_cast<float>(a), static_cast<float>(b)) + 0x1p-10f);
+}
+
+// Rows of the candidate table of K (entries (r1 << 7) | r2 with (r1 + 1)(r2 + 1) <= K, rows
+// in r1 order) written by the four warps of one selection group, wq = 0..3: every warp
+// derives the row starts itself (a shuffle scan of the row lengths), then writes rows wq,
+// wq + 4, ... of the first 32 (whole warp per row) and one lane's share of rows 32 and up
+// (fewer than 4 entries each).
+__device__ __forceinline__ void build_cand_table_group(uint16_t* tab, int K, int wq, int lane) {
+  int len[4], start[4], run = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int r = 4 * lane + q;
+    len[q] = r < K ? quot_small(K, r + 1) : 0;
+    run += len[q];
   }
-  __syncthreads();
-  if (warp == 0 || warp == 2) {
-    const bool rd = warp == 2;
-    FastScratch pair = carve_fast_scratch(smem + L.off_sel + warp * L.sel_stride, a.S1, a.S2, KC);
-    cand_topk_bf16<KC>(pair.a, pair.b, rd ? a.R : a.W, a.S2,
-                       reinterpret_cast<const uint16_t*>(smem + (rd ? L.off_tab_r : L.off_tab_w)),
-                       lane, pair.pv, reinterpret_cast<uint64_t*>(pair.stage),
-                       rd ? idx_r : idx_w, rd ? wt_r : wt_w);
+  int incl = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(FULL_MASK, incl, o);
+    if (lane >= o) incl += t;
+  }
+  int base = incl - run;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    start[q] = base;
+    base += len[q];
+  }
+  const int rl = K < 32 ? K : 32;
+  for (int r = wq; r < rl; r += 4) {  // r is warp-uniform: r & 3 == wq
+    const int s0 = __shfl_sync(FULL_MASK, wq == 0 ? start[0] : wq == 1 ? start[1] : wq == 2 ? start[2] : start[3], r >> 2);
+    const int n = quot_small(K, r + 1);
+    for (int r2 = lane; r2 < n; r2 += 32) tab[s0 + r2] = static_cast<uint16_t>((r << 7) | r2);
+  }
+  const int r = 32 + 4 * lane + wq;  // rows 32..127: row r lives in lane r >> 2, slot wq
+  const int s0 = __shfl_sync(FULL_MASK, wq == 0 ? start[0] : wq == 1 ? start[1] : wq == 2 ? start[2] : start[3], (r >> 2) & 31);
+  if (r < K) {
+    const int n = quot_small(K, r + 1);
+    for (int r2 = 0; r2 < n; ++r2) tab[s0 + r2] = static_cast<uint16_t>((r << 7) | r2);
   }
 }
 
-// R8 == 0 takes the general selection (fp32 halves, halves longer than 1024 values);
-// otherwise the fast path for halves of up to 256*R8 values and K <= KC.  NQ float4 columns
-// per lane: d_v <= 128*NQ.
-template <int R8, int KC, int NQ>
-__global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a) {
+// Step 1 by the group selection: warps 2g, 2g + 1 take half g (0 write first, 1 write second,
+// 2 read first, 3 read second); warps 4s .. 4s + 3 then take the candidates of selection s.
+// E: bf16 scores per thread in units of 8 (halves of up to 512 E scores).  KC: largest K.
+template <int E, int KC>
+__device__ __forceinline__ void decode_select_group(const DecodeArgs& a, const DecLayout& L,
+                                                    unsigned char* smem, int tid,
+                                                    const uint32_t (&key)[E * 8],
+                                                    int32_t* idx_w, float* wt_w, int32_t* idx_r,
+                                                    float* wt_r) {
+  constexpr int NK = E * 8;
+  constexpr int CPT = (cand_count(KC) + 127) / 128;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int g = warp >> 1, gt = tid & 63;
+  const int s = g >> 1, st = tid & 127;
+  const int K = s ? a.R : a.W;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L.off_hist);
+  GroupCtl* ctl = reinterpret_cast<GroupCtl*>(smem + L.off_ctl);
+  uint32_t* sorted = reinterpret_cast<uint32_t*>(smem + L.off_sorted);
+
+  // half g: bracket from every thread's P-th largest key, P = ceil(K / 64)
+  uint32_t t1 = 0u, t2 = 0u;
+#pragma unroll
+  for (int i = 0; i < NK; ++i) {
+    const uint32_t x = key[i];
+    t2 = max(t2, min(t1, x));
+    t1 = max(t1, x);
+  }
+  uint32_t lo, hi;
+  group_bracket<64>(t1, K > 64 ? t2 : t1, ctl + g, gt, 1 + g, lo, hi);
+  int n = 0;
+  const uint32_t cut =
+      group_cut<NK, 64>(key, lo, hi, K, 2 * K, hist + 256 * g, ctl + g, gt, 1 + g, n);
+  uint32_t* list = reinterpret_cast<uint32_t*>(smem + L.off_list + g * L.list_stride);
+  if (gt == 0) reinterpret_cast<uint4*>(list)[n >> 2] = make_uint4(0u, 0u, 0u, 0u);
+  group_bar(1 + g, 64);  // the padding store lands before any composite of the last quad
+  group_collect<NK>(
+      key, cut,
+      [&](int i) {
+        const int idx = (i >> 3) * 512 + gt * 8 + (i & 7);
+        return (key[i] << 16) | (0xffffu - static_cast<uint32_t>(idx));
+      },
+      list, &ctl[g].count, lane);
+  group_bar(1 + g, 64);
+  group_rank32<64>(list, n, K, gt, sorted + KMAX * g);
+  group_bar(5 + s, 128);
+
+  // candidates of selection s
+  const uint32_t* A = sorted + KMAX * (2 * s);
+  const uint32_t* B = sorted + KMAX * (2 * s + 1);
+  const uint16_t* tab = reinterpret_cast<const uint16_t*>(smem + (s ? L.off_tab_r : L.off_tab_w));
+  const int C = s ? L.C_r : L.C_w;
+  uint32_t ck[CPT], cf[CPT];
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) {
+    const int c = st + 128 * j;
+    ck[j] = 0u;
+    cf[j] = 0u;
+    if (c < C) {
+      const int e = tab[c];
+      const uint32_t ca = A[e >> 7], cb = B[e & 127];
+      ck[j] = score_key(__fadd_rn(key16_value(ca >> 16), key16_value(cb >> 16)));
+      cf[j] = (0xffffu - (ca & 0xffffu)) * static_cast<uint32_t>(a.S2) + (0xffffu - (cb & 0xffffu));
+    }
+  }
+  // the K sums A[i] + B[0] and the K sums A[0] + B[i] are candidates: both K-th largest
+  // bound the K-th largest candidate from below
+  const float a0 = key16_value(A[0] >> 16), b0 = key16_value(B[0] >> 16);
+  const uint32_t chi = score_key(__fadd_rn(a0, b0));
+  const uint32_t clo = max(max(score_key(__fadd_rn(key16_value(A[K - 1] >> 16), b0)),
+                               score_key(__fadd_rn(a0, key16_value(B[K - 1] >> 16)))), 1u);
+  GroupCtl* cctl = ctl + 4 + s;
+  const uint32_t ccut = group_cut<CPT, 128>(ck, clo, chi, K, 2 * K, hist + 256 * (2 * s), cctl,
+                                            st, 5 + s, n);
+  uint64_t* clist = reinterpret_cast<uint64_t*>(smem + L.off_clist + s * L.clist_stride);
+  if (st == 0) reinterpret_cast<ulonglong2*>(clist)[n >> 1] = make_ulonglong2(0ull, 0ull);
+  group_bar(5 + s, 128);
+  group_collect<CPT>(
+      ck, ccut,
+      [&](int j) { return (static_cast<uint64_t>(ck[j]) << 32) | (0xffffffffu - cf[j]); }, clist,
+      &cctl->count, lane);
+  group_bar(5 + s, 128);
+  float* ev = reinterpret_cast<float*>(smem + L.off_ev) + KMAX * s;
+  int32_t* out_idx = s ? idx_r : idx_w;
+  float* out_wt = s ? wt_r : wt_w;
+  const float s0 = key_score(chi);
+  group_rank64<128>(clist, n, st, [&](int r, uint64_t c) {
+    if (r < K) {
+      out_idx[r] = static_cast<int32_t>(0xffffffffu - static_cast<uint32_t>(c));
+      ev[r] = expf(key_score(static_cast<uint32_t>(c >> 32)) - s0);
+    }
+  });
+  group_bar(5 + s, 128);
+  if (st < K) {
+    float sum = 0.0f;
+    for (int j = 0; j < K; ++j) sum += ev[j];
+    out_wt[st] = ev[st] * (1.0f / sum);
+  }
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// E == 0: warp-per-row selection (fp32 halves, halves longer than 1024 scores); otherwise
+// the group selection for bf16 halves of up to 512 E scores and K <= KC.  NQ float4
+// columns per lane: d_v <= 128 NQ.
+template <int E, int KC, int NQ>
+__global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, DecLayout L) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int bh = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool bf16 = a.in_bf16 != 0;
-  const DecLayout L = dec_layout(a.S1, a.S2, a.W, a.R, a.d_v, R8 > 0, KC);
-  const int kmax = a.W > a.R ? a.W : a.R;
   const int S = a.S1 + a.S2;
   const int d4 = a.d_v / 4;
-  const size_t esz = bf16 ? 2 : 4;
 
   uint16_t* tab_w = reinterpret_cast<uint16_t*>(smem + L.off_tab_w);
   uint16_t* tab_r = reinterpret_cast<uint16_t*>(smem + L.off_tab_r);
-  int32_t* idx_w = reinterpret_cast<int32_t*>(smem + L.off_list);
+  int32_t* idx_w = reinterpret_cast<int32_t*>(smem + L.off_lists);
   float* wt_w = reinterpret_cast<float*>(idx_w + KMAX);
   int32_t* idx_r = reinterpret_cast<int32_t*>(wt_w + KMAX);
   float* wt_r = reinterpret_cast<float*>(idx_r + KMAX);
   float* vs = reinterpret_cast<float*>(smem + L.off_vec);  // [d_v]
   float* gs = vs + a.d_v;                                  // [d_v]
   float* ab = gs + a.d_v;                                  // alpha, beta
-  float* ssq = ab + 16;                                    // [DEC_WARPS]
   float* part = reinterpret_cast<float*>(smem + L.off_part);  // [DEC_WARPS][d_v]
 
-  build_cand_table(tab_w, a.W, tid, DEC_THREADS);
-  build_cand_table(tab_r, a.R, tid, DEC_THREADS);
-  // the per-token vectors, staged by the warps that do not select
-  const int first_free = R8 > 0 ? 4 : 2;
-  if (warp >= first_free) {
-    const int t0 = tid - 32 * first_free, nt = DEC_THREADS - 32 * first_free;
-    for (int c = t0; c < a.d_v; c += nt) {
-      vs[c] = load_in(a.v, (size_t)bh * a.d_v + c, bf16);
-      gs[c] = a.gate ? gate_act(load_in(a.gate, (size_t)bh * a.d_v + c, bf16), a.act) : 1.0f;
+  if constexpr (E > 0) {
+    // issue this thread's score loads first: everything else overlaps their latency
+    const int g = warp >> 1, gt = tid & 63;
+    const int Sh = (g & 1) ? a.S2 : a.S1;
+    const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>((g >> 1) ? a.qp : a.kp) +
+                               (size_t)bh * S + ((g & 1) ? a.S1 : 0);
+    const bool vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
+    const uint16_t* raw16 = reinterpret_cast<const uint16_t*>(src);
+    uint32_t key[E * 8];
+#pragma unroll
+    for (int r = 0; r < E; ++r) {
+      const int e0 = r * 512 + gt * 8;
+      if (vec && e0 + 8 <= Sh) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + e0));
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          key[r * 8 + 2 * j] = ww[j];
+          key[r * 8 + 2 * j + 1] = ww[j] >> 16;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) key[r * 8 + i] = (e0 + i < Sh) ? raw16[e0 + i] : 0u;
+      }
     }
-    if (t0 == 0) {
-      ab[0] = a.alpha[bh];
-      ab[1] = a.beta[bh];
+    // this thread's v, gate, alpha, beta loads (d_v <= 128 NQ: at most VQ of each)
+    constexpr int VQ = NQ <= 2 ? 1 : NQ / 2;
+    float vr[VQ], gr[VQ], abr = 0.0f;
+#pragma unroll
+    for (int q = 0; q < VQ; ++q) {
+      const int c = tid + DEC_THREADS * q;
+      vr[q] = c < a.d_v ? load_in(a.v, (size_t)bh * a.d_v + c, bf16) : 0.0f;
+      gr[q] = c < a.d_v && a.gate ? load_in(a.gate, (size_t)bh * a.d_v + c, bf16) : 0.0f;
     }
-  }
-  __syncthreads();
-
-  // step 1
-  if (R8 > 0) {
-    decode_select_fast<(R8 > 0 ? R8 : 1), KC>(a, L, smem, warp, lane, idx_w, wt_w, idx_r, wt_r);
-  } else if (warp < 2) {
-    SelScratch sc = carve_sel_scratch(smem + L.off_sel + warp * L.sel_stride, a.S1, a.S2, kmax);
-    const void* src = reinterpret_cast<const unsigned char*>(warp == 0 ? a.kp : a.qp) +
-                      (size_t)bh * S * esz;
-    select_row(src, bf16, a.S1, a.S2, warp == 0 ? a.W : a.R, warp == 0 ? tab_w : tab_r, sc,
-               lane, warp == 0 ? idx_w : idx_r, warp == 0 ? wt_w : wt_r);
+    if (tid < 2) abr = tid == 0 ? a.alpha[bh] : a.beta[bh];
+    // shared state of the group selection: this group's histogram and control words
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L.off_hist);
+    GroupCtl* ctl = reinterpret_cast<GroupCtl*>(smem + L.off_ctl);
+    reinterpret_cast<uint4*>(hist + 256 * g)[gt] = make_uint4(0u, 0u, 0u, 0u);
+    if (gt == 0) ctl[g].count = 0u;
+    if ((tid & 127) == 0) ctl[4 + (tid >> 7)].count = 0u;
+    build_cand_table_group((tid >> 7) ? tab_r : tab_w, (tid >> 7) ? a.R : a.W, warp & 3, lane);
+#pragma unroll
+    for (int q = 0; q < VQ; ++q) {
+      const int c = tid + DEC_THREADS * q;
+      if (c < a.d_v) {
+        vs[c] = vr[q];
+        gs[c] = a.gate ? gate_act(gr[q], a.act) : 1.0f;
+      }
+    }
+    if (tid < 2) ab[tid] = abr;
+#pragma unroll
+    for (int i = 0; i < E * 8; ++i)
+      key[i] = (i >> 3) * 512 + gt * 8 + (i & 7) < Sh ? bf16_key16(key[i]) : 0u;
+    decode_select_group<E, KC>(a, L, smem, tid, key, idx_w, wt_w, idx_r, wt_r);
+  } else {
+    const int kmax = a.W > a.R ? a.W : a.R;
+    const size_t esz = bf16 ? 2 : 4;
+    build_cand_table(tab_w, a.W, tid, DEC_THREADS);
+    build_cand_table(tab_r, a.R, tid, DEC_THREADS);
+    if (warp >= 2) {
+      const int t0 = tid - 64, nt = DEC_THREADS - 64;
+      for (int c = t0; c < a.d_v; c += nt) {
+        vs[c] = load_in(a.v, (size_t)bh * a.d_v + c, bf16);
+        gs[c] = a.gate ? gate_act(load_in(a.gate, (size_t)bh * a.d_v + c, bf16), a.act) : 1.0f;
+      }
+      if (t0 == 0) {
+        ab[0] = a.alpha[bh];
+        ab[1] = a.beta[bh];
+      }
+    } else {
+      SelScratch sc = carve_sel_scratch(smem + L.off_sel + warp * L.sel_stride, a.S1, a.S2, kmax);
+      const void* src = reinterpret_cast<const unsigned char*>(warp == 0 ? a.kp : a.qp) +
+                        (size_t)bh * S * esz;
+      select_row(src, bf16, a.S1, a.S2, warp == 0 ? a.W : a.R, warp == 0 ? tab_w : tab_r, sc,
+                 lane, warp == 0 ? idx_w : idx_r, warp == 0 ? wt_w : wt_r);
+    }
   }
   __syncthreads();
 
@@ -162,6 +350,16 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a) {
   }
 
   float* Mbh = a.M + (size_t)bh * a.N * a.d_v;
+  // the read rows go to L2 now, while the write rows are loaded and rewritten
+  {
+    const int lpr = (a.d_v + 31) / 32;  // 128-byte lines per row
+    for (int l = tid; l < a.R * lpr; l += DEC_THREADS) {
+      const int j = l / lpr;
+      const int sl = idx_r[j];
+      if (static_cast<unsigned>(sl) < static_cast<unsigned>(a.N))
+        prefetch_l2(Mbh + (size_t)sl * a.d_v + (l - j * lpr) * 32);
+    }
+  }
   const float al = ab[0], be = ab[1];
   float4 acc[NQ];
 #pragma unroll
@@ -169,7 +367,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a) {
 
   // step 2: this warp's write rows (warp, warp + 8, ...), RB at a time: every row load is
   // issued before any update, so a warp waits for one memory latency per RB rows
-  constexpr int RB = 8 / NQ;
+  constexpr int RB = NQ >= 8 ? 1 : 8 / NQ;
   for (int j0 = warp; j0 < a.W; j0 += DEC_WARPS * RB) {
     float4 old[RB][NQ];
     int slot[RB];
@@ -194,6 +392,13 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a) {
         if (lane == 0) record_status(STATUS_BAD_INDEX);
         continue;
       }
+      // read weight of this slot if the token also reads it
+      int rpos = -1;
+      for (int e0 = 0; e0 < a.R; e0 += 32) {
+        const unsigned m = __ballot_sync(FULL_MASK, e0 + lane < a.R && idx_r[e0 + lane] == slot[r]);
+        if (m && rpos < 0) rpos = e0 + __ffs(m) - 1;
+      }
+      const float qr = rpos >= 0 ? wt_r[rpos] : 0.0f;
       const float kb = be * wt_w[j];
       const float ka = al * (1.0f - kb);
       float4* row = reinterpret_cast<float4*>(Mbh + (size_t)slot[r] * a.d_v);
@@ -209,12 +414,17 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a) {
           nw.z = fmaf(ka, old[r][q].z, kb * vv.z);
           nw.w = fmaf(ka, old[r][q].w, kb * vv.w);
           row[c] = nw;
+          if (rpos >= 0) {
+            acc[q].x = fmaf(qr, nw.x, acc[q].x);
+            acc[q].y = fmaf(qr, nw.y, acc[q].y);
+            acc[q].z = fmaf(qr, nw.z, acc[q].z);
+            acc[q].w = fmaf(qr, nw.w, acc[q].w);
+          }
         }
       }
     }
   }
-  // step 3 for the read rows this token does not write (no dependence on step 2), RB at a
-  // time in the same way
+  // step 3 for the read rows this token does not write, RB at a time
   for (int j0 = warp; j0 < a.R; j0 += DEC_WARPS * RB) {
     float4 val[RB][NQ];
     bool use[RB];
@@ -256,28 +466,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a) {
       }
     }
   }
-  __syncthreads();
-  // step 3 for read rows inside the write set: this CTA's own stores, visible after the
-  // barrier
-  for (int j = warp; j < a.R; j += DEC_WARPS) {
-    const int s = idx_r[j];
-    bool in_w = false;
-    for (int e = lane; e < a.W; e += 32) in_w |= (idx_w[e] == s);
-    if (!__any_sync(FULL_MASK, in_w)) continue;
-    const float q = wt_r[j];
-    const float4* row = reinterpret_cast<const float4*>(Mbh + (size_t)s * a.d_v);
-#pragma unroll
-    for (int qq = 0; qq < NQ; ++qq) {
-      const int c = lane + 32 * qq;
-      if (c < d4) {
-        const float4 val = row[c];
-        acc[qq].x = fmaf(q, val.x, acc[qq].x);
-        acc[qq].y = fmaf(q, val.y, acc[qq].y);
-        acc[qq].z = fmaf(q, val.z, acc[qq].z);
-        acc[qq].w = fmaf(q, val.w, acc[qq].w);
-      }
-    }
-  }
 #pragma unroll
   for (int qq = 0; qq < NQ; ++qq) {
     const int c = lane + 32 * qq;
@@ -285,36 +473,48 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a) {
   }
   __syncthreads();
 
-  // y and step 4
-  float yv[4];
+  // y and step 4 on warp 0
+  if (warp != 0) return;
+  float4 yv[NQ];
   float ss = 0.0f;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int c = tid + DEC_THREADS * q;
-    yv[q] = 0.0f;
-    if (c < a.d_v) {
-      float s = 0.0f;
-      for (int w = 0; w < DEC_WARPS; ++w) s += part[(size_t)w * a.d_v + c];
-      yv[q] = s;
-      a.y[(size_t)bh * a.d_v + c] = s;
-      ss = fmaf(s, s, ss);
+  for (int qq = 0; qq < NQ; ++qq) {
+    const int c = lane + 32 * qq;
+    yv[qq] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (c < d4) {
+      float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int w = 0; w < DEC_WARPS; ++w) {
+        const float4 p = reinterpret_cast<const float4*>(part + (size_t)w * a.d_v)[c];
+        t.x += p.x;
+        t.y += p.y;
+        t.z += p.z;
+        t.w += p.w;
+      }
+      yv[qq] = t;
+      reinterpret_cast<float4*>(a.y + (size_t)bh * a.d_v)[c] = t;
+      ss = fmaf(t.x, t.x, ss);
+      ss = fmaf(t.y, t.y, ss);
+      ss = fmaf(t.z, t.z, ss);
+      ss = fmaf(t.w, t.w, ss);
     }
   }
-  if (a.o) {
+  if (!a.o) return;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(FULL_MASK, ss, o);
-    if (lane == 0) ssq[warp] = ss;
-    __syncthreads();
-    float tot = 0.0f;
-    for (int w = 0; w < DEC_WARPS; ++w) tot += ssq[w];
-    const float inv = rsqrtf(tot / static_cast<float>(a.d_v) + a.eps);
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(FULL_MASK, ss, o);
+  const float inv = rsqrtf(ss / static_cast<float>(a.d_v) + a.eps);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int c = tid + DEC_THREADS * q;
-      if (c < a.d_v) {
-        const float gm = a.gamma ? a.gamma[c] : 1.0f;
-        a.o[(size_t)bh * a.d_v + c] = yv[q] * inv * gm * gs[c];
-      }
+  for (int qq = 0; qq < NQ; ++qq) {
+    const int c = lane + 32 * qq;
+    if (c < d4) {
+      const float4 g4 = reinterpret_cast<const float4*>(gs)[c];
+      const float4 m4 = a.gamma ? reinterpret_cast<const float4*>(a.gamma)[c]
+                                : make_float4(1.f, 1.f, 1.f, 1.f);
+      float4 r;
+      r.x = yv[qq].x * inv * m4.x * g4.x;
+      r.y = yv[qq].y * inv * m4.y * g4.y;
+      r.z = yv[qq].z * inv * m4.z * g4.z;
+      r.w = yv[qq].w * inv * m4.w * g4.w;
+      reinterpret_cast<float4*>(a.o + (size_t)bh * a.d_v)[c] = r;
     }
   }
 }

@@ -21,10 +21,10 @@ namespace {
 
 constexpr int MAX_DEVICES = 64;
 
-// decode_kernel instantiations, cheapest first: (halves class R8, K class, float4 columns
-// per lane).  R8 == 0 is the general selection.
+// decode_kernel instantiations, cheapest first: (scores per thread / 8, K class, float4
+// columns per lane).  E == 0 is the warp-per-row selection.
 #define SDM_DEC_VARIANTS(X) \
-  X(1, 32, 1) X(2, 64, 1) X(4, 64, 2) X(4, 128, 8) X(0, 128, 8)
+  X(1, 64, 1) X(1, 128, 2) X(2, 128, 2) X(2, 128, 8) X(0, 128, 8)
 constexpr size_t WS_ALIGN = 256;
 
 #define SDM_CUDA_TRY(expr)                       \
@@ -702,20 +702,12 @@ sdm_status sdm_decode_step(const void* kp, const void* qp, const void* v, const 
   sdm_status rc = device_info(&di);
   if (rc != SDM_OK) return rc;
   const bool fast = fast_select_ok(s.in_dtype == SDM_BF16, s.S1, s.S2, s.W > s.R ? s.W : s.R);
-  const int need_r8 = fast ? fast_r8(s.S1, s.S2) : 0;
-  const int need_kc = fast_kc(s.W > s.R ? s.W : s.R);
+  const int need_e = fast ? ((s.S1 > s.S2 ? s.S1 : s.S2) <= 512 ? 1 : 2) : 0;
+  const int need_kc = (s.W > s.R ? s.W : s.R) <= 64 ? 64 : 128;
   const int need_nq = (s.d_v / 4 + 31) / 32;
-  int v_r8 = -1, v_kc = 0;
-#define SDM_DEC_PICK(R8, KC, NQ)                                                   \
-  if (v_r8 < 0 && (fast ? (R8 >= need_r8 && R8 > 0) : R8 == 0) && KC >= need_kc && \
-      NQ >= need_nq) {                                                              \
-    v_r8 = R8;                                                                      \
-    v_kc = KC;                                                                      \
-  }
-  SDM_DEC_VARIANTS(SDM_DEC_PICK)
-#undef SDM_DEC_PICK
-  if (v_r8 < 0) return SDM_ERR_UNSUPPORTED;
-  const DecLayout L = dec_layout(s.S1, s.S2, s.W, s.R, s.d_v, v_r8 > 0, v_kc);
+#define SDM_DEC_FITS(E, KC, NQ) \
+  ((fast ? (E >= need_e && E > 0) : E == 0) && KC >= need_kc && NQ >= need_nq)
+  const DecLayout L = dec_layout(s.S1, s.S2, s.W, s.R, s.d_v, fast);
   if (L.total > (size_t)di->max_smem_optin) return SDM_ERR_UNSUPPORTED;
   DecodeArgs a;
   a.kp = kp;
@@ -741,15 +733,15 @@ sdm_status sdm_decode_step(const void* kp, const void* qp, const void* v, const 
   a.in_bf16 = s.in_dtype == SDM_BF16;
   ProfScope ps(SDM_KERNEL_DECODE, static_cast<cudaStream_t>(stream));
   bool launched = false;
-#define SDM_DEC_LAUNCH(R8, KC, NQ)                                                        \
-  if (!launched && (fast ? (R8 >= need_r8 && R8 > 0) : R8 == 0) && KC >= need_kc &&        \
-      NQ >= need_nq) {                                                                     \
-    decode_kernel<R8, KC, NQ><<<a.BH, DEC_THREADS, L.total, static_cast<cudaStream_t>(stream)>>>(a); \
-    g_launches.fetch_add(1, std::memory_order_relaxed);                                    \
-    launched = true;                                                                       \
+#define SDM_DEC_LAUNCH(E, KC, NQ)                                                        \
+  if (!launched && SDM_DEC_FITS(E, KC, NQ)) {                                             \
+    decode_kernel<E, KC, NQ><<<a.BH, DEC_THREADS, L.total, static_cast<cudaStream_t>(stream)>>>(a, L); \
+    g_launches.fetch_add(1, std::memory_order_relaxed);                                   \
+    launched = true;                                                                      \
   }
   SDM_DEC_VARIANTS(SDM_DEC_LAUNCH)
 #undef SDM_DEC_LAUNCH
+#undef SDM_DEC_FITS
   if (!launched) return SDM_ERR_UNSUPPORTED;
   SDM_CUDA_TRY(cudaGetLastError());
   return SDM_OK;

@@ -273,6 +273,8 @@ def decode_steps(sdm, wl, steps, M, gamma=None):
     dict(B=2, H=3, S1=20, S2=12, W=7, R=3, d_v=12, in_dtype=F32),
     dict(B=1, H=1, S1=256, S2=256, W=128, R=64, d_v=256, in_dtype=BF16),
     dict(B=2, H=1, S1=64, S2=64, W=16, R=16, d_v=1024, in_dtype=BF16),
+    dict(B=2, H=2, S1=1024, S2=1024, W=64, R=32, d_v=128, in_dtype=BF16),
+    dict(B=1, H=3, S1=200, S2=136, W=100, R=128, d_v=32, in_dtype=BF16),
 ])
 def test_decode_matches_oracle(sdm, kw):
     wl = sdm_synth.WORKLOADS["decode"].replace(T=6, seed=21, **kw)
@@ -293,6 +295,41 @@ def test_decode_matches_oracle(sdm, kw):
     assert_close(host(y), ref["y"], "decode y")
     assert_close(host(o), ref["o"], "decode o")
     assert_close(host(M), ref["M"], "decode M")
+
+
+@pytest.mark.parametrize("S1,S2,W,R", [(64, 64, 16, 16), (512, 512, 64, 64),
+                                         (128, 160, 128, 100)])
+def test_decode_ties_and_signed_zeros(sdm, S1, S2, W, R):
+    """Decode selection on scores drawn from a small palette (many equal sums, -0 and +0):
+    equal scores take the lowest indices, exactly as the oracle orders them."""
+    wl = sdm_synth.WORKLOADS["decode"].replace(B=3, H=2, T=3, S1=S1, S2=S2, W=W, R=R,
+                                               d_v=64, seed=29)
+    rng = np.random.default_rng(S1 + W)
+    palette = np.array([-1.0, -0.0, 0.0, 0.5, 1.0, 1.0, 2.0, 0.25], np.float32)
+    steps = []
+    for s in range(wl.T):
+        st = sdm_synth.make_inputs(wl, step=s)
+        for k in ("kp", "qp"):
+            x = palette[rng.integers(0, palette.size, tuple(st[k].shape))]
+            if s == 1:
+                x[0] = 0.0
+                x[1] = -0.0
+            st[k] = torch.from_numpy(x).to(BF16)
+        steps.append(st)
+    M0 = steps[0]["M0"]
+    M = M0.to(DEV).unsqueeze(0).expand(wl.B, -1, -1, -1).contiguous()
+    y, o, sels = decode_steps(sdm, wl, steps, M)
+    st = lambda k: np.stack([host(s[k]) for s in steps], 1)  # noqa: E731
+    ref = oracle.forward(st("kp"), st("qp"), st("v"), st("alpha"), st("beta"), host(M0),
+                         S1=wl.S1, W=wl.W, R=wl.R, gate=st("gate"))
+    for t, sel in enumerate(sels):
+        nw = wl.B * wl.H * wl.W
+        np.testing.assert_array_equal(sel[:nw].view(wl.B, wl.H, wl.W).cpu().numpy(),
+                                      ref["idx_w"][:, t])
+        np.testing.assert_array_equal(sel[nw:].view(wl.B, wl.H, wl.R).cpu().numpy(),
+                                      ref["idx_r"][:, t])
+    assert_close(host(y), ref["y"], "decode ties y")
+    assert_close(host(M), ref["M"], "decode ties M")
 
 
 def test_decode_equals_scan(sdm):

@@ -9,11 +9,13 @@
 //   selection of select_group.cuh; four warps per selection then take the top K of the
 //   rank-pair candidate sums the same way and write slot indices and softmax weights.
 //   Other shapes: warps 0 and 1 run the warp-per-row selection of select.cuh;
+//   steps 2 and 3 issue every row load of the token at once: each warp's write rows go to
+//   shared memory (over the dead selection scratch) by cp.async and its first read rows to
+//   registers, so the step waits for one memory latency;
 //   step 2: every warp rewrites its share of the W write rows; a write row that the token
 //   also reads is added to the warp's read sum straight from the registers that hold its
 //   new value;
-//   step 3: the read rows that the token does not write were prefetched into L2 when the
-//   selection ended; every warp adds its share;
+//   step 3: every warp adds its share of the read rows that the token does not write;
 //   step 4: warp 0 sums the eight partial reads, normalises and gates them.
 #pragma once
 
@@ -43,13 +45,20 @@ struct DecodeArgs {
 
 constexpr int DEC_THREADS = 256;
 constexpr int DEC_WARPS = DEC_THREADS / 32;
+// Largest write-row set staged in shared memory (W * d_v * 4 bytes); larger sets are loaded
+// into registers a batch at a time.
+constexpr size_t DEC_ROWS_SMEM_MAX = 64 * 1024;
 
 struct DecLayout {
   uint32_t off_tab_w, off_tab_r, off_lists, off_vec, off_part;
   // group selection
   uint32_t off_hist, off_ctl, off_list, list_stride, off_clist, clist_stride, off_sorted, off_ev;
+  uint32_t off_bits;  // 2048-bit membership filters of the write and the read slots
   // warp-per-row selection
   uint32_t off_sel, sel_stride;
+  // write rows staged over the selection scratch (dead once the selection is done)
+  uint32_t off_rows;
+  int rows_smem;
   uint32_t total;
   int C_w, C_r;  // candidate counts of W and R
 };
@@ -74,12 +83,14 @@ inline DecLayout dec_layout(int S1, int S2, int W, int R, int d_v, bool group) {
   L.off_lists = take(4 * (size_t)KMAX * 4);  // idx_w, wt_w, idx_r, wt_r
   L.off_vec = take((2 * (size_t)d_v + 4) * 4);  // v, act(gate), alpha, beta
   L.off_part = take((size_t)DEC_WARPS * d_v * 4);
+  L.off_bits = take(2 * 64 * 4);
+  const size_t scratch = p;
   if (group) {
-    L.off_hist = take(4 * 256 * 4);
+    L.off_hist = take(6 * 256 * 4);  // four halves, two candidate sets
     L.off_ctl = take(6 * sizeof(GroupCtl));
     L.list_stride = ((size_t)(smax + 4) * 4 + 15) / 16 * 16;
     L.off_list = take(4 * L.list_stride);
-    L.clist_stride = ((size_t)(cand_count(kmax) + 2) * 8 + 15) / 16 * 16;
+    L.clist_stride = ((size_t)(cand_count(kmax) + 4) * 8 + 15) / 16 * 16;
     L.off_clist = take(2 * L.clist_stride);
     L.off_sorted = take(4 * (size_t)KMAX * 4);
     L.off_ev = take(2 * (size_t)KMAX * 4);
@@ -87,6 +98,10 @@ inline DecLayout dec_layout(int S1, int S2, int W, int R, int d_v, bool group) {
     L.sel_stride = (sel_scratch_bytes(S1, S2, kmax) + 15) / 16 * 16;
     L.off_sel = take(2 * L.sel_stride);
   }
+  const size_t rows_bytes = (size_t)W * d_v * 4;
+  L.rows_smem = rows_bytes <= DEC_ROWS_SMEM_MAX;
+  L.off_rows = static_cast<uint32_t>(scratch);
+  if (L.rows_smem && scratch + rows_bytes > p) p = scratch + rows_bytes;
   L.total = static_cast<uint32_t>(p);
   return L;
 }
@@ -166,21 +181,19 @@ __device__ __forceinline__ void decode_select_group(const DecodeArgs& a, const D
   }
   uint32_t lo, hi;
   group_bracket<64>(t1, K > 64 ? t2 : t1, ctl + g, gt, 1 + g, lo, hi);
-  int n = 0;
-  const uint32_t cut =
-      group_cut<NK, 64>(key, lo, hi, K, 2 * K, hist + 256 * g, ctl + g, gt, 1 + g, n);
+  const CutResult cr =
+      group_cut<NK, 64>(key, lo, hi, K, 2 * K, hist + 256 * g, ctl + g, gt, 1 + g);
   uint32_t* list = reinterpret_cast<uint32_t*>(smem + L.off_list + g * L.list_stride);
-  if (gt == 0) reinterpret_cast<uint4*>(list)[n >> 2] = make_uint4(0u, 0u, 0u, 0u);
-  group_bar(1 + g, 64);  // the padding store lands before any composite of the last quad
-  group_collect<NK>(
-      key, cut,
+  uint32_t* out_half = sorted + KMAX * g;
+  group_order<NK, 64>(
+      key, cr,
       [&](int i) {
         const int idx = (i >> 3) * 512 + gt * 8 + (i & 7);
         return (key[i] << 16) | (0xffffu - static_cast<uint32_t>(idx));
       },
-      list, &ctl[g].count, lane);
-  group_bar(1 + g, 64);
-  group_rank32<64>(list, n, K, gt, sorted + KMAX * g);
+      list, &ctl[g].count, gt, lane, 1 + g, [&](int r, uint32_t c) {
+        if (r < K) out_half[r] = c;
+      });
   group_bar(5 + s, 128);
 
   // candidates of selection s
@@ -208,36 +221,39 @@ __device__ __forceinline__ void decode_select_group(const DecodeArgs& a, const D
   const uint32_t clo = max(max(score_key(__fadd_rn(key16_value(A[K - 1] >> 16), b0)),
                                score_key(__fadd_rn(a0, key16_value(B[K - 1] >> 16)))), 1u);
   GroupCtl* cctl = ctl + 4 + s;
-  const uint32_t ccut = group_cut<CPT, 128>(ck, clo, chi, K, 2 * K, hist + 256 * (2 * s), cctl,
-                                            st, 5 + s, n);
+  const CutResult cc =
+      group_cut<CPT, 128>(ck, clo, chi, K, 2 * K, hist + 256 * (4 + s), cctl, st, 5 + s);
   uint64_t* clist = reinterpret_cast<uint64_t*>(smem + L.off_clist + s * L.clist_stride);
-  if (st == 0) reinterpret_cast<ulonglong2*>(clist)[n >> 1] = make_ulonglong2(0ull, 0ull);
-  group_bar(5 + s, 128);
-  group_collect<CPT>(
-      ck, ccut,
-      [&](int j) { return (static_cast<uint64_t>(ck[j]) << 32) | (0xffffffffu - cf[j]); }, clist,
-      &cctl->count, lane);
-  group_bar(5 + s, 128);
   float* ev = reinterpret_cast<float*>(smem + L.off_ev) + KMAX * s;
   int32_t* out_idx = s ? idx_r : idx_w;
   float* out_wt = s ? wt_r : wt_w;
+  uint32_t* bits = reinterpret_cast<uint32_t*>(smem + L.off_bits) + 64 * s;
   const float s0 = key_score(chi);
-  group_rank64<128>(clist, n, st, [&](int r, uint64_t c) {
-    if (r < K) {
-      out_idx[r] = static_cast<int32_t>(0xffffffffu - static_cast<uint32_t>(c));
-      ev[r] = expf(key_score(static_cast<uint32_t>(c >> 32)) - s0);
-    }
-  });
+  group_order<CPT, 128>(
+      ck, cc, [&](int j) { return (static_cast<uint64_t>(ck[j]) << 32) | (0xffffffffu - cf[j]); },
+      clist, &cctl->count, st, lane, 5 + s, [&](int r, uint64_t c) {
+        if (r < K) {
+          const uint32_t flat = 0xffffffffu - static_cast<uint32_t>(c);
+          out_idx[r] = static_cast<int32_t>(flat);
+          ev[r] = expf(key_score(static_cast<uint32_t>(c >> 32)) - s0);
+          atomicOr(&bits[(flat >> 5) & 63u], 1u << (flat & 31u));
+        }
+      });
   group_bar(5 + s, 128);
   if (st < K) {
-    float sum = 0.0f;
-    for (int j = 0; j < K; ++j) sum += ev[j];
-    out_wt[st] = ev[st] * (1.0f / sum);
+    // the softmax denominator, the same sum in the same order on every thread (ev is zero
+    // past K up to the next multiple of 4)
+    const float4* e4 = reinterpret_cast<const float4*>(ev);
+    float s_0 = 0.0f, s_1 = 0.0f, s_2 = 0.0f, s_3 = 0.0f;
+    for (int j = 0; j < (K + 3) / 4; ++j) {
+      const float4 e = e4[j];
+      s_0 += e.x;
+      s_1 += e.y;
+      s_2 += e.z;
+      s_3 += e.w;
+    }
+    out_wt[st] = ev[st] * (1.0f / ((s_0 + s_1) + (s_2 + s_3)));
   }
-}
-
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 // E == 0: warp-per-row selection (fp32 halves, halves longer than 1024 scores); otherwise
@@ -304,6 +320,15 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
     reinterpret_cast<uint4*>(hist + 256 * g)[gt] = make_uint4(0u, 0u, 0u, 0u);
     if (gt == 0) ctl[g].count = 0u;
     if ((tid & 127) == 0) ctl[4 + (tid >> 7)].count = 0u;
+    {
+      // this selection group's candidate histogram, filter words and softmax tail
+      const int s = tid >> 7, st = tid & 127;
+      reinterpret_cast<uint2*>(hist + 256 * (4 + s))[st] = make_uint2(0u, 0u);
+      if (st < 64) reinterpret_cast<uint32_t*>(smem + L.off_bits)[64 * s + st] = 0u;
+      const int K = s ? a.R : a.W;
+      float* ev = reinterpret_cast<float*>(smem + L.off_ev) + KMAX * s;
+      if (K + st < ((K + 3) & ~3)) ev[K + st] = 0.0f;
+    }
     build_cand_table_group((tid >> 7) ? tab_r : tab_w, (tid >> 7) ? a.R : a.W, warp & 3, lane);
 #pragma unroll
     for (int q = 0; q < VQ; ++q) {
@@ -321,6 +346,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
   } else {
     const int kmax = a.W > a.R ? a.W : a.R;
     const size_t esz = bf16 ? 2 : 4;
+    if (tid < 128) reinterpret_cast<uint32_t*>(smem + L.off_bits)[tid] = 0u;
     build_cand_table(tab_w, a.W, tid, DEC_THREADS);
     build_cand_table(tab_r, a.R, tid, DEC_THREADS);
     if (warp >= 2) {
@@ -342,6 +368,18 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
     }
   }
   __syncthreads();
+  if constexpr (E == 0) {
+    uint32_t* bits = reinterpret_cast<uint32_t*>(smem + L.off_bits);
+    for (int j = tid; j < a.W; j += DEC_THREADS) {
+      const uint32_t sl = static_cast<uint32_t>(idx_w[j]);
+      atomicOr(&bits[(sl >> 5) & 63u], 1u << (sl & 31u));
+    }
+    for (int j = tid; j < a.R; j += DEC_THREADS) {
+      const uint32_t sl = static_cast<uint32_t>(idx_r[j]);
+      atomicOr(&bits[64 + ((sl >> 5) & 63u)], 1u << (sl & 31u));
+    }
+    __syncthreads();
+  }
 
   if (a.sel_out) {
     for (int j = tid; j < a.W; j += DEC_THREADS) a.sel_out[(size_t)bh * a.W + j] = idx_w[j];
@@ -350,99 +388,45 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
   }
 
   float* Mbh = a.M + (size_t)bh * a.N * a.d_v;
-  // the read rows go to L2 now, while the write rows are loaded and rewritten
-  {
-    const int lpr = (a.d_v + 31) / 32;  // 128-byte lines per row
-    for (int l = tid; l < a.R * lpr; l += DEC_THREADS) {
-      const int j = l / lpr;
-      const int sl = idx_r[j];
-      if (static_cast<unsigned>(sl) < static_cast<unsigned>(a.N))
-        prefetch_l2(Mbh + (size_t)sl * a.d_v + (l - j * lpr) * 32);
-    }
-  }
   const float al = ab[0], be = ab[1];
   float4 acc[NQ];
 #pragma unroll
   for (int q = 0; q < NQ; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-
-  // step 2: this warp's write rows (warp, warp + 8, ...), RB at a time: every row load is
-  // issued before any update, so a warp waits for one memory latency per RB rows
   constexpr int RB = NQ >= 8 ? 1 : 8 / NQ;
-  for (int j0 = warp; j0 < a.W; j0 += DEC_WARPS * RB) {
-    float4 old[RB][NQ];
-    int slot[RB];
-#pragma unroll
-    for (int r = 0; r < RB; ++r) {
-      const int j = j0 + r * DEC_WARPS;
-      slot[r] = j < a.W ? idx_w[j] : -1;
-      if (j < a.W && static_cast<unsigned>(slot[r]) < static_cast<unsigned>(a.N)) {
-        const float4* row = reinterpret_cast<const float4*>(Mbh + (size_t)slot[r] * a.d_v);
-#pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-          const int c = lane + 32 * q;
-          if (c < d4) old[r][q] = row[c];
-        }
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < RB; ++r) {
-      const int j = j0 + r * DEC_WARPS;
-      if (j >= a.W) continue;
-      if (static_cast<unsigned>(slot[r]) >= static_cast<unsigned>(a.N)) {
-        if (lane == 0) record_status(STATUS_BAD_INDEX);
-        continue;
-      }
-      // read weight of this slot if the token also reads it
-      int rpos = -1;
-      for (int e0 = 0; e0 < a.R; e0 += 32) {
-        const unsigned m = __ballot_sync(FULL_MASK, e0 + lane < a.R && idx_r[e0 + lane] == slot[r]);
-        if (m && rpos < 0) rpos = e0 + __ffs(m) - 1;
-      }
-      const float qr = rpos >= 0 ? wt_r[rpos] : 0.0f;
-      const float kb = be * wt_w[j];
-      const float ka = al * (1.0f - kb);
-      float4* row = reinterpret_cast<float4*>(Mbh + (size_t)slot[r] * a.d_v);
-      const float4* v4 = reinterpret_cast<const float4*>(vs);
+  float* wrow = reinterpret_cast<float*>(smem + L.off_rows);  // [W][d_v] when rows_smem
+  // 2048-bit filters of the write and the read slots: a clear bit rules a slot out
+  const uint32_t* wbits = reinterpret_cast<const uint32_t*>(smem + L.off_bits);
+  const uint32_t* rbits = wbits + 64;
+
+  // Every row load of the step is issued before any is used: this warp's write rows
+  // (warp, warp + 8, ...) go to shared memory by cp.async, its first RB read rows to
+  // registers.  A read row that the token also writes is loaded too but not used: its
+  // writer adds the new value (step 3 after step 2).
+  // the variant's largest write-row set (W <= KC, d_v <= 128 NQ) always fits shared memory
+  constexpr bool kRowsSmem = (size_t)KC * 128 * NQ * 4 <= DEC_ROWS_SMEM_MAX;
+  const bool rows_smem = kRowsSmem || L.rows_smem;
+  if (rows_smem) {
+    for (int j = warp; j < a.W; j += DEC_WARPS) {
+      const int sl = idx_w[j];
+      if (static_cast<unsigned>(sl) >= static_cast<unsigned>(a.N)) continue;
+      const float* src = Mbh + (size_t)sl * a.d_v;
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
         const int c = lane + 32 * q;
-        if (c < d4) {
-          const float4 vv = v4[c];
-          float4 nw;
-          nw.x = fmaf(ka, old[r][q].x, kb * vv.x);
-          nw.y = fmaf(ka, old[r][q].y, kb * vv.y);
-          nw.z = fmaf(ka, old[r][q].z, kb * vv.z);
-          nw.w = fmaf(ka, old[r][q].w, kb * vv.w);
-          row[c] = nw;
-          if (rpos >= 0) {
-            acc[q].x = fmaf(qr, nw.x, acc[q].x);
-            acc[q].y = fmaf(qr, nw.y, acc[q].y);
-            acc[q].z = fmaf(qr, nw.z, acc[q].z);
-            acc[q].w = fmaf(qr, nw.w, acc[q].w);
-          }
-        }
+        if (c < d4) cp_async16(wrow + (size_t)j * a.d_v + 4 * c, src + 4 * c);
       }
     }
+    cp_async_commit();
   }
-  // step 3 for the read rows this token does not write, RB at a time
-  for (int j0 = warp; j0 < a.R; j0 += DEC_WARPS * RB) {
-    float4 val[RB][NQ];
-    bool use[RB];
+  float4 val[RB][NQ];
+  int rslot[RB];
+  auto load_reads = [&](int j0) {
 #pragma unroll
     for (int r = 0; r < RB; ++r) {
       const int j = j0 + r * DEC_WARPS;
-      const int s = j < a.R ? idx_r[j] : -1;
-      bool in_w = false;
-      if (j < a.R)
-        for (int e = lane; e < a.W; e += 32) in_w |= (idx_w[e] == s);
-      in_w = __any_sync(FULL_MASK, in_w);
-      use[r] = j < a.R && !in_w;
-      if (use[r] && static_cast<unsigned>(s) >= static_cast<unsigned>(a.N)) {
-        if (lane == 0) record_status(STATUS_BAD_INDEX);
-        use[r] = false;
-      }
-      if (use[r]) {
-        const float4* row = reinterpret_cast<const float4*>(Mbh + (size_t)s * a.d_v);
+      rslot[r] = j < a.R ? idx_r[j] : -1;
+      if (static_cast<unsigned>(rslot[r]) < static_cast<unsigned>(a.N)) {
+        const float4* row = reinterpret_cast<const float4*>(Mbh + (size_t)rslot[r] * a.d_v);
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
           const int c = lane + 32 * q;
@@ -450,10 +434,24 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
         }
       }
     }
+  };
+  auto add_reads = [&](int j0) {
 #pragma unroll
     for (int r = 0; r < RB; ++r) {
-      if (!use[r]) continue;
-      const float q = wt_r[j0 + r * DEC_WARPS];
+      const int j = j0 + r * DEC_WARPS;
+      if (j >= a.R) continue;
+      if (static_cast<unsigned>(rslot[r]) >= static_cast<unsigned>(a.N)) {
+        if (lane == 0) record_status(STATUS_BAD_INDEX);
+        continue;
+      }
+      const uint32_t rs = static_cast<uint32_t>(rslot[r]);
+      if ((wbits[(rs >> 5) & 63u] >> (rs & 31u)) & 1u) {
+        // the filter admits the slot: an exact check against the write list
+        bool in_w = false;
+        for (int e = lane; e < a.W; e += 32) in_w |= (idx_w[e] == rslot[r]);
+        if (__any_sync(FULL_MASK, in_w)) continue;
+      }
+      const float q = wt_r[j];
 #pragma unroll
       for (int qq = 0; qq < NQ; ++qq) {
         const int c = lane + 32 * qq;
@@ -465,6 +463,98 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
         }
       }
     }
+  };
+  if (rows_smem) load_reads(warp);
+
+  // step 2 on one write row whose old value is `old`: store the new row, and add it to the
+  // read sum if the token also reads the slot
+  auto write_row = [&](int j, int sl, const float4 (&old)[NQ]) {
+    int rpos = -1;
+    const uint32_t us = static_cast<uint32_t>(sl);
+    if ((rbits[(us >> 5) & 63u] >> (us & 31u)) & 1u) {
+      for (int e0 = 0; e0 < a.R; e0 += 32) {
+        const unsigned m = __ballot_sync(FULL_MASK, e0 + lane < a.R && idx_r[e0 + lane] == sl);
+        if (m && rpos < 0) rpos = e0 + __ffs(m) - 1;
+      }
+    }
+    const float qr = rpos >= 0 ? wt_r[rpos] : 0.0f;
+    const float kb = be * wt_w[j];
+    const float ka = al * (1.0f - kb);
+    float4* row = reinterpret_cast<float4*>(Mbh + (size_t)sl * a.d_v);
+    const float4* v4 = reinterpret_cast<const float4*>(vs);
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      const int c = lane + 32 * q;
+      if (c < d4) {
+        const float4 vv = v4[c];
+        float4 nw;
+        nw.x = fmaf(ka, old[q].x, kb * vv.x);
+        nw.y = fmaf(ka, old[q].y, kb * vv.y);
+        nw.z = fmaf(ka, old[q].z, kb * vv.z);
+        nw.w = fmaf(ka, old[q].w, kb * vv.w);
+        row[c] = nw;
+        if (rpos >= 0) {
+          acc[q].x = fmaf(qr, nw.x, acc[q].x);
+          acc[q].y = fmaf(qr, nw.y, acc[q].y);
+          acc[q].z = fmaf(qr, nw.z, acc[q].z);
+          acc[q].w = fmaf(qr, nw.w, acc[q].w);
+        }
+      }
+    }
+  };
+  if (rows_smem) {
+    cp_async_wait<0>();  // this lane's own chunks: each lane rewrites exactly what it loaded
+    for (int j = warp; j < a.W; j += DEC_WARPS) {
+      const int sl = idx_w[j];
+      if (static_cast<unsigned>(sl) >= static_cast<unsigned>(a.N)) {
+        if (lane == 0) record_status(STATUS_BAD_INDEX);
+        continue;
+      }
+      float4 old[NQ];
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        const int c = lane + 32 * q;
+        old[q] = c < d4 ? reinterpret_cast<const float4*>(wrow + (size_t)j * a.d_v)[c]
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      write_row(j, sl, old);
+    }
+  } else {
+    // write rows through registers, RB at a time
+    for (int j0 = warp; j0 < a.W; j0 += DEC_WARPS * RB) {
+      float4 old[RB][NQ];
+      int slot[RB];
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+        const int j = j0 + r * DEC_WARPS;
+        slot[r] = j < a.W ? idx_w[j] : -1;
+        if (static_cast<unsigned>(slot[r]) < static_cast<unsigned>(a.N)) {
+          const float4* row = reinterpret_cast<const float4*>(Mbh + (size_t)slot[r] * a.d_v);
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) {
+            const int c = lane + 32 * q;
+            if (c < d4) old[r][q] = row[c];
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+        const int j = j0 + r * DEC_WARPS;
+        if (j >= a.W) continue;
+        if (static_cast<unsigned>(slot[r]) >= static_cast<unsigned>(a.N)) {
+          if (lane == 0) record_status(STATUS_BAD_INDEX);
+          continue;
+        }
+        write_row(j, slot[r], old[r]);
+      }
+    }
+    load_reads(warp);
+  }
+  // step 3 for the read rows this token does not write
+  add_reads(warp);
+  for (int j0 = warp + DEC_WARPS * RB; j0 < a.R; j0 += DEC_WARPS * RB) {
+    load_reads(j0);
+    add_reads(j0);
   }
 #pragma unroll
   for (int qq = 0; qq < NQ; ++qq) {

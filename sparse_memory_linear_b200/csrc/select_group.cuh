@@ -70,13 +70,19 @@ __device__ __forceinline__ void group_bracket(uint32_t vmax, uint32_t vlo, Group
   lo = max(lo, 1u);
 }
 
-// Step 1: a cut `lo` with need <= (keys >= lo) = n_ge, and n_ge <= cap unless a bin of
-// width one holds more.  Entry: at least `need` keys are >= lo, none is > hi, `hist` (256
-// words) is zero; it is zero again on return.
+// Outcome of step 1: keys >= cut are the n survivors.
+struct CutResult {
+  uint32_t cut;
+  int n;
+};
+
+// Step 1: a cut with need <= n, and n <= cap unless a bin of width one holds more.  Entry:
+// at least `need` keys are >= lo, none is > hi, `hist` (256 words) is zero; it is zero again
+// on return.
 template <int NK, int NT>
-__device__ __forceinline__ uint32_t group_cut(const uint32_t (&key)[NK], uint32_t lo,
-                                              uint32_t hi, int need, int cap, uint32_t* hist,
-                                              GroupCtl* ctl, int gt, int bar_id, int& n_ge) {
+__device__ __forceinline__ CutResult group_cut(const uint32_t (&key)[NK], uint32_t lo,
+                                               uint32_t hi, int need, int cap, uint32_t* hist,
+                                               GroupCtl* ctl, int gt, int bar_id) {
   int above = 0;  // keys > hi
   for (;;) {
     const uint32_t range = hi - lo;
@@ -88,15 +94,17 @@ __device__ __forceinline__ uint32_t group_cut(const uint32_t (&key)[NK], uint32_
     }
     group_bar(bar_id, NT);
     if (gt < 32) {
-      // lane l scans bins 255 - 8l down to 248 - 8l, then clears them for the next level
+      // lane l scans bins 255 - 8l down to 248 - 8l
       uint4* h4 = reinterpret_cast<uint4*>(hist);
       const uint4 hh = h4[63 - 2 * gt], hl = h4[62 - 2 * gt];
-      h4[63 - 2 * gt] = make_uint4(0u, 0u, 0u, 0u);
-      h4[62 - 2 * gt] = make_uint4(0u, 0u, 0u, 0u);
       const uint32_t c[8] = {hh.w, hh.z, hh.y, hh.x, hl.w, hl.z, hl.y, hl.x};
+      uint32_t pre[8];  // keys in this lane's bins above bin i
       uint32_t local = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) local += c[i];
+      for (int i = 0; i < 8; ++i) {
+        pre[i] = local;
+        local += c[i];
+      }
       uint32_t incl = local;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -105,20 +113,20 @@ __device__ __forceinline__ uint32_t group_cut(const uint32_t (&key)[NK], uint32_
       }
       const uint32_t excl = incl - local;
       const uint32_t want = static_cast<uint32_t>(need - above);
-      if (excl < want && want <= incl) {
-        uint32_t run = excl, cb = 0;
-        int bi = -1;
+      const bool crossing = excl < want && want <= incl;
+      uint32_t run = 0, cb = 0;
+      int bi = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if (bi < 0) {
-            if (run + c[i] >= want) {
-              bi = i;
-              cb = c[i];
-            } else {
-              run += c[i];
-            }
-          }
+      for (int i = 0; i < 8; ++i) {
+        if (excl + pre[i] < want && want <= excl + pre[i] + c[i]) {
+          bi = i;
+          run = excl + pre[i];
+          cb = c[i];
         }
+      }
+      h4[63 - 2 * gt] = make_uint4(0u, 0u, 0u, 0u);
+      h4[62 - 2 * gt] = make_uint4(0u, 0u, 0u, 0u);
+      if (crossing) {
         ctl->bin = static_cast<uint32_t>(255 - 8 * gt - bi);
         ctl->run = run;
         ctl->cnt_bin = cb;
@@ -127,22 +135,32 @@ __device__ __forceinline__ uint32_t group_cut(const uint32_t (&key)[NK], uint32_
     group_bar(bar_id, NT);
     const uint32_t b = ctl->bin;
     above += static_cast<int>(ctl->run);
-    n_ge = above + static_cast<int>(ctl->cnt_bin);
+    const int n_ge = above + static_cast<int>(ctl->cnt_bin);
     const uint32_t nlo = lo + (b << sh);
     const uint32_t span = (1u << sh) - 1u;
     hi = (hi - nlo > span) ? nlo + span : hi;
     lo = nlo;
-    if (n_ge <= cap || sh == 0) return lo;
+    if (n_ge <= cap || sh == 0) return CutResult{nlo, n_ge};
   }
 }
 
-// Step 2: appends comp(i) for every key[i] >= lo to list (any order; `counter` zero before).
-template <int NK, typename T, typename Comp>
-__device__ __forceinline__ void group_collect(const uint32_t (&key)[NK], uint32_t lo, Comp comp,
-                                              T* list, uint32_t* counter, int lane) {
+// Steps 2 and 3: the survivors of `cr` in selection order.  emit(r, comp) is called once per
+// survivor with its rank r (0 = first); ranks >= K are not part of the top K.  The
+// survivors are listed in any order, then each counts the listed survivors above it.
+// `list` holds cr.n + 4 entries; `counter` is zero on entry.
+template <int NK, int NT, typename T, typename Comp, typename Emit>
+__device__ __forceinline__ void group_order(const uint32_t (&key)[NK], const CutResult& cr,
+                                            Comp comp, T* list, uint32_t* counter, int gt,
+                                            int lane, int bar_id, Emit emit) {
+  // listed survivors, padded with zeros (below every composite) to a multiple of 4
+  if (gt == 0) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) list[(cr.n & ~3) + p] = T(0);
+  }
+  group_bar(bar_id, NT);  // the padding lands before any composite of the last quad
   int m = 0;
 #pragma unroll
-  for (int i = 0; i < NK; ++i) m += key[i] >= lo ? 1 : 0;
+  for (int i = 0; i < NK; ++i) m += key[i] >= cr.cut ? 1 : 0;
   int incl = m;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -155,43 +173,30 @@ __device__ __forceinline__ void group_collect(const uint32_t (&key)[NK], uint32_
   int pos = base + incl - m;
 #pragma unroll
   for (int i = 0; i < NK; ++i)
-    if (key[i] >= lo) list[pos++] = comp(i);
-}
-
-// Step 3 on 32-bit composites: list holds n distinct composites followed by zeros up to a
-// multiple of 4; out[r] = the composite of rank r, r < K.
-template <int NT>
-__device__ __forceinline__ void group_rank32(const uint32_t* list, int n, int K, int gt,
-                                             uint32_t* out) {
-  const uint4* l4 = reinterpret_cast<const uint4*>(list);
-  const int n4 = (n + 3) >> 2;
-  for (int j = gt; j < n; j += NT) {
-    const uint32_t c = list[j];
-    int r = 0;
+    if (key[i] >= cr.cut) list[pos++] = comp(i);
+  group_bar(bar_id, NT);
+  const int n4 = (cr.n + 3) >> 2;
+  for (int j = gt; j < cr.n; j += NT) {
+    const T x = list[j];
+    int r0 = 0, r1 = 0;
+    if constexpr (sizeof(T) == 4) {
+      const uint4* l4 = reinterpret_cast<const uint4*>(list);
 #pragma unroll 4
-    for (int i = 0; i < n4; ++i) {
-      const uint4 x = l4[i];
-      r += (x.x > c ? 1 : 0) + (x.y > c ? 1 : 0) + (x.z > c ? 1 : 0) + (x.w > c ? 1 : 0);
-    }
-    if (r < K) out[r] = c;
-  }
-}
-
-// Step 3 on 64-bit composites (list padded with zeros to an even length).  The caller gets
-// (rank, composite) pairs through `emit`.
-template <int NT, typename Emit>
-__device__ __forceinline__ void group_rank64(const uint64_t* list, int n, int gt, Emit emit) {
-  const ulonglong2* l2 = reinterpret_cast<const ulonglong2*>(list);
-  const int n2 = (n + 1) >> 1;
-  for (int j = gt; j < n; j += NT) {
-    const uint64_t c = list[j];
-    int r = 0;
+      for (int q = 0; q < n4; ++q) {
+        const uint4 y = l4[q];
+        r0 += (y.x > x ? 1 : 0) + (y.y > x ? 1 : 0);
+        r1 += (y.z > x ? 1 : 0) + (y.w > x ? 1 : 0);
+      }
+    } else {
+      const ulonglong2* l2 = reinterpret_cast<const ulonglong2*>(list);
 #pragma unroll 4
-    for (int i = 0; i < n2; ++i) {
-      const ulonglong2 x = l2[i];
-      r += (x.x > c ? 1 : 0) + (x.y > c ? 1 : 0);
+      for (int q = 0; q < 2 * n4; q += 2) {
+        const ulonglong2 y0 = l2[q], y1 = l2[q + 1];
+        r0 += (y0.x > x ? 1 : 0) + (y0.y > x ? 1 : 0);
+        r1 += (y1.x > x ? 1 : 0) + (y1.y > x ? 1 : 0);
+      }
     }
-    emit(r, c);
+    emit(r0 + r1, x);
   }
 }
 

@@ -241,27 +241,34 @@ def bench_prefill(args, dist: Dist, dev):
 
     th = wl.B * wl.T * wl.H
     value = weak_scaling_value(th * args.steps, secs, dist.world)
-    # per-kernel averages over the timed launches (events on the launching stream)
-    launches = {k: n for k, (ms, n) in prof.items() if n}
-    avg_ms = {k: ms / n for k, (ms, n) in prof.items() if n}
+    # per-kind device time per step and launches per step (events on the launching stream)
+    ms_step = {k: ms / args.steps for k, (ms, n) in prof.items() if n}
+    n_step = {k: n / args.steps for k, (ms, n) in prof.items() if n}
     scan_kind = "scan_slot" if prof["scan_slot"][1] else "scan_seq"
     peak, peak_kind = hbm_peak()
+    # the scan kernel runs once per time chunk (slot engine) or once per step: bytes per
+    # launch = the step's algorithmic bytes over its launches, duration = the average launch
     scan_bytes = th * scan_kernel_bytes(wl)
-    achieved = scan_bytes / (avg_ms[scan_kind] * 1e-3) / 1e9
+    per_launch_bytes = scan_bytes / n_step[scan_kind]
+    per_launch_ms = ms_step[scan_kind] / n_step[scan_kind]
+    achieved = per_launch_bytes / (per_launch_ms * 1e-3) / 1e9
     step_ms = secs / args.steps * 1e3
     res = {
         "value": value,
         "ms_per_step": step_ms,
         "clocks": clk.report(),
-        "kernels_avg_ms": avg_ms,
-        "kernels_share": {k: avg_ms[k] / sum(avg_ms.values()) for k in avg_ms},
+        "kernels_ms_per_step": ms_step,
+        "kernel_launches_per_step": n_step,
+        "kernels_share": {k: ms_step[k] / sum(ms_step.values()) for k in ms_step},
         "gpu_launches": int(launched),
         "roofline": {
-            "kernel": f"seq_scan_kernel" if scan_kind == "scan_seq" else "slot_scan_kernel",
+            "kernel": f"seq_scan_kernel" if scan_kind == "scan_seq" else "slot_chunk_kernel",
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_kind": f"{peak_kind} (burst copy)",
             "traffic": None,
-            "algorithmic_bytes_per_launch": scan_bytes,
+            "algorithmic_bytes_per_launch": per_launch_bytes,
+            "launch_ms": per_launch_ms,
+            "launches_per_step": n_step[scan_kind],
             "bytes_per_token_head": scan_kernel_bytes(wl),
         },
         "whole_step_hbm": {
@@ -494,7 +501,9 @@ def main(argv=None):
                        "l2": "inputs larger than L2 (9 GB of inputs, 4 GB state per step)",
                        "step": "sdm_scan_forward: M0 init + select + scan + norm/gate"},
             "roofline": pre["roofline"], "whole_step_hbm": pre["whole_step_hbm"],
-            "kernels_avg_ms": pre["kernels_avg_ms"], "kernels_share": pre["kernels_share"],
+            "kernels_ms_per_step": pre["kernels_ms_per_step"],
+            "kernel_launches_per_step": pre["kernel_launches_per_step"],
+            "kernels_share": pre["kernels_share"],
             "gpu_launches": pre["gpu_launches"], "clocks": pre["clocks"],
         }
         if "e2e" in pre:

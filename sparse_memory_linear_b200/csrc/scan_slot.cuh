@@ -53,29 +53,34 @@ struct EventArgs {
   const float* wt_w;
   const int32_t* idx_r;  // [rows, ldr]
   const float* wt_r;
-  uint32_t* keys;        // [rows * (W + R)]
+  uint32_t* keys;        // [chunk rows * (W + R)]
   uint2* vals;
-  float* y;              // [rows, d_v], zeroed here
-  uint32_t* counters;    // [2 * n_chunks], zeroed here
-  int B, T, H, N, W, R, ldw, ldr, d_v, chunk, n_chunks;
+  float* y;              // [rows, d_v]: the chunk's rows are zeroed here
+  uint32_t* offs;        // {0, events of the chunk}
+  uint32_t* counters;    // {long segments, span queue}, zeroed here
+  int B, T, H, N, W, R, ldw, ldr, d_v;
+  int t0, ct;            // the chunk: tokens [t0, t0 + ct)
   KeyBits kb;
 };
 
-// Event e = row * (W + R) + j: j < W is write j of the row, else read j - W.
-// val = {t << 8 | kind << 7 | j, weight bits}.
+// Events of one time chunk.  Chunk row r = (b * ct + tc) * H + h is token t0 + tc of
+// sequence b, head h; its event e = r * (W + R) + j: j < W is write j of the row, else
+// read j - W.  key = (b, h, slot) bit fields; val = {t << 8 | kind << 7 | j, weight bits}.
 __global__ void __launch_bounds__(256) slot_events_kernel(EventArgs a) {
-  const long long rows = (long long)a.B * a.T * a.H;
+  const long long crow = (long long)a.B * a.ct * a.H;
   const int per = a.W + a.R;
-  const long long n = rows * per;
+  const long long n = crow * per;
   const long long stride = (long long)gridDim.x * blockDim.x;
   const long long tid0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   for (long long e = tid0; e < n; e += stride) {
-    const long long row = e / per;
-    const int j = static_cast<int>(e - row * per);
-    const int h = static_cast<int>(row % a.H);
-    const long long bt = row / a.H;
-    const int t = static_cast<int>(bt % a.T);
-    const int b = static_cast<int>(bt / a.T);
+    const long long r = e / per;
+    const int j = static_cast<int>(e - r * per);
+    const int h = static_cast<int>(r % a.H);
+    const long long bt = r / a.H;
+    const int tc = static_cast<int>(bt % a.ct);
+    const int b = static_cast<int>(bt / a.ct);
+    const int t = a.t0 + tc;
+    const long long row = ((long long)b * a.T + t) * a.H + h;
     const bool rd = j >= a.W;
     const int jj = rd ? j - a.W : j;
     int slot = rd ? a.idx_r[row * a.ldr + jj] : a.idx_w[row * a.ldw + jj];
@@ -84,18 +89,24 @@ __global__ void __launch_bounds__(256) slot_events_kernel(EventArgs a) {
       record_status(STATUS_BAD_INDEX);
       slot = 0;
     }
-    const uint32_t c = static_cast<uint32_t>(t / a.chunk);
-    const uint32_t key = (((((c << a.kb.bbits) | (uint32_t)b) << a.kb.hbits) | (uint32_t)h)
-                          << a.kb.nbits) |
+    const uint32_t key = (((static_cast<uint32_t>(b) << a.kb.hbits) | (uint32_t)h) << a.kb.nbits) |
                          (uint32_t)slot;
     a.keys[e] = key;
     a.vals[e] = make_uint2((static_cast<uint32_t>(t) << 8) | (rd ? 128u : 0u) | jj,
                            __float_as_uint(w));
   }
-  const long long ny = rows * a.d_v / 4;
+  // the chunk's y rows: contiguous per sequence
+  const long long d4 = a.d_v / 4;
+  const long long ny = (long long)a.ct * a.H * d4;
   float4* y4 = reinterpret_cast<float4*>(a.y);
-  for (long long i = tid0; i < ny; i += stride) y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (long long i = tid0; i < 2LL * a.n_chunks; i += stride) a.counters[i] = 0u;
+  for (int b = 0; b < a.B; ++b) {
+    const long long base = ((long long)b * a.T + a.t0) * a.H * d4;
+    for (long long i = tid0; i < ny; i += stride) y4[base + i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  if (tid0 < 2) {
+    a.counters[tid0] = 0u;
+    a.offs[tid0] = tid0 == 0 ? 0u : static_cast<uint32_t>(n);
+  }
 }
 
 // --------------------------------------------------------------------- radix sort
@@ -215,26 +226,6 @@ __global__ void __launch_bounds__(RS_THREADS) radix_scatter_kernel(
       vout[pos] = vin[i];
     }
   }
-}
-
-// First event of every chunk in the sorted keys (binary search); offs[n_chunks] = n.
-__global__ void slot_chunk_offsets_kernel(const uint32_t* __restrict__ keys, long long n,
-                                          int n_chunks, int chunk_shift,
-                                          uint32_t* __restrict__ offs) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c > n_chunks) return;
-  if (c == n_chunks) {
-    offs[c] = static_cast<uint32_t>(n);
-    return;
-  }
-  const unsigned long long target = (unsigned long long)c << chunk_shift;
-  long long lo = 0, hi = n;
-  while (lo < hi) {
-    const long long mid = (lo + hi) >> 1;
-    if ((unsigned long long)keys[mid] < target) lo = mid + 1;
-    else hi = mid;
-  }
-  offs[c] = static_cast<uint32_t>(lo);
 }
 
 // Segments of at least SLOT_LONG events: listed per chunk as {first event, length}.

@@ -186,14 +186,14 @@ WsLayout ws_layout(const sdm_shape& s, int engine) {
   L.total = round_up(L.off_wt_r + rows * L.ldr * 4, WS_ALIGN);
   L.chunk = slot_chunk_tokens(s);
   L.n_chunks = s.T > 0 ? (s.T + L.chunk - 1) / L.chunk : 0;
-  L.events = (long long)rows * (s.W + s.R);
+  // events and their sort buffers hold one time chunk at a time
+  L.events = (long long)L.chunk * s.B * s.H * (s.W + s.R);
   L.ntiles = (int)((L.events + RS_TILE - 1) / RS_TILE);
   L.kb.nbits = bits_for((long long)s.S1 * s.S2);
   L.kb.hbits = bits_for(s.H);
   L.kb.bbits = bits_for(s.B);
-  L.kb.cbits = bits_for(L.n_chunks > 0 ? L.n_chunks : 1);
-  const long long chunk_events = (long long)L.chunk * s.B * s.H * (s.W + s.R);
-  L.hot_cap = (int)(chunk_events / SLOT_LONG + 1);
+  L.kb.cbits = 0;
+  L.hot_cap = (int)(L.events / SLOT_LONG + 1);
   L.off_k0 = L.off_k1 = L.off_v0 = L.off_v1 = L.off_hist = L.off_tot = L.off_offs = 0;
   L.off_cnt = L.off_hot = 0;
   if (engine == SDM_ENGINE_SLOT) {
@@ -205,15 +205,15 @@ WsLayout ws_layout(const sdm_shape& s, int engine) {
     L.off_hist = round_up(L.off_v1 + E * 8, WS_ALIGN);
     L.off_tot = round_up(L.off_hist + (size_t)RS_BINS * L.ntiles * 4, WS_ALIGN);
     L.off_offs = round_up(L.off_tot + RS_BINS * 4, WS_ALIGN);
-    L.off_cnt = round_up(L.off_offs + ((size_t)L.n_chunks + 1) * 4, WS_ALIGN);
-    L.off_hot = round_up(L.off_cnt + (size_t)2 * L.n_chunks * 4, WS_ALIGN);
-    L.total = round_up(L.off_hot + (size_t)L.n_chunks * L.hot_cap * 8, WS_ALIGN);
+    L.off_cnt = round_up(L.off_offs + 2 * 4, WS_ALIGN);
+    L.off_hot = round_up(L.off_cnt + 2 * 4, WS_ALIGN);
+    L.total = round_up(L.off_hot + (size_t)L.hot_cap * 8, WS_ALIGN);
   }
   return L;
 }
 
-// The slot engine packs (chunk, sequence, head, slot) into 31 bits of a key and counts
-// events and state rows in 32 bits.
+// The slot engine packs (sequence, head, slot) into 31 bits of a key and counts a chunk's
+// events and the state rows in 32 bits.
 bool slot_engine_fits(const sdm_shape& s) {
   const WsLayout L = ws_layout(s, SDM_ENGINE_SEQ);
   const long long rows = (long long)s.B * s.T * s.H;
@@ -394,23 +394,21 @@ sdm_status launch_state_init(const float* M0, float* M, const sdm_shape& s, cuda
 }
 
 template <int NQ, int G, int PF>
-sdm_status launch_slot_chunks(const SlotArgs& a, int n_chunks, const DeviceInfo* di,
-                              cudaStream_t st) {
+sdm_status launch_slot_chunk(const SlotArgs& a, const DeviceInfo* di, cudaStream_t st) {
   const size_t smem = SLOT_WARPS * slot_warp_smem(NQ, PF);
   int per_sm = 0;
   SDM_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
       &per_sm, slot_chunk_kernel<NQ, G, PF>, SLOT_THREADS, smem));
   const int grid = di->sms * (per_sm > 0 ? per_sm : 1);
-  for (int c = 0; c < n_chunks; ++c) {
-    slot_chunk_kernel<NQ, G, PF><<<grid, SLOT_THREADS, smem, st>>>(a, c);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    SDM_CUDA_TRY(cudaGetLastError());
-  }
+  slot_chunk_kernel<NQ, G, PF><<<grid, SLOT_THREADS, smem, st>>>(a, 0);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  SDM_CUDA_TRY(cudaGetLastError());
   return SDM_OK;
 }
 
-// Steps 2-3 with the slot-parallel engine: events, radix sort, chunk offsets, long segments,
-// then one launch per time chunk.
+// Steps 2-3 with the slot-parallel engine, one time chunk after another: the chunk's
+// events, their radix sort by (sequence, head, slot), its long segments, then the chunk's
+// segments.  A chunk's events and sort buffers (tens of MB) stay in L2 between the steps.
 sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
                        const float* alpha, const float* beta, const void* v, float* M, float* y,
                        const DeviceInfo* di, cudaStream_t st) {
@@ -421,67 +419,17 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
   uint32_t* hist = reinterpret_cast<uint32_t*>(w + WL.off_hist);
   uint32_t* tot = reinterpret_cast<uint32_t*>(w + WL.off_tot);
   uint32_t* offs = reinterpret_cast<uint32_t*>(w + WL.off_offs);
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(w + WL.off_cnt);  // hot counts | span queues
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(w + WL.off_cnt);  // hot count | span queue
   uint2* hot = reinterpret_cast<uint2*>(w + WL.off_hot);
-  const long long E = WL.events;
   const int N = s.S1 * s.S2;
-  {
-    ProfScope ps(SDM_KERNEL_SLOT_SORT, st);
-    EventArgs ea;
-    ea.idx_w = reinterpret_cast<const int32_t*>(w + WL.off_idx_w);
-    ea.wt_w = reinterpret_cast<const float*>(w + WL.off_wt_w);
-    ea.idx_r = reinterpret_cast<const int32_t*>(w + WL.off_idx_r);
-    ea.wt_r = reinterpret_cast<const float*>(w + WL.off_wt_r);
-    ea.keys = k0;
-    ea.vals = v0;
-    ea.y = y;
-    ea.counters = cnt;
-    ea.B = s.B;
-    ea.T = s.T;
-    ea.H = s.H;
-    ea.N = N;
-    ea.W = s.W;
-    ea.R = s.R;
-    ea.ldw = WL.ldw;
-    ea.ldr = WL.ldr;
-    ea.d_v = s.d_v;
-    ea.chunk = WL.chunk;
-    ea.n_chunks = WL.n_chunks;
-    ea.kb = WL.kb;
-    long long blocks = (E + 255) / 256;
-    if (blocks > (long long)di->sms * 16) blocks = (long long)di->sms * 16;
-    slot_events_kernel<<<(unsigned)blocks, 256, 0, st>>>(ea);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    SDM_CUDA_TRY(cudaGetLastError());
-    // LSD radix sort over the key bits in use
-    const int bits = WL.kb.total();
-    for (int shift = 0; shift < bits; shift += 8) {
-      radix_hist_kernel<<<WL.ntiles, RS_THREADS, 0, st>>>(k0, E, shift, hist, WL.ntiles);
-      radix_scan_kernel<<<RS_BINS, 1024, 0, st>>>(hist, WL.ntiles, tot);
-      radix_scatter_kernel<<<WL.ntiles, RS_THREADS, 0, st>>>(k0, v0, k1, v1, E, shift, hist, tot,
-                                                            WL.ntiles);
-      g_launches.fetch_add(3, std::memory_order_relaxed);
-      SDM_CUDA_TRY(cudaGetLastError());
-      uint32_t* tk = k0;
-      k0 = k1;
-      k1 = tk;
-      uint2* tv = v0;
-      v0 = v1;
-      v1 = tv;
-    }
-    slot_chunk_offsets_kernel<<<(WL.n_chunks + 1 + 127) / 128, 128, 0, st>>>(
-        k0, E, WL.n_chunks, WL.kb.chunk_shift(), offs);
-    long long lblocks = (E / 32 + 7) / 8;
-    if (lblocks > (long long)di->sms * 8) lblocks = (long long)di->sms * 8;
-    if (lblocks < 1) lblocks = 1;
-    slot_long_segments_kernel<<<(unsigned)lblocks, 256, 0, st>>>(k0, E, WL.kb.chunk_shift(), cnt,
-                                                                 hot, WL.hot_cap);
-    g_launches.fetch_add(2, std::memory_order_relaxed);
-    SDM_CUDA_TRY(cudaGetLastError());
-  }
+  const int bits = WL.kb.total();
+  // an even number of passes leaves the sorted events in k0 / v0
+  const int passes = (bits + 7) / 8;
+  uint32_t* ks = passes % 2 ? k1 : k0;
+  uint2* vs = passes % 2 ? v1 : v0;
   SlotArgs a;
-  a.keys = k0;
-  a.vals = v0;
+  a.keys = ks;
+  a.vals = vs;
   a.offs = offs;
   a.alpha = alpha;
   a.beta = beta;
@@ -490,7 +438,7 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
   a.y = y;
   a.hot_count = cnt;
   a.hot_list = hot;
-  a.span_next = cnt + WL.n_chunks;
+  a.span_next = cnt + 1;
   a.hot_cap = WL.hot_cap;
   a.B = s.B;
   a.T = s.T;
@@ -499,12 +447,76 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
   a.d_v = s.d_v;
   a.v_bf16 = s.in_dtype == SDM_BF16;
   a.kb = WL.kb;
-  ProfScope ps(SDM_KERNEL_SCAN_SLOT, st);
   const int d4 = s.d_v / 4;
-  if (d4 <= 32) return launch_slot_chunks<1, 8, 8>(a, WL.n_chunks, di, st);
-  if (d4 <= 64) return launch_slot_chunks<2, 2, 8>(a, WL.n_chunks, di, st);
-  if (d4 <= 128) return launch_slot_chunks<4, 4, 4>(a, WL.n_chunks, di, st);
-  return launch_slot_chunks<8, 2, 2>(a, WL.n_chunks, di, st);
+  for (int t0 = 0; t0 < s.T; t0 += WL.chunk) {
+    const int ct = s.T - t0 < WL.chunk ? s.T - t0 : WL.chunk;
+    const long long E = (long long)ct * s.B * s.H * (s.W + s.R);
+    const int ntiles = (int)((E + RS_TILE - 1) / RS_TILE);
+    {
+      ProfScope ps(SDM_KERNEL_SLOT_SORT, st);
+      EventArgs ea;
+      ea.idx_w = reinterpret_cast<const int32_t*>(w + WL.off_idx_w);
+      ea.wt_w = reinterpret_cast<const float*>(w + WL.off_wt_w);
+      ea.idx_r = reinterpret_cast<const int32_t*>(w + WL.off_idx_r);
+      ea.wt_r = reinterpret_cast<const float*>(w + WL.off_wt_r);
+      ea.keys = k0;
+      ea.vals = v0;
+      ea.y = y;
+      ea.offs = offs;
+      ea.counters = cnt;
+      ea.B = s.B;
+      ea.T = s.T;
+      ea.H = s.H;
+      ea.N = N;
+      ea.W = s.W;
+      ea.R = s.R;
+      ea.ldw = WL.ldw;
+      ea.ldr = WL.ldr;
+      ea.d_v = s.d_v;
+      ea.t0 = t0;
+      ea.ct = ct;
+      ea.kb = WL.kb;
+      long long blocks = (E + 255) / 256;
+      if (blocks > (long long)di->sms * 16) blocks = (long long)di->sms * 16;
+      slot_events_kernel<<<(unsigned)blocks, 256, 0, st>>>(ea);
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+      SDM_CUDA_TRY(cudaGetLastError());
+      // LSD radix sort over the key bits in use
+      uint32_t* ka = k0;
+      uint32_t* kb = k1;
+      uint2* va = v0;
+      uint2* vb = v1;
+      for (int shift = 0; shift < bits; shift += 8) {
+        radix_hist_kernel<<<ntiles, RS_THREADS, 0, st>>>(ka, E, shift, hist, ntiles);
+        radix_scan_kernel<<<RS_BINS, 1024, 0, st>>>(hist, ntiles, tot);
+        radix_scatter_kernel<<<ntiles, RS_THREADS, 0, st>>>(ka, va, kb, vb, E, shift, hist, tot,
+                                                            ntiles);
+        g_launches.fetch_add(3, std::memory_order_relaxed);
+        SDM_CUDA_TRY(cudaGetLastError());
+        uint32_t* tk = ka;
+        ka = kb;
+        kb = tk;
+        uint2* tv = va;
+        va = vb;
+        vb = tv;
+      }
+      long long lblocks = (E / 32 + 7) / 8;
+      if (lblocks > (long long)di->sms * 8) lblocks = (long long)di->sms * 8;
+      if (lblocks < 1) lblocks = 1;
+      slot_long_segments_kernel<<<(unsigned)lblocks, 256, 0, st>>>(ks, E, bits, cnt, hot,
+                                                                   WL.hot_cap);
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+      SDM_CUDA_TRY(cudaGetLastError());
+    }
+    ProfScope ps(SDM_KERNEL_SCAN_SLOT, st);
+    sdm_status rc;
+    if (d4 <= 32) rc = launch_slot_chunk<1, 8, 8>(a, di, st);
+    else if (d4 <= 64) rc = launch_slot_chunk<2, 2, 8>(a, di, st);
+    else if (d4 <= 128) rc = launch_slot_chunk<4, 4, 4>(a, di, st);
+    else rc = launch_slot_chunk<8, 2, 2>(a, di, st);
+    if (rc != SDM_OK) return rc;
+  }
+  return SDM_OK;
 }
 
 bool act_ok(int act) { return act >= SDM_GATE_SILU && act <= SDM_GATE_IDENTITY; }

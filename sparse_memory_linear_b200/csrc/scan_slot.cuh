@@ -63,39 +63,47 @@ struct EventArgs {
   KeyBits kb;
 };
 
-// Events of one time chunk.  Chunk row r = (b * ct + tc) * H + h is token t0 + tc of
-// sequence b, head h; its event e = r * (W + R) + j: j < W is write j of the row, else
-// read j - W.  key = (b, h, slot) bit fields; val = {t << 8 | kind << 7 | j, weight bits}.
+// Events of one time chunk, one warp per chunk row.  Chunk row r = (b * ct + tc) * H + h is
+// token t0 + tc of sequence b, head h; its event e = r * (W + R) + j: j < W is write j of
+// the row, else read j - W.  key = (b, h, slot) bit fields; val = {t << 8 | kind << 7 | j,
+// weight bits}.
 __global__ void __launch_bounds__(256) slot_events_kernel(EventArgs a) {
+  const int lane = threadIdx.x & 31;
   const long long crow = (long long)a.B * a.ct * a.H;
   const int per = a.W + a.R;
-  const long long n = crow * per;
-  const long long stride = (long long)gridDim.x * blockDim.x;
-  const long long tid0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  for (long long e = tid0; e < n; e += stride) {
-    const long long r = e / per;
-    const int j = static_cast<int>(e - r * per);
+  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long r = gw; r < crow; r += nw) {
     const int h = static_cast<int>(r % a.H);
     const long long bt = r / a.H;
     const int tc = static_cast<int>(bt % a.ct);
     const int b = static_cast<int>(bt / a.ct);
     const int t = a.t0 + tc;
     const long long row = ((long long)b * a.T + t) * a.H + h;
-    const bool rd = j >= a.W;
-    const int jj = rd ? j - a.W : j;
-    int slot = rd ? a.idx_r[row * a.ldr + jj] : a.idx_w[row * a.ldw + jj];
-    const float w = rd ? a.wt_r[row * a.ldr + jj] : a.wt_w[row * a.ldw + jj];
-    if (static_cast<unsigned>(slot) >= static_cast<unsigned>(a.N)) {
-      record_status(STATUS_BAD_INDEX);
-      slot = 0;
-    }
-    const uint32_t key = (((static_cast<uint32_t>(b) << a.kb.hbits) | (uint32_t)h) << a.kb.nbits) |
-                         (uint32_t)slot;
-    a.keys[e] = key;
-    a.vals[e] = make_uint2((static_cast<uint32_t>(t) << 8) | (rd ? 128u : 0u) | jj,
+    const uint32_t kbase = ((static_cast<uint32_t>(b) << a.kb.hbits) | (uint32_t)h) << a.kb.nbits;
+    const int32_t* iw = a.idx_w + row * a.ldw;
+    const float* ww = a.wt_w + row * a.ldw;
+    const int32_t* ir = a.idx_r + row * a.ldr;
+    const float* wr = a.wt_r + row * a.ldr;
+    uint32_t* keys = a.keys + r * per;
+    uint2* vals = a.vals + r * per;
+    for (int j = lane; j < per; j += 32) {
+      const bool rd = j >= a.W;
+      const int jj = rd ? j - a.W : j;
+      int slot = rd ? ir[jj] : iw[jj];
+      const float w = rd ? wr[jj] : ww[jj];
+      if (static_cast<unsigned>(slot) >= static_cast<unsigned>(a.N)) {
+        record_status(STATUS_BAD_INDEX);
+        slot = 0;
+      }
+      keys[j] = kbase | (uint32_t)slot;
+      vals[j] = make_uint2((static_cast<uint32_t>(t) << 8) | (rd ? 128u : 0u) | jj,
                            __float_as_uint(w));
+    }
   }
   // the chunk's y rows: contiguous per sequence
+  const long long tid0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long stride = (long long)gridDim.x * blockDim.x;
   const long long d4 = a.d_v / 4;
   const long long ny = (long long)a.ct * a.H * d4;
   float4* y4 = reinterpret_cast<float4*>(a.y);
@@ -105,7 +113,7 @@ __global__ void __launch_bounds__(256) slot_events_kernel(EventArgs a) {
   }
   if (tid0 < 2) {
     a.counters[tid0] = 0u;
-    a.offs[tid0] = tid0 == 0 ? 0u : static_cast<uint32_t>(n);
+    a.offs[tid0] = tid0 == 0 ? 0u : static_cast<uint32_t>(crow * per);
   }
 }
 
@@ -161,40 +169,67 @@ __global__ void __launch_bounds__(1024) radix_scan_kernel(uint32_t* __restrict__
   if (tid == 1023) totals[d] = part[1023];
 }
 
-// Stable scatter of one digit: every tile ranks its items in order (warp by warp, 32
-// items at a time, peers found with match.any), then writes them at
-// digit_base + tile_prefix + rank.
+// Exclusive prefix sum of one value per thread over a CTA of RS_THREADS threads (warp
+// shuffles, one exchange through shared memory); `tot` receives the CTA total.
+__device__ __forceinline__ uint32_t rs_block_excl(uint32_t v, uint32_t* warp_tot, uint32_t& tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(FULL_MASK, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  uint32_t before = 0;
+  tot = 0;
+#pragma unroll
+  for (int w = 0; w < RS_WARPS; ++w) {
+    const uint32_t c = warp_tot[w];
+    before += w < warp ? c : 0u;
+    tot += c;
+  }
+  return before + incl - v;
+}
+
+// Stable scatter of one digit.  Every tile ranks its items in order (warp by warp, 32 items
+// at a time, peers found with match.any) and places their keys and tile positions in shared
+// memory in digit order; then each digit's run is written to digit_base + tile_prefix, the
+// values gathered from the tile by their staged positions: consecutive threads write
+// consecutive addresses of one run.
+constexpr size_t RS_SCATTER_SMEM = (size_t)RS_TILE * 6;  // staged keys and tile positions
+
 __global__ void __launch_bounds__(RS_THREADS) radix_scatter_kernel(
     const uint32_t* __restrict__ kin, const uint2* __restrict__ vin, uint32_t* __restrict__ kout,
     uint2* __restrict__ vout, long long n, int shift, const uint32_t* __restrict__ hist,
     const uint32_t* __restrict__ totals, int ntiles) {
+  extern __shared__ __align__(16) unsigned char rs_smem[];
+  uint32_t* skey = reinterpret_cast<uint32_t*>(rs_smem);                        // [RS_TILE]
+  uint16_t* sidx = reinterpret_cast<uint16_t*>(rs_smem + (size_t)RS_TILE * 4);  // [RS_TILE]
   __shared__ uint32_t wcnt[RS_WARPS][RS_BINS];
-  __shared__ uint32_t dbase[RS_BINS];
+  __shared__ uint32_t dbase[RS_BINS];  // global position of the tile's first item of a digit
+  __shared__ uint32_t lbase[RS_BINS];  // staged position of the tile's first item of a digit
+  __shared__ uint32_t wtot[2][RS_WARPS];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int i = tid; i < RS_WARPS * RS_BINS; i += RS_THREADS) (&wcnt[0][0])[i] = 0u;
-  // digit bases: exclusive prefix of the totals (one digit per thread)
-  {
-    __shared__ uint32_t sc[RS_BINS];
-    sc[tid] = totals[tid];
-    __syncthreads();
-    for (int o = 1; o < RS_BINS; o <<= 1) {
-      const uint32_t v = tid >= o ? sc[tid - o] : 0u;
-      __syncthreads();
-      sc[tid] += v;
-      __syncthreads();
-    }
-    dbase[tid] = sc[tid] - totals[tid] + hist[(size_t)tid * ntiles + blockIdx.x];
-  }
-  __syncthreads();
-  const long long base = (long long)blockIdx.x * RS_TILE + (long long)warp * (RS_TILE / RS_WARPS);
-  const unsigned lt = lanemask_lt();
+  const long long tile0 = (long long)blockIdx.x * RS_TILE;
+  const long long base = tile0 + (long long)warp * (RS_TILE / RS_WARPS);
+  // this thread's keys and its digit's counts, loads first
   uint32_t key[RS_IPT];
+#pragma unroll
+  for (int r = 0; r < RS_IPT; ++r) {
+    const long long i = base + r * 32 + lane;
+    key[r] = i < n ? kin[i] : 0u;
+  }
+  const uint32_t my_total = totals[tid];
+  const uint32_t my_prefix = hist[(size_t)tid * ntiles + blockIdx.x];
+  for (int i = tid; i < RS_WARPS * RS_BINS; i += RS_THREADS) (&wcnt[0][0])[i] = 0u;
+  __syncthreads();
+  const unsigned lt = lanemask_lt();
   uint32_t rank[RS_IPT];
 #pragma unroll
   for (int r = 0; r < RS_IPT; ++r) {
     const long long i = base + r * 32 + lane;
     const bool ok = i < n;
-    key[r] = ok ? kin[i] : 0u;
     const uint32_t d = ok ? ((key[r] >> shift) & 255u) : (256u + lane);
     const unsigned m = __match_any_sync(FULL_MASK, d);
     uint32_t before = 0;
@@ -205,68 +240,81 @@ __global__ void __launch_bounds__(RS_THREADS) radix_scatter_kernel(
     __syncwarp();
   }
   __syncthreads();
-  // per digit: the counts of the warps before this one
-  {
-    uint32_t run = 0;
+  // per digit (one per thread): the counts of the warps before each warp, the tile's count
+  uint32_t run = 0;
 #pragma unroll
-    for (int w = 0; w < RS_WARPS; ++w) {
-      const uint32_t c = wcnt[w][tid];
-      wcnt[w][tid] = run;
-      run += c;
-    }
+  for (int w = 0; w < RS_WARPS; ++w) {
+    const uint32_t c = wcnt[w][tid];
+    wcnt[w][tid] = run;
+    run += c;
   }
+  uint32_t all;
+  dbase[tid] = rs_block_excl(my_total, wtot[0], all) + my_prefix;
+  lbase[tid] = rs_block_excl(run, wtot[1], all);
   __syncthreads();
 #pragma unroll
   for (int r = 0; r < RS_IPT; ++r) {
     const long long i = base + r * 32 + lane;
     if (i < n) {
       const uint32_t d = (key[r] >> shift) & 255u;
-      const uint32_t pos = dbase[d] + wcnt[warp][d] + rank[r];
-      kout[pos] = key[r];
-      vout[pos] = vin[i];
+      const uint32_t lp = lbase[d] + wcnt[warp][d] + rank[r];
+      skey[lp] = key[r];
+      sidx[lp] = static_cast<uint16_t>(i - tile0);
     }
+  }
+  __syncthreads();
+  const int tn = static_cast<int>(min((long long)RS_TILE, n - tile0));
+  for (int i = tid; i < tn; i += RS_THREADS) {
+    const uint32_t k = skey[i];
+    const uint32_t d = (k >> shift) & 255u;
+    const uint32_t pos = dbase[d] + (static_cast<uint32_t>(i) - lbase[d]);
+    kout[pos] = k;
+    vout[pos] = vin[tile0 + sidx[i]];
   }
 }
 
-// Segments of at least SLOT_LONG events: listed per chunk as {first event, length}.
+// Segments of at least SLOT_LONG events, listed as {first event, length}.  Any such segment
+// holds two events 128 apart at a multiple of 128, p and p + 128 (its first 256 events
+// contain a multiple of 128 no later than its 128th): one thread per multiple of 128 tests
+// that pair and reports the segment only from the first multiple of 128 inside it, after
+// finding its two ends by binary searches.
 __global__ void __launch_bounds__(256) slot_long_segments_kernel(
-    const uint32_t* __restrict__ keys, long long n, int chunk_shift, uint32_t* hot_count,
-    uint2* hot_list, int hot_cap) {
-  const int lane = threadIdx.x & 31;
-  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
-  for (long long tile = gw * 32; tile < n; tile += nw * 32) {
-    const long long e = tile + lane;
-    const uint32_t k = e < n ? keys[e] : EV_SENTINEL;
-    uint32_t kprev = __shfl_up_sync(FULL_MASK, k, 1);
-    if (lane == 0) kprev = tile > 0 ? keys[tile - 1] : EV_SENTINEL;
-    const bool head = e < n && k != kprev;
-    const bool is_long = head && e + SLOT_LONG - 1 < n && keys[e + SLOT_LONG - 1] == k;
-    unsigned lm = __ballot_sync(FULL_MASK, is_long);
-    while (lm) {
-      const int hl = __ffs(lm) - 1;
-      lm &= lm - 1;
-      const long long first = tile + hl;
-      const uint32_t K = __shfl_sync(FULL_MASK, k, hl);
-      long long end = first + SLOT_LONG;
-      while (true) {
-        const long long ej = end + lane;
-        const bool same = ej < n && keys[ej] == K;
-        const unsigned m = __ballot_sync(FULL_MASK, same);
-        if (m == FULL_MASK) {
-          end += 32;
-          continue;
-        }
-        end += __ffs(~m) - 1;
-        break;
-      }
-      if (lane == 0) {
-        const uint32_t c = K >> chunk_shift;
-        const uint32_t pos = atomicAdd(&hot_count[c], 1u);
-        if (pos < (uint32_t)hot_cap)
-          hot_list[(size_t)c * hot_cap + pos] =
-              make_uint2(static_cast<uint32_t>(first), static_cast<uint32_t>(end - first));
-      }
+    const uint32_t* __restrict__ keys, long long n, uint32_t* hot_count, uint2* hot_list,
+    int hot_cap) {
+  static_assert(SLOT_LONG >= 256, "two samples 128 apart must fit in a long segment");
+  const long long nsamp = (n + 127) / 128;
+  for (long long si = (long long)blockIdx.x * blockDim.x + threadIdx.x; si < nsamp;
+       si += (long long)gridDim.x * blockDim.x) {
+    const long long p = si * 128;
+    if (p + 128 >= n) continue;
+    const uint32_t K = keys[p];
+    if (keys[p + 128] != K) continue;
+    if (p >= 128 && keys[p - 128] == K) continue;  // an earlier sample lies in the segment
+    // first event: in (p - 128, p]
+    long long lo = p >= 127 ? p - 127 : 0, hi = p;  // keys[hi] == K
+    while (lo < hi) {
+      const long long mid = (lo + hi) >> 1;
+      if (keys[mid] == K) hi = mid;
+      else lo = mid + 1;
+    }
+    const long long first = lo;
+    // one past the last event: gallop from p + 128, then bisect
+    long long good = p + 128, step = 128;
+    while (good + step < n && keys[good + step] == K) {
+      good += step;
+      step *= 2;
+    }
+    long long bad = good + step < n ? good + step : n;  // keys[bad] != K or bad == n
+    while (bad - good > 1) {
+      const long long mid = (good + bad) >> 1;
+      if (keys[mid] == K) good = mid;
+      else bad = mid;
+    }
+    const long long len = bad - first;
+    if (len >= SLOT_LONG) {
+      const uint32_t pos = atomicAdd(hot_count, 1u);
+      if (pos < (uint32_t)hot_cap)
+        hot_list[pos] = make_uint2(static_cast<uint32_t>(first), static_cast<uint32_t>(len));
     }
   }
 }

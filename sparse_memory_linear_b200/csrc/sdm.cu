@@ -84,6 +84,9 @@ sdm_status device_info(DeviceInfo** out) {
     SDM_SEQ_ATTR(4, 4) SDM_SEQ_ATTR(4, 8) SDM_SEQ_ATTR(8, 4) SDM_SEQ_ATTR(8, 8)
     SDM_SEQ_ATTR(16, 4) SDM_SEQ_ATTR(16, 8) SDM_SEQ_ATTR(32, 4) SDM_SEQ_ATTR(32, 8)
 #undef SDM_SEQ_ATTR
+    SDM_CUDA_TRY(cudaFuncSetAttribute(radix_scatter_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)RS_SCATTER_SMEM));
 #define SDM_SLOT_ATTR(NQ, G, PF) \
   SDM_CUDA_TRY(allow_max_dynamic_smem(slot_chunk_kernel<NQ, G, PF>, m));
     SDM_SLOT_ATTR(1, 8, 8) SDM_SLOT_ATTR(2, 2, 8) SDM_SLOT_ATTR(4, 4, 4) SDM_SLOT_ATTR(8, 2, 2)
@@ -253,6 +256,8 @@ sdm_status launch_select_fast_t(const SelJob& j0, const SelJob* j1, long long ro
                                                              warps * 32, smem));
   if (per_sm < 1) return SDM_ERR_UNSUPPORTED;
   const long long total_rows = rows * (j1 ? 2 : 1);
+  const int cap = env_int("SDM_SEL_CTAS", 0);
+  if (cap > 0 && cap < per_sm) per_sm = cap;
   long long grid = (long long)di->sms * per_sm;
   const long long need = (total_rows + warps - 1) / warps;
   if (grid > need) grid = need;
@@ -299,6 +304,8 @@ sdm_status launch_select(const SelJob& j0, const SelJob* j1, long long rows, int
   SDM_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sel_kernel, warps * 32, smem));
   if (per_sm < 1) return SDM_ERR_UNSUPPORTED;
   const long long total_rows = rows * (j1 ? 2 : 1);
+  const int cap = env_int("SDM_SEL_CTAS", 0);
+  if (cap > 0 && cap < per_sm) per_sm = cap;
   long long grid = (long long)di->sms * per_sm;
   const long long need = (total_rows + warps - 1) / warps;
   if (grid > need) grid = need;
@@ -399,7 +406,10 @@ sdm_status launch_slot_chunk(const SlotArgs& a, const DeviceInfo* di, cudaStream
   int per_sm = 0;
   SDM_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
       &per_sm, slot_chunk_kernel<NQ, G, PF>, SLOT_THREADS, smem));
-  const int grid = di->sms * (per_sm > 0 ? per_sm : 1);
+  int ctas = per_sm > 0 ? per_sm : 1;
+  const int cap = env_int("SDM_SLOT_CTAS", 0);
+  if (cap > 0 && cap < ctas) ctas = cap;
+  const int grid = di->sms * ctas;
   slot_chunk_kernel<NQ, G, PF><<<grid, SLOT_THREADS, smem, st>>>(a, 0);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   SDM_CUDA_TRY(cudaGetLastError());
@@ -476,7 +486,8 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
       ea.t0 = t0;
       ea.ct = ct;
       ea.kb = WL.kb;
-      long long blocks = (E + 255) / 256;
+      const long long crow = (long long)ct * s.B * s.H;
+      long long blocks = (crow + 7) / 8;  // a warp per chunk row
       if (blocks > (long long)di->sms * 16) blocks = (long long)di->sms * 16;
       slot_events_kernel<<<(unsigned)blocks, 256, 0, st>>>(ea);
       g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -489,8 +500,8 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
       for (int shift = 0; shift < bits; shift += 8) {
         radix_hist_kernel<<<ntiles, RS_THREADS, 0, st>>>(ka, E, shift, hist, ntiles);
         radix_scan_kernel<<<RS_BINS, 1024, 0, st>>>(hist, ntiles, tot);
-        radix_scatter_kernel<<<ntiles, RS_THREADS, 0, st>>>(ka, va, kb, vb, E, shift, hist, tot,
-                                                            ntiles);
+        radix_scatter_kernel<<<ntiles, RS_THREADS, RS_SCATTER_SMEM, st>>>(ka, va, kb, vb, E, shift,
+                                                                          hist, tot, ntiles);
         g_launches.fetch_add(3, std::memory_order_relaxed);
         SDM_CUDA_TRY(cudaGetLastError());
         uint32_t* tk = ka;
@@ -500,11 +511,11 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
         va = vb;
         vb = tv;
       }
-      long long lblocks = (E / 32 + 7) / 8;
+      const long long nsamp = (E + 127) / 128;
+      long long lblocks = (nsamp + 255) / 256;
       if (lblocks > (long long)di->sms * 8) lblocks = (long long)di->sms * 8;
       if (lblocks < 1) lblocks = 1;
-      slot_long_segments_kernel<<<(unsigned)lblocks, 256, 0, st>>>(ks, E, bits, cnt, hot,
-                                                                   WL.hot_cap);
+      slot_long_segments_kernel<<<(unsigned)lblocks, 256, 0, st>>>(ks, E, cnt, hot, WL.hot_cap);
       g_launches.fetch_add(1, std::memory_order_relaxed);
       SDM_CUDA_TRY(cudaGetLastError());
     }

@@ -8,12 +8,13 @@
 //   2. every lane keeps its P = ceil(K/32) largest keys; the K-th largest key T lies between
 //      the smallest and the largest of the lanes' P-th largest keys (each lane then has at
 //      least P keys >= the smallest, and fewer than 32(P-1) < K keys exceed the largest);
-//   3. keys inside that bracket are compacted to shared memory in index order, T is found by
-//      binary search on counts, and the top K are the keys > T plus the lowest-index ties;
+//   3. keys inside that bracket are compacted to shared memory in index order; histogram
+//      levels (256 bins over the bracket, then over the bin that holds it) find the K-th
+//      largest key T, and the top K are the keys > T plus the lowest-index ties;
 //   4. a register bitonic sort (shuffles) orders them: (key desc, index asc).
 // Candidates: the rank pairs with (r1+1)(r2+1) <= K; their K-th largest sum is at least
-// max_p A[p-1] + B[ceil(K/p)-1] (p*ceil(K/p) >= K pairs reach that sum), which brackets the
-// same binary search; equal sums at the threshold take the lowest flat slot indices.
+// both A[K-1] + B[0] and A[0] + B[K-1] (K candidate sums reach each), which brackets the same
+// histogram search; equal sums at the threshold take the lowest flat slot indices.
 #pragma once
 
 #include "select.cuh"
@@ -42,29 +43,94 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
   return v;
 }
 
-// Descending bitonic sort of 32*NPL values held NPL per lane (position q*32 + lane).  The
-// stage loops stay rolled (small code); the per-lane element loops are unrolled.
+// The K-th largest key of a warp's keys, by histogram levels: 256 bins of 2^sh keys over
+// [lo, hi] locate the bin that holds it; the next level splits that bin, until a bin holds a
+// single key value T.  Entry: at least K keys are >= lo and none is > hi; `hist` (256 words)
+// is zero, and zero again on return.  for_each(f) calls f(key) on each of this lane's keys.
+struct WarpKth {
+  uint32_t T;  // the K-th largest key
+  int ngt;     // keys > T
+  int neq;     // keys == T
+};
+
+template <typename ForEach>
+__device__ __forceinline__ WarpKth warp_kth_key(ForEach for_each, uint32_t lo, uint32_t hi, int K,
+                                                uint32_t* hist, int lane) {
+  int above = 0;
+  while (true) {
+    const uint32_t range = hi - lo;
+    const int sh = range >= 256u ? 24 - __clz(static_cast<int>(range)) : 0;
+    for_each([&](uint32_t k) {
+      if (k >= lo && k <= hi) atomicAdd(&hist[(k - lo) >> sh], 1u);
+    });
+    __syncwarp();
+    // lane l reads bins 255 - 8l down to 248 - 8l and clears them for the next level
+    uint4* h4 = reinterpret_cast<uint4*>(hist);
+    const uint4 hh = h4[63 - 2 * lane], hl = h4[62 - 2 * lane];
+    h4[63 - 2 * lane] = make_uint4(0u, 0u, 0u, 0u);
+    h4[62 - 2 * lane] = make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t c[8] = {hh.w, hh.z, hh.y, hh.x, hl.w, hl.z, hl.y, hl.x};
+    uint32_t pre[8], local = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      pre[i] = local;
+      local += c[i];
+    }
+    const uint32_t incl = static_cast<uint32_t>(warp_incl_scan(static_cast<int>(local), lane));
+    const uint32_t excl = incl - local;
+    const uint32_t want = static_cast<uint32_t>(K - above);
+    uint32_t bin = 0, run = 0, cb = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (excl + pre[i] < want && want <= excl + pre[i] + c[i]) {
+        bin = static_cast<uint32_t>(255 - 8 * lane - i);
+        run = excl + pre[i];
+        cb = c[i];
+      }
+    }
+    const int cl = __ffs(__ballot_sync(FULL_MASK, excl < want && want <= incl)) - 1;
+    bin = __shfl_sync(FULL_MASK, bin, cl);
+    above += static_cast<int>(__shfl_sync(FULL_MASK, run, cl));
+    cb = __shfl_sync(FULL_MASK, cb, cl);
+    const uint32_t nlo = lo + (bin << sh);
+    const uint32_t span = (1u << sh) - 1u;
+    hi = (hi - nlo > span) ? nlo + span : hi;
+    lo = nlo;
+    __syncwarp();  // the cleared bins land before the next level counts
+    if (sh == 0) return WarpKth{lo, above, static_cast<int>(cb)};
+  }
+}
+
+// Compare-exchange of register pairs (q, q | QS) for the stages whose stride spans whole
+// registers (stride = 32 QS); QS is a constant so the array stays in registers.
+template <typename V, int NPL, int QS>
+__device__ __forceinline__ void bitonic_cross_regs(V (&v)[NPL], int size, int lane) {
+#pragma unroll
+  for (int q = 0; q < NPL; ++q) {
+    if ((q & QS) == 0 && (q | QS) < NPL) {
+      const int p = q * 32 + lane;
+      const bool desc = (p & size) == 0;
+      const V a = v[q], b = v[q | QS];
+      const bool sw = desc ? (a < b) : (a > b);
+      v[q] = sw ? b : a;
+      v[q | QS] = sw ? a : b;
+    }
+  }
+}
+
+// Descending bitonic sort of 32*NPL values held NPL per lane (position q*32 + lane), NPL <=
+// 4.  The stage loops stay rolled (small code); the per-lane element loops are unrolled.
 template <typename V, int NPL>
 __device__ __forceinline__ void bitonic_desc_reg(V (&v)[NPL], int lane) {
+  static_assert(NPL == 1 || NPL == 2 || NPL == 4, "one, two or four values per lane");
   constexpr int P2 = 32 * NPL;
 #pragma unroll 1
   for (int size = 2; size <= P2; size <<= 1) {
 #pragma unroll 1
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
       if (stride >= 32) {
-        const int qs = stride >> 5;
-#pragma unroll
-        for (int q = 0; q < NPL; ++q) {
-          if ((q & qs) == 0) {
-            const int q2 = q | qs;
-            const int p = q * 32 + lane;
-            const bool desc = (p & size) == 0;
-            const V a = v[q], b = v[q2];
-            const bool sw = desc ? (a < b) : (a > b);
-            v[q] = sw ? b : a;
-            v[q2] = sw ? a : b;
-          }
-        }
+        if (stride == 32) bitonic_cross_regs<V, NPL, 1>(v, size, lane);
+        else bitonic_cross_regs<V, NPL, 2>(v, size, lane);
       } else {
         const bool lower = (lane & stride) == 0;
 #pragma unroll
@@ -82,6 +148,7 @@ __device__ __forceinline__ void bitonic_desc_reg(V (&v)[NPL], int lane) {
 
 // Shared scratch of one warp of the fast path.
 struct FastScratch {
+  uint32_t* hist;   // [256] threshold histogram, zero between uses
   uint32_t* surv;   // [max(S1, S2)] bracket survivors of one half (composites)
   uint32_t* a;      // [KMAX] first half: sorted composites key16 << 16 | (0xffff - idx)
   uint32_t* b;      // [KMAX] second half
@@ -92,13 +159,15 @@ struct FastScratch {
 __host__ __device__ inline size_t fast_scratch_bytes(int S1, int S2, int K) {
   const int smax = S1 > S2 ? S1 : S2;
   (void)K;
-  return ((size_t)smax * 4 + 15) / 16 * 16 + 2 * (size_t)KMAX * 4 + 4 * (size_t)KMAX * 4 +
-         (size_t)KMAX * 8;
+  return 256 * 4 + ((size_t)smax * 4 + 15) / 16 * 16 + 2 * (size_t)KMAX * 4 +
+         4 * (size_t)KMAX * 4 + (size_t)KMAX * 8;
 }
 
 __device__ inline FastScratch carve_fast_scratch(unsigned char* p, int S1, int S2, int K) {
   FastScratch s;
   const int smax = S1 > S2 ? S1 : S2;
+  s.hist = reinterpret_cast<uint32_t*>(p);
+  p += 256 * 4;
   s.surv = reinterpret_cast<uint32_t*>(p);
   p += ((size_t)smax * 4 + 15) / 16 * 16;
   s.a = reinterpret_cast<uint32_t*>(p);
@@ -114,8 +183,8 @@ __device__ inline FastScratch carve_fast_scratch(unsigned char* p, int S1, int S
 // Top-K of one bf16 half of S values (S <= 256 * R8), written sorted to out[0..K).
 template <int R8, int KC>
 __device__ __forceinline__ void half_topk_bf16(const __nv_bfloat16* src, int S, int K, int lane,
-                                               uint32_t* surv, uint32_t* stage, uint32_t* out,
-                                               int idx_base = 0) {
+                                               uint32_t* surv, uint32_t* stage, uint32_t* hist,
+                                               uint32_t* out, int idx_base = 0) {
   constexpr int P = KC / 32;  // enough per-lane leaders for any K <= KC
   const unsigned lt = lanemask_lt();
   uint32_t k[R8][8];
@@ -160,7 +229,7 @@ __device__ __forceinline__ void half_topk_bf16(const __nv_bfloat16* src, int S, 
   for (int q = 1; q < P; ++q)
     if (q == pe - 1) lead = t[q];
   const uint32_t lo = max(__reduce_min_sync(FULL_MASK, lead), 1u);
-  const uint32_t hi = __reduce_max_sync(FULL_MASK, lead);
+  const uint32_t hi = __reduce_max_sync(FULL_MASK, t[0]);  // the largest key
   // bracket survivors, index order, as composites
   int base = 0;
 #pragma unroll
@@ -179,19 +248,13 @@ __device__ __forceinline__ void half_topk_bf16(const __nv_bfloat16* src, int S, 
   }
   __syncwarp();
   const int ns = base;
-  auto count_ge = [&](uint32_t x) {
-    int c = 0;
-    for (int s = lane; s < ns; s += 32) c += (surv[s] >> 16) >= x ? 1 : 0;
-    return __reduce_add_sync(FULL_MASK, c);
-  };
-  uint32_t a = lo, b = hi + 1u;
-  while (b - a > 1u) {
-    const uint32_t m = (a + b) >> 1;
-    if (count_ge(m) >= K) a = m;
-    else b = m;
-  }
-  const uint32_t T = a;
-  const int need = K - count_ge(T + 1u);
+  const WarpKth kth = warp_kth_key(
+      [&](auto f) {
+        for (int s = lane; s < ns; s += 32) f(surv[s] >> 16);
+      },
+      lo, hi, K, hist, lane);
+  const uint32_t T = kth.T;
+  const int need = K - kth.ngt;
   int tb = 0, ob = 0;
   for (int s0 = 0; s0 < ns; s0 += 32) {
     const int s = s0 + lane;
@@ -244,14 +307,16 @@ __device__ __forceinline__ void merge_top_sorted(const uint32_t* a, const uint32
 #pragma unroll 1
   for (int stride = P2 >> 1; stride > 0; stride >>= 1) {
     if (stride >= 32) {
-      const int qs = stride >> 5;
+      // half-cleaner across registers: every pair (q, q | qs) takes max / min
 #pragma unroll
       for (int q = 0; q < NPL; ++q) {
-        if ((q & qs) == 0) {
-          const int q2 = q | qs;
-          const uint32_t x = v[q], y = v[q2];
-          v[q] = x > y ? x : y;
-          v[q2] = x > y ? y : x;
+#pragma unroll
+        for (int qs = 1; qs < NPL; qs <<= 1) {
+          if (qs == (stride >> 5) && (q & qs) == 0) {
+            const uint32_t x = v[q], y = v[q | qs];
+            v[q] = x > y ? x : y;
+            v[q | qs] = x > y ? y : x;
+          }
         }
       }
     } else {
@@ -281,8 +346,8 @@ __device__ __forceinline__ int comp16_index(uint32_t c) { return (int)(0xffffu -
 template <int KC>
 __device__ __forceinline__ void cand_topk_bf16(const uint32_t* A, const uint32_t* B, int K,
                                                int S2, const uint16_t* ctab, int lane,
-                                               float* pv, uint64_t* stage, int32_t* out_idx,
-                                               float* out_wt) {
+                                               float* pv, uint64_t* stage, uint32_t* hist,
+                                               int32_t* out_idx, float* out_wt) {
   constexpr int CPL = (cand_count(KC) + 31) / 32;
   const unsigned lt = lanemask_lt();
   const int C = cand_count(K);
@@ -314,32 +379,24 @@ __device__ __forceinline__ void cand_topk_bf16(const uint32_t* A, const uint32_t
       cf[q] = (uint32_t)(ai[r1] + bi[r2]);
     }
   }
-  // bracket of the K-th largest sum
-  uint32_t lo = 0u;
-  for (int p = lane + 1; p <= K; p += 32) {
-    const int q = (K + p - 1) / p;
-    lo = max(lo, score_key(__fadd_rn(av[p - 1], bv[q - 1])));
-  }
-  lo = max(__reduce_max_sync(FULL_MASK, lo), 1u);
+  // bracket of the K-th largest sum: the K sums A[i] + B[0] and the K sums A[0] + B[i] are
+  // candidates, so both K-th largest bound it from below; A[0] + B[0] is the largest
   const uint32_t hi = score_key(__fadd_rn(av[0], bv[0]));
+  const uint32_t lo = max(score_key(__fadd_rn(av[K - 1], bv[0])),
+                          score_key(__fadd_rn(av[0], bv[K - 1])));
   orbits = __reduce_or_sync(FULL_MASK, orbits);
   const int tz = orbits ? __ffs(orbits) - 1 : 0;
-  auto count_ge = [&](uint32_t x) {
-    int c = 0;
+  const WarpKth kth = warp_kth_key(
+      [&](auto f) {
 #pragma unroll
-    for (int q = 0; q < CPL; ++q) c += (ck[q] != 0u && (ck[q] >> tz) >= x) ? 1 : 0;
-    return __reduce_add_sync(FULL_MASK, c);
-  };
-  uint32_t a = lo >> tz, b = (hi >> tz) + 1u;
-  while (b - a > 1u) {
-    const uint32_t m = a + ((b - a) >> 1);
-    if (count_ge(m) >= K) a = m;
-    else b = m;
-  }
-  const uint32_t T = a;  // shifted key of the K-th largest sum
-  const int ngt = count_ge(T + 1u);
+        for (int q = 0; q < CPL; ++q)
+          if (ck[q] != 0u) f(ck[q] >> tz);
+      },
+      lo >> tz, hi >> tz, K, hist, lane);
+  const uint32_t T = kth.T;  // shifted key of the K-th largest sum
+  const int ngt = kth.ngt;
   const int need = K - ngt;
-  const int nties = count_ge(T) - ngt;
+  const int nties = kth.neq;
   int ob = 0;
 #pragma unroll
   for (int q = 0; q < CPL; ++q) {
@@ -406,10 +463,10 @@ template <int R8, int KC>
 __device__ __forceinline__ void select_row_fast(const __nv_bfloat16* row, int S1, int S2, int K,
                                                 const uint16_t* ctab, FastScratch& sc, int lane,
                                                 int32_t* out_idx, float* out_wt) {
-  half_topk_bf16<R8, KC>(row, S1, K, lane, sc.surv, sc.stage, sc.a);
-  half_topk_bf16<R8, KC>(row + S1, S2, K, lane, sc.surv, sc.stage, sc.b);
+  half_topk_bf16<R8, KC>(row, S1, K, lane, sc.surv, sc.stage, sc.hist, sc.a);
+  half_topk_bf16<R8, KC>(row + S1, S2, K, lane, sc.surv, sc.stage, sc.hist, sc.b);
   cand_topk_bf16<KC>(sc.a, sc.b, K, S2, ctab, lane, sc.pv,
-                     reinterpret_cast<uint64_t*>(sc.stage), out_idx, out_wt);
+                     reinterpret_cast<uint64_t*>(sc.stage), sc.hist, out_idx, out_wt);
 }
 
 // Whether a row shape takes the fast path, and its template parameters.
@@ -439,6 +496,9 @@ __global__ void __launch_bounds__(256, 3) sel_fast_kernel(SelJob job0, SelJob jo
   const int wpc = blockDim.x >> 5;
   FastScratch sc = carve_fast_scratch(scratch_base + (size_t)warp * fast_scratch_bytes(S1, S2, KC),
                                       S1, S2, KC);
+  reinterpret_cast<uint4*>(sc.hist)[2 * lane] = make_uint4(0u, 0u, 0u, 0u);
+  reinterpret_cast<uint4*>(sc.hist)[2 * lane + 1] = make_uint4(0u, 0u, 0u, 0u);
+  __syncwarp();
   const long long total = n_rows * njobs;
   const int S = S1 + S2;
   for (long long r = (long long)blockIdx.x * wpc + warp; r < total;

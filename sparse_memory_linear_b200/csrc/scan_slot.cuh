@@ -447,6 +447,7 @@ __global__ void __launch_bounds__(SLOT_THREADS) slot_chunk_kernel(SlotArgs a, in
   const uint32_t e0 = a.offs[chunk], e1 = a.offs[chunk + 1];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int d4 = a.d_v / 4;
+  const bool bf16 = a.v_bf16 != 0;
   const unsigned lt = lanemask_lt();
   const uint32_t nmask = (1u << a.kb.nbits) - 1u;
   const uint32_t hmask = (1u << a.kb.hbits) - 1u;
@@ -542,6 +543,24 @@ __global__ void __launch_bounds__(SLOT_THREADS) slot_chunk_kernel(SlotArgs a, in
       nh += __popc(hm);
     }
     __syncwarp();
+    if (nh == 0) continue;
+    // The warp's events: [first, stop), every event of the short segments that start in the
+    // span (a long segment can only be the span's last head, and then no head follows it).
+    const uint32_t first = heads[0];
+    uint32_t stop = heads[nh - 1];
+    {
+      const uint32_t K = a.keys[stop];
+      while (true) {
+        const uint32_t ek = stop + lane;
+        const unsigned m2 = __ballot_sync(FULL_MASK, ek < e1 && a.keys[ek] == K);
+        if (m2 == FULL_MASK) {
+          stop += 32;
+          continue;
+        }
+        stop += __ffs(~m2) - 1;
+        break;
+      }
+    }
 
     auto issue = [&](int i) {
       if (i < nh) {
@@ -559,44 +578,118 @@ __global__ void __launch_bounds__(SLOT_THREADS) slot_chunk_kernel(SlotArgs a, in
 #pragma unroll
     for (int i = 0; i < PF - 1; ++i) issue(i);
 
-    for (int si = 0; si < nh; ++si) {
-      issue(si + PF - 1);
-      cp_async_wait<PF - 1>();
-      __syncwarp();
-      const uint32_t first = heads[si];
-      const uint32_t K = a.keys[first];
-      int b, h;
-      float* row = row_of(K, b, h);
-      // the segment's end (it is shorter than SLOT_LONG)
-      uint32_t last = first;
-      while (true) {
-        const uint32_t ek = last + lane;
-        const unsigned m2 = __ballot_sync(FULL_MASK, ek < e1 && a.keys[ek] == K);
-        if (m2 == FULL_MASK) {
-          last += 32;
-          continue;
-        }
-        last += __ffs(~m2) - 1;
-        break;
-      }
-      const float* slot_row = ring + (size_t)(si % PF) * 128 * NQ;
-      float4 m[NQ];
+    // Events stream in batches of 32, one per lane: the batch's key and value were loaded
+    // while the batch before it was processed, and its coefficients take one round trip
+    // (alpha, beta) issued before the batch's first state row is waited for.
+    int seg = -1;
+    float* row = nullptr;
+    bool dirty = false;
+    float4 m[NQ];
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        const int c = lane + 32 * q;
-        if (c < d4) m[q] = reinterpret_cast<const float4*>(slot_row)[c];
-      }
-      float unused = 1.0f;
-      const bool dirty = walk_events<NQ, G>(a, first, last, b, h, lane, m, false, unused);
-      if (dirty) {
+    for (int q = 0; q < NQ; ++q) m[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto close_segment = [&]() {
+      if (seg >= 0 && dirty) {
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
           const int c = lane + 32 * q;
           if (c < d4) reinterpret_cast<float4*>(row)[c] = m[q];
         }
       }
-      __syncwarp();  // the ring slot is refilled by the next iteration's issue()
+      __syncwarp();  // the ring slot is refilled by the next issue()
+    };
+    uint32_t nk = EV_SENTINEL;
+    uint2 npv = make_uint2(0u, 0u);
+    if (first + lane < stop) {
+      nk = a.keys[first + lane];
+      npv = a.vals[first + lane];
     }
+    uint32_t kcarry = EV_SENTINEL;  // the key before the batch (first is a head)
+    for (uint32_t b0 = first; b0 < stop; b0 += 32) {
+      const int cnt = static_cast<int>(min(32u, stop - b0));
+      const uint32_t ck = nk;
+      const uint2 pv = npv;
+      if (b0 + 32 + lane < stop) {
+        nk = a.keys[b0 + 32 + lane];
+        npv = a.vals[b0 + 32 + lane];
+      }
+      uint32_t kp = __shfl_up_sync(FULL_MASK, ck, 1);
+      if (lane == 0) kp = kcarry;
+      kcarry = __shfl_sync(FULL_MASK, ck, cnt - 1);
+      const bool head = lane < cnt && ck != kp;
+      // this lane's event: state row coefficients and token row
+      uint32_t r32 = 0u;
+      float ca = 0.f, cb = 0.f;
+      if (lane < cnt) {
+        const uint32_t t = pv.x >> 8;
+        const uint32_t kind = (pv.x >> 7) & 1u;
+        const uint32_t eh = (ck >> a.kb.nbits) & hmask;
+        const uint32_t eb = (ck >> (a.kb.nbits + a.kb.hbits)) & bmask;
+        const uint32_t r = (eb * a.T + t) * a.H + eh;
+        const float w = __uint_as_float(pv.y);
+        if (kind == 0u) {
+          const float kb = a.beta[r] * w;
+          ca = a.alpha[r] * (1.0f - kb);
+          cb = kb;
+        } else {
+          ca = w;
+        }
+        r32 = r | (kind << 31);
+      }
+      for (int i0 = 0; i0 < cnt; i0 += G) {
+        float4 vv[G][NQ];
+        uint32_t rr[G];
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+          rr[i] = __shfl_sync(FULL_MASK, r32, (i0 + i) & 31);
+          if (i0 + i < cnt && (rr[i] >> 31) == 0u)
+            load_v<NQ>(a.v, (size_t)(rr[i] & 0x7fffffffu) * a.d_v, bf16, lane, d4, vv[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+          const bool hd = __shfl_sync(FULL_MASK, head, (i0 + i) & 31) != 0;
+          const float A = __shfl_sync(FULL_MASK, ca, (i0 + i) & 31);
+          const float Bc = __shfl_sync(FULL_MASK, cb, (i0 + i) & 31);
+          if (i0 + i < cnt) {
+            if (hd) {
+              close_segment();
+              ++seg;
+              issue(seg + PF - 1);
+              cp_async_wait<PF - 1>();
+              __syncwarp();
+              int bb, hh;
+              row = row_of(a.keys[heads[seg]], bb, hh);
+              const float* slot_row = ring + (size_t)(seg % PF) * 128 * NQ;
+#pragma unroll
+              for (int q = 0; q < NQ; ++q) {
+                const int c = lane + 32 * q;
+                if (c < d4) m[q] = reinterpret_cast<const float4*>(slot_row)[c];
+              }
+              dirty = false;
+            }
+            if ((rr[i] >> 31) == 0u) {
+#pragma unroll
+              for (int q = 0; q < NQ; ++q) {
+                m[q].x = fmaf(A, m[q].x, Bc * vv[i][q].x);
+                m[q].y = fmaf(A, m[q].y, Bc * vv[i][q].y);
+                m[q].z = fmaf(A, m[q].z, Bc * vv[i][q].z);
+                m[q].w = fmaf(A, m[q].w, Bc * vv[i][q].w);
+              }
+              dirty = true;
+            } else {
+              float* yrow = a.y + (size_t)(rr[i] & 0x7fffffffu) * a.d_v;
+#pragma unroll
+              for (int q = 0; q < NQ; ++q) {
+                const int c = lane + 32 * q;
+                if (c < d4)
+                  atomicAdd(reinterpret_cast<float4*>(yrow) + c,
+                            make_float4(A * m[q].x, A * m[q].y, A * m[q].z, A * m[q].w));
+              }
+            }
+          }
+        }
+      }
+    }
+    close_segment();
     cp_async_wait<0>();
     __syncwarp();
   }

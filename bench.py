@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import hashlib
 import json
 import os
 import statistics
@@ -51,6 +52,21 @@ def algorithmic_bytes(wl) -> int:
     s_in = 2 if wl.in_dtype == torch.bfloat16 else 4
     return (2 * wl.W + wl.R) * wl.d_v * 4 + 2 * (wl.S1 + wl.S2) * s_in + wl.d_v * s_in
 
+
+
+def measured_traffic(kernel: str, units: float, unit_key: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture, scaled to `units`
+    units (token-heads or (b, h) pairs) per launch; None once the kernel's source no longer
+    has the hash the capture was taken with."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path))[kernel]
+        src = open(os.path.join(ROOT, rec["source"]), "rb").read()
+    except (OSError, KeyError, ValueError):
+        return None
+    if hashlib.sha256(src).hexdigest()[:16] != rec["source_sha256_16"]:
+        return None
+    return rec[unit_key] * units
 
 def scan_kernel_bytes(wl) -> int:
     """Bytes per token-head of the scan engine alone: the state rows only."""
@@ -265,7 +281,9 @@ def bench_prefill(args, dist: Dist, dev):
             "kernel": f"seq_scan_kernel" if scan_kind == "scan_seq" else "slot_chunk_kernel",
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_kind": f"{peak_kind} (burst copy)",
-            "traffic": None,
+            "traffic": (measured_traffic("slot_chunk_kernel", th / n_step[scan_kind],
+                                         "dram_bytes_per_token_head")
+                        if scan_kind == "scan_slot" else None),
             "algorithmic_bytes_per_launch": per_launch_bytes,
             "launch_ms": per_launch_ms,
             "launches_per_step": n_step[scan_kind],
@@ -339,7 +357,9 @@ def bench_decode(args, dist: Dist, dev):
                      "achieved": step_bytes / kernel_s / 1e9, "peak": peak, "unit": "GB/s",
                      "frac": step_bytes / kernel_s / 1e9 / peak,
                      "peak_kind": f"{peak_kind} (burst copy)",
-                     "algorithmic_bytes_per_launch": step_bytes, "kernel_us": kernel_s * 1e6},
+                     "algorithmic_bytes_per_launch": step_bytes, "kernel_us": kernel_s * 1e6,
+                     "traffic": measured_traffic("decode_kernel", wl.B * wl.H,
+                                                 "dram_bytes_per_unit")},
     }
     # the same 256 steps captured once into a CUDA graph and replayed
     try:

@@ -442,7 +442,7 @@ __host__ __device__ constexpr inline size_t slot_warp_smem(int NQ, int PF) {
 // each shorter segment that starts in its span, streaming the segments' state rows through
 // a ring of PF shared-memory rows with cp.async.
 template <int NQ, int G, int PF>
-__global__ void __launch_bounds__(SLOT_THREADS, (NQ <= 2 ? 3 : 1)) slot_chunk_kernel(SlotArgs a, int chunk) {
+__global__ void __launch_bounds__(SLOT_THREADS, (NQ <= 2 ? 4 : 1)) slot_chunk_kernel(SlotArgs a, int chunk) {
   extern __shared__ __align__(16) unsigned char smem[];
   const uint32_t e0 = a.offs[chunk], e1 = a.offs[chunk + 1];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;

@@ -89,7 +89,7 @@ sdm_status device_info(DeviceInfo** out) {
                                       (int)RS_SCATTER_SMEM));
 #define SDM_SLOT_ATTR(NQ, G, PF) \
   SDM_CUDA_TRY(allow_max_dynamic_smem(slot_chunk_kernel<NQ, G, PF>, m));
-    SDM_SLOT_ATTR(1, 4, 8) SDM_SLOT_ATTR(2, 2, 8) SDM_SLOT_ATTR(4, 4, 4) SDM_SLOT_ATTR(8, 2, 2)
+    SDM_SLOT_ATTR(1, 4, 6) SDM_SLOT_ATTR(2, 2, 6) SDM_SLOT_ATTR(4, 4, 4) SDM_SLOT_ATTR(8, 2, 2)
 #undef SDM_SLOT_ATTR
     d.attrs_set = true;
   }
@@ -521,8 +521,8 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
     }
     ProfScope ps(SDM_KERNEL_SCAN_SLOT, st);
     sdm_status rc;
-    if (d4 <= 32) rc = launch_slot_chunk<1, 4, 8>(a, di, st);
-    else if (d4 <= 64) rc = launch_slot_chunk<2, 2, 8>(a, di, st);
+    if (d4 <= 32) rc = launch_slot_chunk<1, 4, 6>(a, di, st);
+    else if (d4 <= 64) rc = launch_slot_chunk<2, 2, 6>(a, di, st);
     else if (d4 <= 128) rc = launch_slot_chunk<4, 4, 4>(a, di, st);
     else rc = launch_slot_chunk<8, 2, 2>(a, di, st);
     if (rc != SDM_OK) return rc;

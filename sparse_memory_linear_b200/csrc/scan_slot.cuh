@@ -128,11 +128,16 @@ __global__ void __launch_bounds__(RS_THREADS) radix_hist_kernel(const uint32_t* 
   for (int i = tid; i < RS_WARPS * RS_BINS; i += RS_THREADS) (&h[0][0])[i] = 0u;
   __syncthreads();
   const long long base = (long long)blockIdx.x * RS_TILE;
-#pragma unroll 4
+  // all of this thread's keys are loaded before the first count
+  uint32_t k16[RS_IPT];
+#pragma unroll
   for (int k = 0; k < RS_IPT; ++k) {
     const long long i = base + (long long)k * RS_THREADS + tid;
-    if (i < n) atomicAdd(&h[warp][(keys[i] >> shift) & 255u], 1u);
+    k16[k] = i < n ? keys[i] : EV_SENTINEL;
   }
+#pragma unroll
+  for (int k = 0; k < RS_IPT; ++k)
+    if (base + (long long)k * RS_THREADS + tid < n) atomicAdd(&h[warp][(k16[k] >> shift) & 255u], 1u);
   __syncthreads();
   uint32_t s = 0;
 #pragma unroll
@@ -199,7 +204,7 @@ __device__ __forceinline__ uint32_t rs_block_excl(uint32_t v, uint32_t* warp_tot
 // consecutive addresses of one run.
 constexpr size_t RS_SCATTER_SMEM = (size_t)RS_TILE * 6;  // staged keys and tile positions
 
-__global__ void __launch_bounds__(RS_THREADS) radix_scatter_kernel(
+__global__ void __launch_bounds__(RS_THREADS, 3) radix_scatter_kernel(
     const uint32_t* __restrict__ kin, const uint2* __restrict__ vin, uint32_t* __restrict__ kout,
     uint2* __restrict__ vout, long long n, int shift, const uint32_t* __restrict__ hist,
     const uint32_t* __restrict__ totals, int ntiles) {
@@ -225,7 +230,7 @@ __global__ void __launch_bounds__(RS_THREADS) radix_scatter_kernel(
   for (int i = tid; i < RS_WARPS * RS_BINS; i += RS_THREADS) (&wcnt[0][0])[i] = 0u;
   __syncthreads();
   const unsigned lt = lanemask_lt();
-  uint32_t rank[RS_IPT];
+  uint32_t rank2[RS_IPT / 2];  // two in-warp ranks (< 512) per register
 #pragma unroll
   for (int r = 0; r < RS_IPT; ++r) {
     const long long i = base + r * 32 + lane;
@@ -234,7 +239,9 @@ __global__ void __launch_bounds__(RS_THREADS) radix_scatter_kernel(
     const unsigned m = __match_any_sync(FULL_MASK, d);
     uint32_t before = 0;
     if (ok) before = wcnt[warp][d];
-    rank[r] = before + __popc(m & lt);
+    const uint32_t rk = before + __popc(m & lt);
+    if (r & 1) rank2[r >> 1] |= rk << 16;
+    else rank2[r >> 1] = rk;
     __syncwarp();
     if (ok && (m & lt) == 0) wcnt[warp][d] = before + __popc(m);
     __syncwarp();
@@ -257,7 +264,7 @@ __global__ void __launch_bounds__(RS_THREADS) radix_scatter_kernel(
     const long long i = base + r * 32 + lane;
     if (i < n) {
       const uint32_t d = (key[r] >> shift) & 255u;
-      const uint32_t lp = lbase[d] + wcnt[warp][d] + rank[r];
+      const uint32_t lp = lbase[d] + wcnt[warp][d] + ((rank2[r >> 1] >> (16 * (r & 1))) & 0xffffu);
       skey[lp] = key[r];
       sidx[lp] = static_cast<uint16_t>(i - tile0);
     }

@@ -50,7 +50,7 @@ constexpr int DEC_WARPS = DEC_THREADS / 32;
 constexpr size_t DEC_ROWS_SMEM_MAX = 64 * 1024;
 
 struct DecLayout {
-  uint32_t off_tab_w, off_tab_r, off_lists, off_vec, off_part;
+  uint32_t off_lists, off_vec, off_part;
   // group selection
   uint32_t off_hist, off_ctl, off_list, list_stride, off_clist, clist_stride, off_sorted, off_ev;
   uint32_t off_bits;  // 2048-bit membership filters of the write and the read slots
@@ -78,8 +78,6 @@ inline DecLayout dec_layout(int S1, int S2, int W, int R, int d_v, bool group) {
   L.C_r = cand_count(R);
   const int kmax = W > R ? W : R;
   const int smax = S1 > S2 ? S1 : S2;
-  L.off_tab_w = take((size_t)cand_count(W) * 2);
-  L.off_tab_r = take((size_t)cand_count(R) * 2);
   L.off_lists = take(4 * (size_t)KMAX * 4);  // idx_w, wt_w, idx_r, wt_r
   L.off_vec = take((2 * (size_t)d_v + 4) * 4);  // v, act(gate), alpha, beta
   L.off_part = take((size_t)DEC_WARPS * d_v * 4);
@@ -104,52 +102,6 @@ inline DecLayout dec_layout(int S1, int S2, int W, int R, int d_v, bool group) {
   if (L.rows_smem && scratch + rows_bytes > p) p = scratch + rows_bytes;
   L.total = static_cast<uint32_t>(p);
   return L;
-}
-
-// floor(a / b) for 0 <= a, b <= 128: the approximate quotient is within 2^-15 of a / b, and a
-// non-integer a / b is at least 1/128 below the next integer, so adding 2^-10 before the
-// floor recovers the exact quotient.
-__device__ __forceinline__ int quot_small(int a, int b) {
-  return static_cast<int>(__fdividef(static_cast<float>(a), static_cast<float>(b)) + 0x1p-10f);
-}
-
-// Rows of the candidate table of K (entries (r1 << 7) | r2 with (r1 + 1)(r2 + 1) <= K, rows
-// in r1 order) written by the four warps of one selection group, wq = 0..3: every warp
-// derives the row starts itself (a shuffle scan of the row lengths), then writes rows wq,
-// wq + 4, ... of the first 32 (whole warp per row) and one lane's share of rows 32 and up
-// (fewer than 4 entries each).
-__device__ __forceinline__ void build_cand_table_group(uint16_t* tab, int K, int wq, int lane) {
-  int len[4], start[4], run = 0;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int r = 4 * lane + q;
-    len[q] = r < K ? quot_small(K, r + 1) : 0;
-    run += len[q];
-  }
-  int incl = run;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int t = __shfl_up_sync(FULL_MASK, incl, o);
-    if (lane >= o) incl += t;
-  }
-  int base = incl - run;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    start[q] = base;
-    base += len[q];
-  }
-  const int rl = K < 32 ? K : 32;
-  for (int r = wq; r < rl; r += 4) {  // r is warp-uniform: r & 3 == wq
-    const int s0 = __shfl_sync(FULL_MASK, wq == 0 ? start[0] : wq == 1 ? start[1] : wq == 2 ? start[2] : start[3], r >> 2);
-    const int n = quot_small(K, r + 1);
-    for (int r2 = lane; r2 < n; r2 += 32) tab[s0 + r2] = static_cast<uint16_t>((r << 7) | r2);
-  }
-  const int r = 32 + 4 * lane + wq;  // rows 32..127: row r lives in lane r >> 2, slot wq
-  const int s0 = __shfl_sync(FULL_MASK, wq == 0 ? start[0] : wq == 1 ? start[1] : wq == 2 ? start[2] : start[3], (r >> 2) & 31);
-  if (r < K) {
-    const int n = quot_small(K, r + 1);
-    for (int r2 = 0; r2 < n; ++r2) tab[s0 + r2] = static_cast<uint16_t>((r << 7) | r2);
-  }
 }
 
 // Step 1 by the group selection: warps 2g, 2g + 1 take half g (0 write first, 1 write second,
@@ -199,7 +151,7 @@ __device__ __forceinline__ void decode_select_group(const DecodeArgs& a, const D
   // candidates of selection s
   const uint32_t* A = sorted + KMAX * (2 * s);
   const uint32_t* B = sorted + KMAX * (2 * s + 1);
-  const uint16_t* tab = reinterpret_cast<const uint16_t*>(smem + (s ? L.off_tab_r : L.off_tab_w));
+  const uint16_t* tab = cand_table(K);
   const int C = s ? L.C_r : L.C_w;
   uint32_t ck[CPT], cf[CPT];
 #pragma unroll
@@ -208,7 +160,7 @@ __device__ __forceinline__ void decode_select_group(const DecodeArgs& a, const D
     ck[j] = 0u;
     cf[j] = 0u;
     if (c < C) {
-      const int e = tab[c];
+      const int e = __ldg(tab + c);
       const uint32_t ca = A[e >> 7], cb = B[e & 127];
       ck[j] = score_key(__fadd_rn(key16_value(ca >> 16), key16_value(cb >> 16)));
       cf[j] = (0xffffu - (ca & 0xffffu)) * static_cast<uint32_t>(a.S2) + (0xffffu - (cb & 0xffffu));
@@ -268,8 +220,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
   const int S = a.S1 + a.S2;
   const int d4 = a.d_v / 4;
 
-  uint16_t* tab_w = reinterpret_cast<uint16_t*>(smem + L.off_tab_w);
-  uint16_t* tab_r = reinterpret_cast<uint16_t*>(smem + L.off_tab_r);
   int32_t* idx_w = reinterpret_cast<int32_t*>(smem + L.off_lists);
   float* wt_w = reinterpret_cast<float*>(idx_w + KMAX);
   int32_t* idx_r = reinterpret_cast<int32_t*>(wt_w + KMAX);
@@ -329,7 +279,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
       float* ev = reinterpret_cast<float*>(smem + L.off_ev) + KMAX * s;
       if (K + st < ((K + 3) & ~3)) ev[K + st] = 0.0f;
     }
-    build_cand_table_group((tid >> 7) ? tab_r : tab_w, (tid >> 7) ? a.R : a.W, warp & 3, lane);
 #pragma unroll
     for (int q = 0; q < VQ; ++q) {
       const int c = tid + DEC_THREADS * q;
@@ -347,8 +296,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
     const int kmax = a.W > a.R ? a.W : a.R;
     const size_t esz = bf16 ? 2 : 4;
     if (tid < 128) reinterpret_cast<uint32_t*>(smem + L.off_bits)[tid] = 0u;
-    build_cand_table(tab_w, a.W, tid, DEC_THREADS);
-    build_cand_table(tab_r, a.R, tid, DEC_THREADS);
     if (warp >= 2) {
       const int t0 = tid - 64, nt = DEC_THREADS - 64;
       for (int c = t0; c < a.d_v; c += nt) {
@@ -363,7 +310,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
       SelScratch sc = carve_sel_scratch(smem + L.off_sel + warp * L.sel_stride, a.S1, a.S2, kmax);
       const void* src = reinterpret_cast<const unsigned char*>(warp == 0 ? a.kp : a.qp) +
                         (size_t)bh * S * esz;
-      select_row(src, bf16, a.S1, a.S2, warp == 0 ? a.W : a.R, warp == 0 ? tab_w : tab_r, sc,
+      select_row(src, bf16, a.S1, a.S2, warp == 0 ? a.W : a.R, cand_table(warp == 0 ? a.W : a.R), sc,
                  lane, warp == 0 ? idx_w : idx_r, warp == 0 ? wt_w : wt_r);
     }
   }

@@ -37,28 +37,39 @@ __host__ __device__ constexpr inline int pow2_at_least(int x) {
   return p;
 }
 
-// Fills tab[0 .. cand_count(K)) with the rank pairs, packed as r1 << 7 | r2: one division
-// per row, a prefix sum of the row lengths, then every row written by its own thread.  Every
-// thread of the block must call it (it synchronises the block).
-__device__ inline void build_cand_table(uint16_t* tab, int K, int tid, int nthreads) {
-  __shared__ int start[KMAX + 1];
-  for (int r = tid; r < K; r += nthreads) start[r] = K / (r + 1);
-  __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int r = 0; r < K; ++r) {
-      const int len = start[r];
-      start[r] = run;
-      run += len;
-    }
-    start[K] = run;
+// The rank pairs of every K in [1, KMAX], packed as r1 << 7 | r2 in (r1, r2) order,
+// computed at compile time: table K starts at off[K] and holds off[K + 1] - off[K] pairs.
+constexpr int cand_total() {
+  int s = 0;
+  for (int K = 1; K <= KMAX; ++K) s += cand_count(K);
+  return s;
+}
+constexpr int CAND_TOTAL = cand_total();
+
+struct CandTables {
+  uint16_t e[CAND_TOTAL];
+  int off[KMAX + 2];
+};
+
+constexpr CandTables make_cand_tables() {
+  CandTables t{};
+  int p = 0;
+  for (int K = 1; K <= KMAX; ++K) {
+    t.off[K] = p;
+    for (int r1 = 0; r1 < K; ++r1)
+      for (int r2 = 0; r2 < K / (r1 + 1); ++r2) t.e[p++] = static_cast<uint16_t>((r1 << 7) | r2);
   }
-  __syncthreads();
-  for (int r1 = tid; r1 < K; r1 += nthreads) {
-    const int off = start[r1], len = start[r1 + 1] - off;
-    for (int r2 = 0; r2 < len; ++r2) tab[off + r2] = static_cast<uint16_t>((r1 << 7) | r2);
-  }
-  __syncthreads();
+  t.off[KMAX + 1] = p;
+  return t;
+}
+
+__device__ const CandTables g_cand_tables = make_cand_tables();
+
+__device__ __forceinline__ const uint16_t* cand_table(int K) {
+  return g_cand_tables.e + g_cand_tables.off[K];
+}
+__device__ __forceinline__ int cand_count_dev(int K) {
+  return g_cand_tables.off[K + 1] - g_cand_tables.off[K];
 }
 
 // Shared scratch of one selecting warp.
@@ -88,7 +99,7 @@ __host__ __device__ inline size_t sel_scratch_bytes(int S1, int S2, int K) {
 
 __device__ inline SelScratch carve_sel_scratch(unsigned char* p, int S1, int S2, int K) {
   SelScratch s;
-  const int C = cand_count(K);
+  const int C = cand_count_dev(K);  // K <= KMAX: the table's count, no division loop
   s.keys = reinterpret_cast<uint32_t*>(p);
   p += ((size_t)(S1 + S2) * 4 + 15) / 16 * 16;
   s.hist = reinterpret_cast<uint32_t*>(p);
@@ -237,7 +248,7 @@ __device__ inline void half_topk(const uint32_t* keys, int n, int K, int min_shi
 
 // Selects the top-K slots of one score row (first half S1 values, then S2 values) and
 // writes flat slot indices and softmax weights to out_idx[j], out_wt[j], j < K.
-// ctab holds cand_count(K) rank pairs.  Every lane of the warp must call it.
+// ctab holds the cand_count(K) rank pairs of K.  Every lane of the warp must call it.
 __device__ inline void select_row(const void* row, bool bf16, int S1, int S2, int K,
                                   const uint16_t* ctab, SelScratch& sc, int lane,
                                   int32_t* out_idx, float* out_wt) {
@@ -259,9 +270,9 @@ __device__ inline void select_row(const void* row, bool bf16, int S1, int S2, in
   half_topk(sc.keys + S1, S2, K, min_shift, sc, lane, sc.b_key, sc.b_idx);
 
   // candidate sums of the rank pairs
-  const int C = cand_count(K);
+  const int C = cand_count_dev(K);
   for (int c = lane; c < C; c += 32) {
-    const int e = ctab[c];
+    const int e = __ldg(ctab + c);
     const int r1 = e >> 7, r2 = e & 127;
     const float s = __fadd_rn(key_score(sc.a_key[r1]), key_score(sc.b_key[r2]));
     sc.c_key[c] = score_key(s);
@@ -354,16 +365,9 @@ __global__ void __launch_bounds__(256) sel_kernel(SelJob job0, SelJob job1, long
                                                   int njobs, int S1, int S2, int bf16,
                                                   int kmax_all) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const int C0 = cand_count(job0.K);
-  const int C1 = njobs > 1 ? cand_count(job1.K) : 0;
-  uint16_t* tab0 = reinterpret_cast<uint16_t*>(smem);
-  uint16_t* tab1 = tab0 + ((C0 + 7) / 8) * 8;
-  unsigned char* scratch_base =
-      reinterpret_cast<unsigned char*>(tab1 + ((C1 + 7) / 8) * 8);
-  build_cand_table(tab0, job0.K, threadIdx.x, blockDim.x);
-  if (njobs > 1) build_cand_table(tab1, job1.K, threadIdx.x, blockDim.x);
-  __syncthreads();
-
+  unsigned char* scratch_base = smem;
+  const uint16_t* tab0 = cand_table(job0.K);
+  const uint16_t* tab1 = cand_table(njobs > 1 ? job1.K : job0.K);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wpc = blockDim.x >> 5;
   SelScratch sc = carve_sel_scratch(
@@ -384,8 +388,7 @@ __global__ void __launch_bounds__(256) sel_kernel(SelJob job0, SelJob job1, long
 
 inline size_t sel_smem_bytes(int S1, int S2, int K0, int K1, int warps) {
   const int kmax = K0 > K1 ? K0 : K1;
-  size_t tabs = (size_t)((cand_count(K0) + 7) / 8) * 16 + (size_t)((cand_count(K1) + 7) / 8) * 16;
-  return tabs + (size_t)warps * sel_scratch_bytes(S1, S2, kmax);
+  return (size_t)warps * sel_scratch_bytes(S1, S2, kmax);
 }
 
 }  // namespace sdm

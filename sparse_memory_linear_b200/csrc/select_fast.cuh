@@ -88,7 +88,14 @@ __device__ __forceinline__ WarpKth warp_kth_key(ForEach for_each, uint32_t lo, u
         cb = c[i];
       }
     }
-    const int cl = __ffs(__ballot_sync(FULL_MASK, excl < want && want <= incl)) - 1;
+    const unsigned cm = __ballot_sync(FULL_MASK, excl < want && want <= incl);
+    if (cm == 0u) {
+      // fewer than K keys in range: only inputs outside the contract (NaN scores) get here;
+      // stop with every key in range taken
+      __syncwarp();
+      return WarpKth{lo, above, static_cast<int>(__shfl_sync(FULL_MASK, incl, 31))};
+    }
+    const int cl = __ffs(cm) - 1;
     bin = __shfl_sync(FULL_MASK, bin, cl);
     above += static_cast<int>(__shfl_sync(FULL_MASK, run, cl));
     cb = __shfl_sync(FULL_MASK, cb, cl);
@@ -265,7 +272,7 @@ __device__ __forceinline__ void half_topk_bf16(const __nv_bfloat16* src, int S, 
     const unsigned tm = __ballot_sync(FULL_MASK, tie);
     const bool take = gt || (tie && tb + __popc(tm & lt) < need);
     const unsigned sm = __ballot_sync(FULL_MASK, take);
-    if (take) stage[ob + __popc(sm & lt)] = c;
+    if (take && ob + __popc(sm & lt) < K) stage[ob + __popc(sm & lt)] = c;
     ob += __popc(sm);
     tb += __popc(tm);
   }
@@ -350,7 +357,7 @@ __device__ __forceinline__ void cand_topk_bf16(const uint32_t* A, const uint32_t
                                                int32_t* out_idx, float* out_wt) {
   constexpr int CPL = (cand_count(KC) + 31) / 32;
   const unsigned lt = lanemask_lt();
-  const int C = cand_count(K);
+  const int C = cand_count_dev(K);
   float* av = pv;                                   // [KMAX] first-half values
   float* bv = pv + KMAX;                            // [KMAX] second-half values
   int* ai = reinterpret_cast<int*>(pv + 2 * KMAX);  // [KMAX] first-half index * S2
@@ -371,7 +378,7 @@ __device__ __forceinline__ void cand_topk_bf16(const uint32_t* A, const uint32_t
     ck[q] = 0u;  // no candidate (every real score has a key >= 1)
     cf[q] = 0u;
     if (c < C) {
-      const int e = ctab[c];
+      const int e = __ldg(ctab + c);
       const int r1 = e >> 7, r2 = e & 127;
       const float s = __fadd_rn(av[r1], bv[r2]);
       orbits |= __float_as_uint(s) & 0x7fffffffu;
@@ -403,7 +410,8 @@ __device__ __forceinline__ void cand_topk_bf16(const uint32_t* A, const uint32_t
     const uint32_t sk = ck[q] >> tz;
     const bool take = ck[q] != 0u && (sk > T || (sk == T && nties == need));
     const unsigned sm = __ballot_sync(FULL_MASK, take);
-    if (take) stage[ob + __popc(sm & lt)] = (static_cast<uint64_t>(ck[q]) << 32) | (0xffffffffu - cf[q]);
+    if (take && ob + __popc(sm & lt) < K)
+      stage[ob + __popc(sm & lt)] = (static_cast<uint64_t>(ck[q]) << 32) | (0xffffffffu - cf[q]);
     ob += __popc(sm);
   }
   if (nties != need) {
@@ -421,7 +429,7 @@ __device__ __forceinline__ void cand_topk_bf16(const uint32_t* A, const uint32_t
         const uint64_t t2 = __shfl_xor_sync(FULL_MASK, best, o);
         best = t2 > best ? t2 : best;
       }
-      if (lane == 0) stage[ob] = best;
+      if (lane == 0 && ob < K) stage[ob] = best;
       floor_c = best;
       ++ob;
     }
@@ -484,14 +492,9 @@ template <int R8, int KC>
 __global__ void __launch_bounds__(256, 3) sel_fast_kernel(SelJob job0, SelJob job1, long long n_rows,
                                                        int njobs, int S1, int S2) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const int C0 = cand_count(job0.K);
-  const int C1 = njobs > 1 ? cand_count(job1.K) : 0;
-  uint16_t* tab0 = reinterpret_cast<uint16_t*>(smem);
-  uint16_t* tab1 = tab0 + ((C0 + 7) / 8) * 8;
-  unsigned char* scratch_base = reinterpret_cast<unsigned char*>(tab1 + ((C1 + 7) / 8) * 8);
-  build_cand_table(tab0, job0.K, threadIdx.x, blockDim.x);
-  if (njobs > 1) build_cand_table(tab1, job1.K, threadIdx.x, blockDim.x);
-  __syncthreads();
+  unsigned char* scratch_base = smem;
+  const uint16_t* tab0 = cand_table(job0.K);
+  const uint16_t* tab1 = cand_table(njobs > 1 ? job1.K : job0.K);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wpc = blockDim.x >> 5;
   FastScratch sc = carve_fast_scratch(scratch_base + (size_t)warp * fast_scratch_bytes(S1, S2, KC),
@@ -514,8 +517,7 @@ __global__ void __launch_bounds__(256, 3) sel_fast_kernel(SelJob job0, SelJob jo
 
 inline size_t sel_fast_smem_bytes(int S1, int S2, int K0, int K1, int warps) {
   const int kc = fast_kc(K0 > K1 ? K0 : K1);
-  size_t tabs = (size_t)((cand_count(K0) + 7) / 8) * 16 + (size_t)((cand_count(K1) + 7) / 8) * 16;
-  return tabs + (size_t)warps * fast_scratch_bytes(S1, S2, kc);
+  return (size_t)warps * fast_scratch_bytes(S1, S2, kc);
 }
 
 }  // namespace sdm

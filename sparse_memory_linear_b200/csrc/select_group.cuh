@@ -131,6 +131,14 @@ __device__ __forceinline__ CutResult group_cut(const uint32_t (&key)[NK], uint32
         ctl->run = run;
         ctl->cnt_bin = cb;
       }
+      // fewer than `want` keys in range can only come from inputs outside the contract (NaN
+      // or infinite scores): take the bottom bin with every key in range, so the range still
+      // shrinks and the loop ends
+      if (__ballot_sync(FULL_MASK, crossing) == 0u && gt == 31) {
+        ctl->bin = 0u;
+        ctl->run = 0u;
+        ctl->cnt_bin = incl;
+      }
     }
     group_bar(bar_id, NT);
     const uint32_t b = ctl->bin;
@@ -147,17 +155,11 @@ __device__ __forceinline__ CutResult group_cut(const uint32_t (&key)[NK], uint32
 // Steps 2 and 3: the survivors of `cr` in selection order.  emit(r, comp) is called once per
 // survivor with its rank r (0 = first); ranks >= K are not part of the top K.  The
 // survivors are listed in any order, then each counts the listed survivors above it.
-// `list` holds cr.n + 4 entries; `counter` is zero on entry.
+// `list` holds every key of the group plus 4 entries; `counter` is zero on entry.
 template <int NK, int NT, typename T, typename Comp, typename Emit>
 __device__ __forceinline__ void group_order(const uint32_t (&key)[NK], const CutResult& cr,
                                             Comp comp, T* list, uint32_t* counter, int gt,
                                             int lane, int bar_id, Emit emit) {
-  // listed survivors, padded with zeros (below every composite) to a multiple of 4
-  if (gt == 0) {
-#pragma unroll
-    for (int p = 0; p < 4; ++p) list[(cr.n & ~3) + p] = T(0);
-  }
-  group_bar(bar_id, NT);  // the padding lands before any composite of the last quad
   int m = 0;
 #pragma unroll
   for (int i = 0; i < NK; ++i) m += key[i] >= cr.cut ? 1 : 0;
@@ -175,8 +177,13 @@ __device__ __forceinline__ void group_order(const uint32_t (&key)[NK], const Cut
   for (int i = 0; i < NK; ++i)
     if (key[i] >= cr.cut) list[pos++] = comp(i);
   group_bar(bar_id, NT);
-  const int n4 = (cr.n + 3) >> 2;
-  for (int j = gt; j < cr.n; j += NT) {
+  // the survivors listed (cr.n of them for inputs inside the contract), padded with zeros
+  // (below every composite) to a multiple of 4
+  const int n = static_cast<int>(*counter);
+  if (gt < 4 && (n & ~3) + gt >= n) list[(n & ~3) + gt] = T(0);
+  group_bar(bar_id, NT);
+  const int n4 = (n + 3) >> 2;
+  for (int j = gt; j < n; j += NT) {
     const T x = list[j];
     int r0 = 0, r1 = 0;
     if constexpr (sizeof(T) == 4) {

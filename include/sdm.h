@@ -158,6 +158,12 @@ sdm_status sdm_scan_forward_noalloc(const void *kp, const void *qp, const void *
  *   o [B,H,d_v] fp32 out, nullable; gamma [d_v] nullable;
  *   sel_out nullable: write slots [B,H,W] followed by read slots [B,H,R].
  * shape.T is ignored.  No scratch memory is used.
+ * The launch allows programmatic stream serialisation: the step's selection, which reads only
+ * kp, qp, v, gate, alpha, beta and gamma, may run while the kernel ahead of it on the stream
+ * (typically the previous decode step) is finishing.  The step waits for that kernel before
+ * it touches M, y, o or sel_out.  A step's inputs therefore must not be the outputs (M, y, o,
+ * sel_out) of the kernel launched right before it.  SDM_NO_PDL=1 in the environment turns
+ * this off.
  */
 sdm_status sdm_decode_step(const void *kp, const void *qp, const void *v, const float *alpha,
                            const float *beta, float *M, float *y, const void *gate,

@@ -14,6 +14,9 @@ __global__ void __launch_bounds__(256) norm_gate_kernel(const float* __restrict_
                                                         const float* __restrict__ gamma,
                                                         float eps, int act, long long rows,
                                                         int d_v, float* o) {
+  // wait for the kernel ahead in the stream (programmatic launch), then let the next one in
+  grid_dependency_wait();
+  grid_launch_dependents();
   const int lane = threadIdx.x & 31;
   const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
@@ -52,6 +55,9 @@ __global__ void __launch_bounds__(256) norm_gate_kernel(const float* __restrict_
 __global__ void __launch_bounds__(256) state_init_kernel(const float4* __restrict__ M0,
                                                          float4* __restrict__ M, int B, int H,
                                                          long long per_head4) {
+  // wait for the kernel ahead in the stream (programmatic launch), then let the next one in
+  grid_dependency_wait();
+  grid_launch_dependents();
   const long long total = (long long)B * H * per_head4;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {

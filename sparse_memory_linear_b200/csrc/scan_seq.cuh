@@ -74,6 +74,9 @@ __host__ __device__ inline SeqLayout seq_layout(int ldw, int ldr, int CW, int v_
 
 template <int CW, int D>
 __global__ void __launch_bounds__(SEQ_THREADS, 1) seq_scan_kernel(SeqArgs a) {
+  // wait for the kernel ahead in the stream (programmatic launch), then let the next one in
+  grid_dependency_wait();
+  grid_launch_dependents();
   constexpr int LPR = CW / 4;             // lanes per row, one float4 each
   constexpr int NG = SEQ_THREADS / LPR;   // row groups
   constexpr int NW = SEQ_THREADS / 32;

@@ -68,6 +68,9 @@ struct EventArgs {
 // the row, else read j - W.  key = (b, h, slot) bit fields; val = {t << 8 | kind << 7 | j,
 // weight bits}.
 __global__ void __launch_bounds__(256) slot_events_kernel(EventArgs a) {
+  // wait for the kernel ahead in the stream (programmatic launch), then let the next one in
+  grid_dependency_wait();
+  grid_launch_dependents();
   const int lane = threadIdx.x & 31;
   const long long crow = (long long)a.B * a.ct * a.H;
   const int per = a.W + a.R;
@@ -123,6 +126,9 @@ __global__ void __launch_bounds__(RS_THREADS) radix_hist_kernel(const uint32_t* 
                                                                 long long n, int shift,
                                                                 uint32_t* __restrict__ hist,
                                                                 int ntiles) {
+  // wait for the kernel ahead in the stream (programmatic launch), then let the next one in
+  grid_dependency_wait();
+  grid_launch_dependents();
   __shared__ uint32_t h[RS_WARPS][RS_BINS];
   const int tid = threadIdx.x, warp = tid >> 5;
   for (int i = tid; i < RS_WARPS * RS_BINS; i += RS_THREADS) (&h[0][0])[i] = 0u;
@@ -149,6 +155,9 @@ __global__ void __launch_bounds__(RS_THREADS) radix_hist_kernel(const uint32_t* 
 // totals[digit] receives the digit's count.
 __global__ void __launch_bounds__(1024) radix_scan_kernel(uint32_t* __restrict__ hist, int ntiles,
                                                           uint32_t* __restrict__ totals) {
+  // wait for the kernel ahead in the stream (programmatic launch), then let the next one in
+  grid_dependency_wait();
+  grid_launch_dependents();
   __shared__ uint32_t part[1024];
   const int d = blockIdx.x, tid = threadIdx.x;
   uint32_t* row = hist + (size_t)d * ntiles;
@@ -208,6 +217,9 @@ __global__ void __launch_bounds__(RS_THREADS, 3) radix_scatter_kernel(
     const uint32_t* __restrict__ kin, const uint2* __restrict__ vin, uint32_t* __restrict__ kout,
     uint2* __restrict__ vout, long long n, int shift, const uint32_t* __restrict__ hist,
     const uint32_t* __restrict__ totals, int ntiles) {
+  // wait for the kernel ahead in the stream (programmatic launch), then let the next one in
+  grid_dependency_wait();
+  grid_launch_dependents();
   extern __shared__ __align__(16) unsigned char rs_smem[];
   uint32_t* skey = reinterpret_cast<uint32_t*>(rs_smem);                        // [RS_TILE]
   uint16_t* sidx = reinterpret_cast<uint16_t*>(rs_smem + (size_t)RS_TILE * 4);  // [RS_TILE]
@@ -288,6 +300,9 @@ __global__ void __launch_bounds__(RS_THREADS, 3) radix_scatter_kernel(
 __global__ void __launch_bounds__(256) slot_long_segments_kernel(
     const uint32_t* __restrict__ keys, long long n, uint32_t* hot_count, uint2* hot_list,
     int hot_cap) {
+  // wait for the kernel ahead in the stream (programmatic launch), then let the next one in
+  grid_dependency_wait();
+  grid_launch_dependents();
   static_assert(SLOT_LONG >= 256, "two samples 128 apart must fit in a long segment");
   const long long nsamp = (n + 127) / 128;
   for (long long si = (long long)blockIdx.x * blockDim.x + threadIdx.x; si < nsamp;
@@ -450,6 +465,9 @@ __host__ __device__ constexpr inline size_t slot_warp_smem(int NQ, int PF) {
 // a ring of PF shared-memory rows with cp.async.
 template <int NQ, int G, int PF>
 __global__ void __launch_bounds__(SLOT_THREADS, (NQ <= 2 ? 4 : 1)) slot_chunk_kernel(SlotArgs a, int chunk) {
+  // wait for the kernel ahead in the stream (programmatic launch), then let the next one in
+  grid_dependency_wait();
+  grid_launch_dependents();
   extern __shared__ __align__(16) unsigned char smem[];
   const uint32_t e0 = a.offs[chunk], e1 = a.offs[chunk + 1];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;

@@ -5,6 +5,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "common.cuh"
@@ -34,6 +35,36 @@ constexpr size_t WS_ALIGN = 256;
       return SDM_ERR_CUDA;                       \
     }                                            \
   } while (0)
+
+// SDM_NO_PDL=1 launches the decode step in plain stream order (for comparison).
+inline bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("SDM_NO_PDL");
+    return !(e && e[0] == '1');
+  }();
+  return on;
+}
+
+// Launches `kernel` in stream order.  Every kernel of this library starts with
+// griddepcontrol.wait / launch_dependents, so any of them may also be launched with
+// programmatic stream serialisation (scheduled while the kernel ahead of it finishes) without
+// changing results; only the decode step does that (a step's selection then overlaps the end
+// of the step before it).  For the prefill's chain of kernels it measured slower.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 0;  // plain stream order: overlapped launches measured slower in the prefill
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Kernels launched by this library in this process (all devices).
 std::atomic<unsigned long long> g_launches{0};
@@ -261,8 +292,8 @@ sdm_status launch_select_fast_t(const SelJob& j0, const SelJob* j1, long long ro
   long long grid = (long long)di->sms * per_sm;
   const long long need = (total_rows + warps - 1) / warps;
   if (grid > need) grid = need;
-  sel_fast_kernel<R8, KC><<<(unsigned)grid, warps * 32, smem, st>>>(j0, j1 ? *j1 : j0, rows,
-                                                                    j1 ? 2 : 1, S1, S2);
+  SDM_CUDA_TRY(launch_pdl(sel_fast_kernel<R8, KC>, dim3((unsigned)grid), dim3(warps * 32), smem, st,
+                          j0, j1 ? *j1 : j0, rows, j1 ? 2 : 1, S1, S2));
   g_launches.fetch_add(1, std::memory_order_relaxed);
   SDM_CUDA_TRY(cudaGetLastError());
   return SDM_OK;
@@ -310,8 +341,8 @@ sdm_status launch_select(const SelJob& j0, const SelJob* j1, long long rows, int
   const long long need = (total_rows + warps - 1) / warps;
   if (grid > need) grid = need;
   const int kmax = j0.K > K1 ? j0.K : K1;
-  sel_kernel<<<(unsigned)grid, warps * 32, smem, st>>>(j0, j1 ? *j1 : j0, rows, j1 ? 2 : 1, S1,
-                                                       S2, bf16, kmax);
+  SDM_CUDA_TRY(launch_pdl(sel_kernel, dim3((unsigned)grid), dim3(warps * 32), smem, st,
+                          j0, j1 ? *j1 : j0, rows, j1 ? 2 : 1, S1, S2, bf16, kmax));
   g_launches.fetch_add(1, std::memory_order_relaxed);
   SDM_CUDA_TRY(cudaGetLastError());
   return SDM_OK;
@@ -319,7 +350,8 @@ sdm_status launch_select(const SelJob& j0, const SelJob* j1, long long rows, int
 
 template <int CW, int D>
 sdm_status launch_seq_t(const SeqArgs& a, int grid, size_t smem, cudaStream_t st) {
-  seq_scan_kernel<CW, D><<<grid, SEQ_THREADS, smem, st>>>(a);
+  SDM_CUDA_TRY(launch_pdl(seq_scan_kernel<CW, D>, dim3(grid), dim3(SEQ_THREADS), smem, st,
+                          a));
   g_launches.fetch_add(1, std::memory_order_relaxed);
   SDM_CUDA_TRY(cudaGetLastError());
   return SDM_OK;
@@ -376,8 +408,8 @@ sdm_status launch_norm_gate(const float* y, const void* gate, int gate_bf16, con
   long long blocks = (rows + 7) / 8;
   const long long cap = (long long)di->sms * 8;
   if (blocks > cap) blocks = cap;
-  norm_gate_kernel<<<(unsigned)blocks, 256, 0, st>>>(y, gate, gate_bf16, gamma, eps, act, rows,
-                                                     d_v, o);
+  SDM_CUDA_TRY(launch_pdl(norm_gate_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
+                          y, gate, gate_bf16, gamma, eps, act, rows, d_v, o));
   g_launches.fetch_add(1, std::memory_order_relaxed);
   SDM_CUDA_TRY(cudaGetLastError());
   return SDM_OK;
@@ -392,9 +424,8 @@ sdm_status launch_state_init(const float* M0, float* M, const sdm_shape& s, cuda
   long long blocks = (total + 255) / 256;
   const long long cap = (long long)di->sms * 16;
   if (blocks > cap) blocks = cap;
-  state_init_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(M0),
-                                                      reinterpret_cast<float4*>(M), s.B, s.H,
-                                                      per_head4);
+  SDM_CUDA_TRY(launch_pdl(state_init_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
+                          reinterpret_cast<const float4*>(M0), reinterpret_cast<float4*>(M), s.B, s.H, per_head4));
   g_launches.fetch_add(1, std::memory_order_relaxed);
   SDM_CUDA_TRY(cudaGetLastError());
   return SDM_OK;
@@ -410,7 +441,8 @@ sdm_status launch_slot_chunk(const SlotArgs& a, const DeviceInfo* di, cudaStream
   const int cap = env_int("SDM_SLOT_CTAS", 0);
   if (cap > 0 && cap < ctas) ctas = cap;
   const int grid = di->sms * ctas;
-  slot_chunk_kernel<NQ, G, PF><<<grid, SLOT_THREADS, smem, st>>>(a, 0);
+  SDM_CUDA_TRY(launch_pdl(slot_chunk_kernel<NQ, G, PF>, dim3(grid), dim3(SLOT_THREADS), smem, st,
+                          a, 0));
   g_launches.fetch_add(1, std::memory_order_relaxed);
   SDM_CUDA_TRY(cudaGetLastError());
   return SDM_OK;
@@ -489,7 +521,8 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
       const long long crow = (long long)ct * s.B * s.H;
       long long blocks = (crow + 7) / 8;  // a warp per chunk row
       if (blocks > (long long)di->sms * 16) blocks = (long long)di->sms * 16;
-      slot_events_kernel<<<(unsigned)blocks, 256, 0, st>>>(ea);
+      SDM_CUDA_TRY(launch_pdl(slot_events_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
+                              ea));
       g_launches.fetch_add(1, std::memory_order_relaxed);
       SDM_CUDA_TRY(cudaGetLastError());
       // LSD radix sort over the key bits in use
@@ -498,10 +531,12 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
       uint2* va = v0;
       uint2* vb = v1;
       for (int shift = 0; shift < bits; shift += 8) {
-        radix_hist_kernel<<<ntiles, RS_THREADS, 0, st>>>(ka, E, shift, hist, ntiles);
-        radix_scan_kernel<<<RS_BINS, 1024, 0, st>>>(hist, ntiles, tot);
-        radix_scatter_kernel<<<ntiles, RS_THREADS, RS_SCATTER_SMEM, st>>>(ka, va, kb, vb, E, shift,
-                                                                          hist, tot, ntiles);
+        SDM_CUDA_TRY(launch_pdl(radix_hist_kernel, dim3(ntiles), dim3(RS_THREADS), 0, st,
+                                ka, E, shift, hist, ntiles));
+        SDM_CUDA_TRY(launch_pdl(radix_scan_kernel, dim3(RS_BINS), dim3(1024), 0, st,
+                                hist, ntiles, tot));
+        SDM_CUDA_TRY(launch_pdl(radix_scatter_kernel, dim3(ntiles), dim3(RS_THREADS), RS_SCATTER_SMEM, st,
+                                ka, va, kb, vb, E, shift, hist, tot, ntiles));
         g_launches.fetch_add(3, std::memory_order_relaxed);
         SDM_CUDA_TRY(cudaGetLastError());
         uint32_t* tk = ka;
@@ -515,7 +550,8 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
       long long lblocks = (nsamp + 255) / 256;
       if (lblocks > (long long)di->sms * 8) lblocks = (long long)di->sms * 8;
       if (lblocks < 1) lblocks = 1;
-      slot_long_segments_kernel<<<(unsigned)lblocks, 256, 0, st>>>(ks, E, cnt, hot, WL.hot_cap);
+      SDM_CUDA_TRY(launch_pdl(slot_long_segments_kernel, dim3((unsigned)lblocks), dim3(256), 0, st,
+                              ks, E, cnt, hot, WL.hot_cap));
       g_launches.fetch_add(1, std::memory_order_relaxed);
       SDM_CUDA_TRY(cudaGetLastError());
     }
@@ -756,9 +792,22 @@ sdm_status sdm_decode_step(const void* kp, const void* qp, const void* v, const 
   a.in_bf16 = s.in_dtype == SDM_BF16;
   ProfScope ps(SDM_KERNEL_DECODE, static_cast<cudaStream_t>(stream));
   bool launched = false;
+  // Programmatic stream serialisation: the step's selection (which reads only its inputs)
+  // may overlap the end of the kernel ahead of it; the kernel waits for that kernel before
+  // its first state access.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.BH);
+  cfg.blockDim = dim3(DEC_THREADS);
+  cfg.dynamicSmemBytes = L.total;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
 #define SDM_DEC_LAUNCH(E, KC, NQ)                                                        \
   if (!launched && SDM_DEC_FITS(E, KC, NQ)) {                                             \
-    decode_kernel<E, KC, NQ><<<a.BH, DEC_THREADS, L.total, static_cast<cudaStream_t>(stream)>>>(a, L); \
+    SDM_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_kernel<E, KC, NQ>, a, L));              \
     g_launches.fetch_add(1, std::memory_order_relaxed);                                   \
     launched = true;                                                                      \
   }

@@ -364,6 +364,9 @@ struct SelJob {
 __global__ void __launch_bounds__(256) sel_kernel(SelJob job0, SelJob job1, long long n_rows,
                                                   int njobs, int S1, int S2, int bf16,
                                                   int kmax_all) {
+  // wait for the kernel ahead in the stream (programmatic launch), then let the next one in
+  grid_dependency_wait();
+  grid_launch_dependents();
   extern __shared__ __align__(16) unsigned char smem[];
   unsigned char* scratch_base = smem;
   const uint16_t* tab0 = cand_table(job0.K);

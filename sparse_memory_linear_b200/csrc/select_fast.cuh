@@ -491,6 +491,9 @@ __host__ __device__ inline int fast_kc(int K) { return K <= 32 ? 32 : (K <= 64 ?
 template <int R8, int KC>
 __global__ void __launch_bounds__(256, 3) sel_fast_kernel(SelJob job0, SelJob job1, long long n_rows,
                                                        int njobs, int S1, int S2) {
+  // wait for the kernel ahead in the stream (programmatic launch), then let the next one in
+  grid_dependency_wait();
+  grid_launch_dependents();
   extern __shared__ __align__(16) unsigned char smem[];
   unsigned char* scratch_base = smem;
   const uint16_t* tab0 = cand_table(job0.K);

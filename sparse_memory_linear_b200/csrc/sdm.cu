@@ -45,12 +45,13 @@ inline bool pdl_enabled() {
   return on;
 }
 
-// Launches `kernel` in stream order.  Every kernel of this library starts with
-// griddepcontrol.wait / launch_dependents, so any of them may also be launched with
-// programmatic stream serialisation (scheduled while the kernel ahead of it finishes) without
-// changing results; only the decode step does that (a step's selection then overlaps the end
-// of the step before it).  For the prefill's chain of kernels it measured slower.
-template <typename... KArgs, typename... Args>
+// Launches `kernel` in stream order, or with PDL = true with programmatic stream
+// serialisation: scheduled while the kernel ahead of it finishes.  Every kernel of this
+// library starts with griddepcontrol.wait / launch_dependents, so either launch gives the
+// same results; the programmatic one hides launch latency.  It is used where the kernel
+// ahead is a short one (inside a chunk's sort chain).  Behind the long persistent kernels
+// (selection, chunk scan), dependents that sat waiting on the SMs made the step slower.
+template <bool PDL = false, typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t st, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
@@ -62,7 +63,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 0;  // plain stream order: overlapped launches measured slower in the prefill
+  cfg.numAttrs = PDL && pdl_enabled() ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
@@ -531,11 +532,11 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
       uint2* va = v0;
       uint2* vb = v1;
       for (int shift = 0; shift < bits; shift += 8) {
-        SDM_CUDA_TRY(launch_pdl(radix_hist_kernel, dim3(ntiles), dim3(RS_THREADS), 0, st,
+        SDM_CUDA_TRY(launch_pdl<true>(radix_hist_kernel, dim3(ntiles), dim3(RS_THREADS), 0, st,
                                 ka, E, shift, hist, ntiles));
-        SDM_CUDA_TRY(launch_pdl(radix_scan_kernel, dim3(RS_BINS), dim3(1024), 0, st,
+        SDM_CUDA_TRY(launch_pdl<true>(radix_scan_kernel, dim3(RS_BINS), dim3(1024), 0, st,
                                 hist, ntiles, tot));
-        SDM_CUDA_TRY(launch_pdl(radix_scatter_kernel, dim3(ntiles), dim3(RS_THREADS), RS_SCATTER_SMEM, st,
+        SDM_CUDA_TRY(launch_pdl<true>(radix_scatter_kernel, dim3(ntiles), dim3(RS_THREADS), RS_SCATTER_SMEM, st,
                                 ka, va, kb, vb, E, shift, hist, tot, ntiles));
         g_launches.fetch_add(3, std::memory_order_relaxed);
         SDM_CUDA_TRY(cudaGetLastError());
@@ -550,7 +551,7 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
       long long lblocks = (nsamp + 255) / 256;
       if (lblocks > (long long)di->sms * 8) lblocks = (long long)di->sms * 8;
       if (lblocks < 1) lblocks = 1;
-      SDM_CUDA_TRY(launch_pdl(slot_long_segments_kernel, dim3((unsigned)lblocks), dim3(256), 0, st,
+      SDM_CUDA_TRY(launch_pdl<true>(slot_long_segments_kernel, dim3((unsigned)lblocks), dim3(256), 0, st,
                               ks, E, cnt, hot, WL.hot_cap));
       g_launches.fetch_add(1, std::memory_order_relaxed);
       SDM_CUDA_TRY(cudaGetLastError());

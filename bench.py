@@ -327,6 +327,15 @@ def bench_prefill(args, dist: Dist, dev):
     return res
 
 
+def step_bytes_of(wl) -> float:
+    """Algorithmic bytes of one decode step of every (sequence, head)."""
+    return wl.B * wl.H * algorithmic_bytes(wl)
+
+
+def per_step_of(secs: float, reps: int, nsteps: int) -> float:
+    return secs / (reps * nsteps)
+
+
 def bench_decode(args, dist: Dist, dev):
     import sparse_memory_linear_b200 as sdm
 
@@ -364,6 +373,10 @@ def bench_decode(args, dist: Dist, dev):
     kernel_s = ms_k / n_k * 1e-3
     out = {
         "workload": wl.note, "steps_per_run": nsteps, "runs": reps,
+        # the step's algorithmic bytes over the step time: consecutive steps overlap (the
+        # selection of a step runs while the step before it drains), so this is above the
+        # per-kernel fraction of `roofline`, whose duration is a launch timed alone
+        "step_roofline_frac": step_bytes_of(wl) / per_step_of(secs, reps, nsteps) / 1e9 / hbm_peak()[0],
         "value": weak_scaling_value(th, per_step, dist.world), "unit": UNIT,
         "us_per_step": per_step * 1e6,
         "roofline": {"kernel": "decode_kernel", "bound": "hbm",
@@ -534,6 +547,7 @@ def main(argv=None):
                        "l2": "inputs larger than L2 (9 GB of inputs, 4 GB state per step)",
                        "step": "sdm_scan_forward with SDM_CONTINUE: select + scan + norm/gate (M0 init timed apart: state_init_ms)"},
             "roofline": pre["roofline"], "whole_step_hbm": pre["whole_step_hbm"],
+            "state_init_ms": pre["state_init_ms"],
             "kernels_ms_per_step": pre["kernels_ms_per_step"],
             "kernel_launches_per_step": pre["kernel_launches_per_step"],
             "kernels_share": pre["kernels_share"],

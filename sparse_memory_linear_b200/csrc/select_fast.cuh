@@ -191,7 +191,7 @@ __device__ inline FastScratch carve_fast_scratch(unsigned char* p, int S1, int S
 template <int R8, int KC>
 __device__ __forceinline__ void half_topk_bf16(const __nv_bfloat16* src, int S, int K, int lane,
                                                uint32_t* surv, uint32_t* stage, uint32_t* hist,
-                                               uint32_t* out, int idx_base = 0) {
+                                               uint32_t* out) {
   constexpr int P = KC / 32;  // enough per-lane leaders for any K <= KC
   const unsigned lt = lanemask_lt();
   uint32_t k[R8][8];
@@ -249,7 +249,7 @@ __device__ __forceinline__ void half_topk_bf16(const __nv_bfloat16* src, int S, 
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       if (k[r][i] >= lo)
-        surv[pos++] = (k[r][i] << 16) | (0xffffu - (uint32_t)(idx_base + r * 256 + lane * 8 + i));
+        surv[pos++] = (k[r][i] << 16) | (0xffffu - (uint32_t)(r * 256 + lane * 8 + i));
     }
     base += __shfl_sync(FULL_MASK, incl, 31);
   }
@@ -285,56 +285,6 @@ __device__ __forceinline__ void half_topk_bf16(const __nv_bfloat16* src, int S, 
     v[q] = p < K ? stage[p] : 0u;
   }
   bitonic_desc_reg<uint32_t, NPL>(v, lane);
-#pragma unroll
-  for (int q = 0; q < NPL; ++q) {
-    const int p = q * 32 + lane;
-    if (p < K) out[p] = v[q];
-  }
-  __syncwarp();
-}
-
-// Top-K of two sorted (descending) lists of K composites, a and b, written sorted to out:
-// the element-wise larger of a[i] and b[K-1-i] forms a bitonic sequence holding the K
-// largest, which half-cleaner stages then sort.  K <= 32*NPL.
-template <int NPL>
-__device__ __forceinline__ void merge_top_sorted(const uint32_t* a, const uint32_t* b, int K,
-                                                 int lane, uint32_t* out) {
-  constexpr int P2 = 32 * NPL;
-  uint32_t v[NPL];
-#pragma unroll
-  for (int q = 0; q < NPL; ++q) {
-    const int p = q * 32 + lane;
-    // pad to P2 with the smallest composite; b reversed within the padded length
-    const uint32_t x = p < K ? a[p] : 0u;
-    const int pr = P2 - 1 - p;
-    const uint32_t y = pr < K ? b[pr] : 0u;
-    v[q] = x > y ? x : y;
-  }
-  // the sequence is bitonic over P2 positions: sort it descending with half-cleaners
-#pragma unroll 1
-  for (int stride = P2 >> 1; stride > 0; stride >>= 1) {
-    if (stride >= 32) {
-      // half-cleaner across registers: every pair (q, q | qs) takes max / min
-#pragma unroll
-      for (int q = 0; q < NPL; ++q) {
-#pragma unroll
-        for (int qs = 1; qs < NPL; qs <<= 1) {
-          if (qs == (stride >> 5) && (q & qs) == 0) {
-            const uint32_t x = v[q], y = v[q | qs];
-            v[q] = x > y ? x : y;
-            v[q | qs] = x > y ? y : x;
-          }
-        }
-      }
-    } else {
-      const bool lower = (lane & stride) == 0;
-#pragma unroll
-      for (int q = 0; q < NPL; ++q) {
-        const uint32_t o = __shfl_xor_sync(FULL_MASK, v[q], stride);
-        v[q] = lower ? (v[q] > o ? v[q] : o) : (v[q] < o ? v[q] : o);
-      }
-    }
-  }
 #pragma unroll
   for (int q = 0; q < NPL; ++q) {
     const int p = q * 32 + lane;

@@ -47,7 +47,7 @@ extern "C" {
 typedef enum {
     SDM_OK = 0,
     SDM_ERR_INVALID_ARG = 1,  /* a pointer, size, alignment or enum is not accepted     */
-    SDM_ERR_UNSUPPORTED = 2,  /* valid request that this build does not implement      */
+    SDM_ERR_UNSUPPORTED = 2,  /* valid request that the library does not implement    */
     SDM_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed            */
     SDM_ERR_DEVICE_CHECK = 4, /* a kernel found an out-of-range index in its inputs     */
     SDM_ERR_TIMEOUT = 5       /* a bounded wait inside a kernel ran out                 */

@@ -218,8 +218,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool bf16 = a.in_bf16 != 0;
   const int S = a.S1 + a.S2;
-  // the next step may be scheduled now: it waits for this grid before its own state access
-  grid_launch_dependents();
   const int d4 = a.d_v / 4;
 
   int32_t* idx_w = reinterpret_cast<int32_t*>(smem + L.off_lists);
@@ -330,6 +328,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
     __syncthreads();
   }
 
+  // The selection is done: the next step may be scheduled now (its CTAs take the SM slots
+  // freed by this step, and their selection overlaps this step's row traffic).
+  grid_launch_dependents();
   // Everything above reads only this step's inputs.  A step launched with programmatic
   // stream serialisation may have started while the step before it still ran: wait for that
   // grid (and its memory) before touching anything it writes (sel_out, M, y, o).

@@ -123,3 +123,12 @@ def test_status_strings(sdm):
     assert sdm.sdm_status_string(0) == "SDM_OK"
     assert sdm.sdm_status_string(4) == "SDM_ERR_DEVICE_CHECK"
     assert sdm.sdm_status_string(99) == "SDM_ERR_UNKNOWN"
+
+
+def test_missing_library_raises_instead_of_falling_back(monkeypatch, tmp_path):
+    """Without the built library every call raises: there is no CPU or torch fallback."""
+    import sparse_memory_linear_b200._binding as B
+    monkeypatch.setattr(B, "_lib", None)
+    monkeypatch.setattr(B, "library_path", str(tmp_path / "libsdm.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        B.library()

@@ -66,3 +66,36 @@ def test_single_process_defaults():
     assert d.world == int(os.environ.get("WORLD_SIZE", "1"))
     assert d.max(3.5) == 3.5
     assert bench.weak_scaling_value(10.0, 2.0, 1) == 5.0
+
+
+def test_measured_traffic_scales_and_expires(tmp_path, monkeypatch):
+    """The roofline's `traffic` comes from the committed capture, scaled to a launch; once
+    the kernel's source no longer has the recorded hash it is reported as null."""
+    import hashlib
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    src = tmp_path / "kernel.cuh"
+    src.write_text("// kernel source\n")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    (tmp_path / "profiles").mkdir()
+    rec = {"k": {"dram_bytes_per_unit": 100, "source": "kernel.cuh", "source_sha256_16": sha}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("k", 512, "dram_bytes_per_unit") == 51200
+    assert bench.measured_traffic("other", 512, "dram_bytes_per_unit") is None
+    src.write_text("// kernel source, changed\n")
+    assert bench.measured_traffic("k", 512, "dram_bytes_per_unit") is None
+
+
+def test_committed_traffic_records_are_well_formed():
+    """profiles/traffic.json names, per kernel, its capture summary, the kernel source and
+    the source hash the capture was taken with (a changed source reports null traffic)."""
+    import json
+    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    assert {"slot_chunk_kernel", "decode_kernel"} <= set(rec)
+    for name, r in rec.items():
+        assert os.path.exists(os.path.join(ROOT, "profiles", r["capture"])), name
+        assert os.path.exists(os.path.join(ROOT, r["source"])), name
+        assert len(r["source_sha256_16"]) == 16, name
+        assert [k for k in r if k.startswith("dram_bytes_per_")], name

@@ -78,9 +78,10 @@ typedef struct {
 sdm_status sdm_select(const void *halves, sdm_shape shape, int32_t K, int32_t *idx, float *wt,
                       void *stream);
 
-/* Bytes of scratch that sdm_scan_forward needs for this shape and engine (the
- * selections of every token: B*T*H*(W+R) indices and weights, plus engine buffers).
- * Returns 0 for an invalid shape. */
+/* Bytes of scratch that sdm_scan_forward needs for this shape and engine: the selections
+ * of every token (B*T*H*(W+R) indices and weights), plus for the slot engine the events of
+ * one time chunk (double-buffered for the radix sort), its histogram and its long-segment
+ * list.  SDM_ENGINE_AUTO reserves room for either engine.  Returns 0 for an invalid shape. */
 size_t sdm_workspace_size(sdm_shape shape, int32_t engine);
 
 /*

@@ -159,30 +159,36 @@ struct FastScratch {
   uint32_t* surv;   // [max(S1, S2)] bracket survivors of one half (composites)
   uint32_t* a;      // [KMAX] first half: sorted composites key16 << 16 | (0xffff - idx)
   uint32_t* b;      // [KMAX] second half
-  float* pv;        // [4 * KMAX] candidate phase: half values and scaled indices
-  uint32_t* stage;  // [KMAX] unsorted winners of a half (u32) / of the candidates (u64)
+  uint32_t* stage;  // [KMAX] unsorted winners of a half (u32)
+  // candidate phase, over the survivors of the halves (no longer needed by then):
+  float* pv;         // [4 * KMAX] half values and scaled indices
+  uint64_t* cstage;  // [KMAX] unsorted winners of the candidates
 };
 
-__host__ __device__ inline size_t fast_scratch_bytes(int S1, int S2, int K) {
+__host__ __device__ inline size_t fast_surv_bytes(int S1, int S2) {
   const int smax = S1 > S2 ? S1 : S2;
+  const size_t surv = (size_t)smax * 4;
+  const size_t cand = 4 * (size_t)KMAX * 4 + (size_t)KMAX * 8;
+  return ((surv > cand ? surv : cand) + 15) / 16 * 16;
+}
+
+__host__ __device__ inline size_t fast_scratch_bytes(int S1, int S2, int K) {
   (void)K;
-  return 256 * 4 + ((size_t)smax * 4 + 15) / 16 * 16 + 2 * (size_t)KMAX * 4 +
-         4 * (size_t)KMAX * 4 + (size_t)KMAX * 8;
+  return 256 * 4 + fast_surv_bytes(S1, S2) + 2 * (size_t)KMAX * 4 + (size_t)KMAX * 4;
 }
 
 __device__ inline FastScratch carve_fast_scratch(unsigned char* p, int S1, int S2, int K) {
   FastScratch s;
-  const int smax = S1 > S2 ? S1 : S2;
   s.hist = reinterpret_cast<uint32_t*>(p);
   p += 256 * 4;
   s.surv = reinterpret_cast<uint32_t*>(p);
-  p += ((size_t)smax * 4 + 15) / 16 * 16;
+  s.pv = reinterpret_cast<float*>(p);
+  s.cstage = reinterpret_cast<uint64_t*>(p + 4 * (size_t)KMAX * 4);
+  p += fast_surv_bytes(S1, S2);
   s.a = reinterpret_cast<uint32_t*>(p);
   p += KMAX * 4;
   s.b = reinterpret_cast<uint32_t*>(p);
   p += KMAX * 4;
-  s.pv = reinterpret_cast<float*>(p);
-  p += 4 * (size_t)KMAX * 4;
   s.stage = reinterpret_cast<uint32_t*>(p);
   return s;
 }
@@ -423,8 +429,7 @@ __device__ __forceinline__ void select_row_fast(const __nv_bfloat16* row, int S1
                                                 int32_t* out_idx, float* out_wt) {
   half_topk_bf16<R8, KC>(row, S1, K, lane, sc.surv, sc.stage, sc.hist, sc.a);
   half_topk_bf16<R8, KC>(row + S1, S2, K, lane, sc.surv, sc.stage, sc.hist, sc.b);
-  cand_topk_bf16<KC>(sc.a, sc.b, K, S2, ctab, lane, sc.pv,
-                     reinterpret_cast<uint64_t*>(sc.stage), sc.hist, out_idx, out_wt);
+  cand_topk_bf16<KC>(sc.a, sc.b, K, S2, ctab, lane, sc.pv, sc.cstage, sc.hist, out_idx, out_wt);
 }
 
 // Whether a row shape takes the fast path, and its template parameters.
@@ -439,7 +444,7 @@ __host__ __device__ inline int fast_kc(int K) { return K <= 32 ? 32 : (K <= 64 ?
 
 // Persistent fast selection kernel over rows of job0 followed by rows of job1.
 template <int R8, int KC>
-__global__ void __launch_bounds__(256, 3) sel_fast_kernel(SelJob job0, SelJob job1, long long n_rows,
+__global__ void __launch_bounds__(256, 4) sel_fast_kernel(SelJob job0, SelJob job1, long long n_rows,
                                                        int njobs, int S1, int S2) {
   // wait for the kernel ahead in the stream (programmatic launch), then let the next one in
   grid_dependency_wait();

@@ -5,12 +5,12 @@
 // (paper.rainbus.top summary), method step 1; ai-paper-analysis.pages.dev SDM write-up,
 // 步骤 1.  Per half, per warp:
 //   1. 16-byte loads; lane l holds elements r*256 + 8l + i as 16-bit order keys;
-//   2. every lane keeps its P = ceil(K/32) largest keys; the K-th largest key T lies between
-//      the smallest and the largest of the lanes' P-th largest keys (each lane then has at
-//      least P keys >= the smallest, and fewer than 32(P-1) < K keys exceed the largest);
-//   3. keys inside that bracket are compacted to shared memory in index order; histogram
-//      levels (256 bins over the bracket, then over the bin that holds it) find the K-th
-//      largest key T, and the top K are the keys > T plus the lowest-index ties;
+//   2. every lane keeps its P = ceil(K/32) largest keys; the K-th largest key T is at least
+//      the smallest of the lanes' P-th largest keys (every lane has P keys at or above it),
+//      and at most the largest key;
+//   3. keys in that bracket are compacted to shared memory in index order; histogram levels
+//      (256 bins over the bracket, then over the bin that holds T) find T, and the top K are
+//      the keys > T plus the lowest-index ties;
 //   4. a register bitonic sort (shuffles) orders them: (key desc, index asc).
 // Candidates: the rank pairs with (r1+1)(r2+1) <= K; their K-th largest sum is at least
 // both A[K-1] + B[0] and A[0] + B[K-1] (K candidate sums reach each), which brackets the same
@@ -153,7 +153,8 @@ __device__ __forceinline__ void bitonic_desc_reg(V (&v)[NPL], int lane) {
   }
 }
 
-// Shared scratch of one warp of the fast path.
+// Shared scratch of one warp of the fast path (6.5 KB for halves of 1024: four warps'
+// CTAs of 8 warps fit one SM).
 struct FastScratch {
   uint32_t* hist;   // [256] threshold histogram, zero between uses
   uint32_t* surv;   // [max(S1, S2)] bracket survivors of one half (composites)

@@ -8,7 +8,8 @@
 //   and read selection, first and second half) find the half's top K with the group
 //   selection of select_group.cuh; four warps per selection then take the top K of the
 //   rank-pair candidate sums the same way and write slot indices and softmax weights.
-//   Other shapes: warps 0 and 1 run the warp-per-row selection of select.cuh;
+//   Other shapes: warps 0 and 1 run the warp-per-row selection of select.cuh.
+//   CTAs 0 .. 63 also prefetch into L2 the inputs of the CTAs dispatched after them;
 //   steps 2 and 3 issue every row load of the token at once: each warp's write rows go to
 //   shared memory (over the dead selection scratch) by cp.async and its first read rows to
 //   registers, so the step waits for one memory latency;
@@ -102,6 +103,52 @@ inline DecLayout dec_layout(int S1, int S2, int W, int R, int d_v, bool group) {
   if (L.rows_smem && scratch + rows_bytes > p) p = scratch + rows_bytes;
   L.total = static_cast<uint32_t>(p);
   return L;
+}
+
+// CTAs 0 .. DEC_PF_CTAS - 1 are dispatched first and prefetch for the others (a 64 x 8
+// batch at 4 CTAs per SM leaves 80 of the 592 slots free for the next step's first CTAs).
+constexpr int DEC_PF_CTAS = 64;
+
+// L2 prefetch of the 128-byte lines of [p, p + bytes) by the lanes of one warp; every
+// address prefetched lies inside the span.
+__device__ __forceinline__ void prefetch_l2_span(const void* p, size_t bytes, int lane) {
+  const uintptr_t s = reinterpret_cast<uintptr_t>(p);
+  const uintptr_t first = s & ~static_cast<uintptr_t>(127);
+  const int nl = static_cast<int>((s + bytes - first + 127) >> 7);
+  for (int l = lane; l < nl; l += 32) {
+    const uintptr_t ad = l == 0 ? s : first + (static_cast<uintptr_t>(l) << 7);
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(ad));
+  }
+}
+
+// The CTAs dispatched first warm L2 with the step inputs (score halves, v, gate, alpha,
+// beta) of units bh + DEC_PF_CTAS, bh + 2 DEC_PF_CTAS, ...  Under programmatic launch the
+// later CTAs of a step start only as the previous step's CTAs leave the SMs, and their
+// score loads would otherwise add a DRAM round trip to the step's critical path.
+__device__ __forceinline__ void dec_prefetch_later_units(const DecodeArgs& a, int bh, int warp,
+                                                         int lane) {
+  if (bh >= DEC_PF_CTAS) return;
+  const size_t esz = a.in_bf16 ? 2 : 4;
+  const size_t srow = static_cast<size_t>(a.S1 + a.S2) * esz;
+  const size_t vrow = static_cast<size_t>(a.d_v) * esz;
+  const int nu = (a.BH - 1 - bh) / DEC_PF_CTAS;
+  for (int t = warp; t < 4 * nu; t += DEC_WARPS) {
+    const int u = bh + DEC_PF_CTAS * (1 + (t >> 2));
+    switch (t & 3) {
+      case 0: prefetch_l2_span(static_cast<const char*>(a.kp) + u * srow, srow, lane); break;
+      case 1: prefetch_l2_span(static_cast<const char*>(a.qp) + u * srow, srow, lane); break;
+      case 2:
+        prefetch_l2_span(static_cast<const char*>(a.v) + u * vrow, vrow, lane);
+        if (lane == 0) {
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(a.alpha + u));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(a.beta + u));
+        }
+        break;
+      default:
+        if (a.gate) prefetch_l2_span(static_cast<const char*>(a.gate) + u * vrow, vrow, lane);
+        break;
+    }
+  }
 }
 
 // Step 1 by the group selection: warps 2g, 2g + 1 take half g (0 write first, 1 write second,
@@ -264,6 +311,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
       gr[q] = c < a.d_v && a.gate ? load_in(a.gate, (size_t)bh * a.d_v + c, bf16) : 0.0f;
     }
     if (tid < 2) abr = tid == 0 ? a.alpha[bh] : a.beta[bh];
+    dec_prefetch_later_units(a, bh, warp, lane);
     // shared state of the group selection: this group's histogram and control words
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L.off_hist);
     GroupCtl* ctl = reinterpret_cast<GroupCtl*>(smem + L.off_ctl);
@@ -293,6 +341,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
       key[i] = (i >> 3) * 512 + gt * 8 + (i & 7) < Sh ? bf16_key16(key[i]) : 0u;
     decode_select_group<E, KC>(a, L, smem, tid, key, idx_w, wt_w, idx_r, wt_r);
   } else {
+    dec_prefetch_later_units(a, bh, warp, lane);
     const int kmax = a.W > a.R ? a.W : a.R;
     const size_t esz = bf16 ? 2 : 4;
     if (tid < 128) reinterpret_cast<uint32_t*>(smem + L.off_bits)[tid] = 0u;

@@ -8,7 +8,8 @@ sparse read and RMSNorm + gate.  Reported as token*heads/s (whole job), beside t
 roofline of the scan kernel, the end-to-end figure through the C ABI with host buffers,
 and the CPU oracle timed on the host cores.  A second object reports decode on the
 batched-decode workload (64 sequences x 8 heads, N=262144, d_v=128): 256 successive
-sdm_decode_step calls, as plain launches and replayed from a CUDA graph.
+sdm_decode_step_chained calls over inputs staged on the device beforehand (each step's
+selection may overlap the step before), as plain launches and replayed from a CUDA graph.
 
 Multi-GPU: the pass has no exchange step (every (sequence, head) is independent), so each
 rank runs its own batch of the same shape (weak scaling), timed between barriers and
@@ -353,7 +354,8 @@ def bench_decode(args, dist: Dist, dev):
     def run_all():
         for s in steps:
             sdm.sdm_decode_step(s["kp"], s["qp"], s["v"], s["alpha"], s["beta"], M, W=wl.W,
-                                R=wl.R, S1=wl.S1, gate=s["gate"], y=y, o=o, stream=stream)
+                                R=wl.R, S1=wl.S1, gate=s["gate"], y=y, o=o, stream=stream,
+                                chained=True)
 
     reps = max(1, args.steps // 2)
     # plain launches, timed without the library's per-launch events (these would sit between
@@ -373,6 +375,7 @@ def bench_decode(args, dist: Dist, dev):
     kernel_s = ms_k / n_k * 1e-3
     out = {
         "workload": wl.note, "steps_per_run": nsteps, "runs": reps,
+        "launch": "sdm_decode_step_chained (programmatic stream serialisation)",
         # the step's algorithmic bytes over the step time: consecutive steps overlap (the
         # selection of a step runs while the step before it drains), so this is above the
         # per-kernel fraction of `roofline`, whose duration is a launch timed alone
@@ -399,7 +402,7 @@ def bench_decode(args, dist: Dist, dev):
             for s in steps:
                 sdm.sdm_decode_step(s["kp"], s["qp"], s["v"], s["alpha"], s["beta"], M,
                                     W=wl.W, R=wl.R, S1=wl.S1, gate=s["gate"], y=y, o=o,
-                                    stream=side)
+                                    stream=side, chained=True)
         secs_g = timed(graph.replay, reps, 1, dist, stream)
         out["graph_us_per_step"] = secs_g / (reps * nsteps) * 1e6
         out["graph_value"] = weak_scaling_value(th, secs_g / (reps * nsteps), dist.world)

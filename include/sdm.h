@@ -158,18 +158,31 @@ sdm_status sdm_scan_forward_noalloc(const void *kp, const void *qp, const void *
  *   alpha, beta [B,H] fp32; M [B,H,N,d_v] fp32 in/out; y [B,H,d_v] fp32 out;
  *   o [B,H,d_v] fp32 out, nullable; gamma [d_v] nullable;
  *   sel_out nullable: write slots [B,H,W] followed by read slots [B,H,R].
- * shape.T is ignored.  No scratch memory is used.
- * The launch allows programmatic stream serialisation: the step's selection, which reads only
- * kp, qp, v, gate, alpha, beta and gamma, may run while the kernel ahead of it on the stream
- * (typically the previous decode step) is finishing.  The step waits for that kernel before
- * it touches M, y, o or sel_out.  A step's inputs therefore must not be the outputs (M, y, o,
- * sel_out) of the kernel launched right before it.  SDM_NO_PDL=1 in the environment turns
- * this off.
+ * shape.T is ignored.  No scratch memory is used.  The kernel is launched in plain stream
+ * order: it starts once the work ahead of it on the stream has finished.
  */
 sdm_status sdm_decode_step(const void *kp, const void *qp, const void *v, const float *alpha,
                            const float *beta, float *M, float *y, const void *gate,
                            const float *gamma, float eps, int32_t act, float *o,
                            int32_t *sel_out, sdm_shape shape, void *stream);
+
+/*
+ * sdm_decode_step for a chain of decode steps whose inputs are all in device memory before
+ * the chain starts (same arguments, same results).  The launch allows programmatic stream
+ * serialisation: the step's selection, which reads only kp, qp, v, gate, alpha, beta and
+ * gamma, may run while the kernel ahead of it on the stream is finishing (typically the
+ * previous step), and the step waits for that kernel before it touches M, y, o or sel_out.
+ * Precondition, which the library cannot check: the kernel launched right before this one
+ * writes none of this step's inputs.  A kernel that produces them (a projection, for
+ * instance) may let its dependents start before its own stores are visible; after such a
+ * kernel call sdm_decode_step instead.  SDM_NO_PDL=1 in the environment makes this call
+ * launch in plain stream order.
+ */
+sdm_status sdm_decode_step_chained(const void *kp, const void *qp, const void *v,
+                                   const float *alpha, const float *beta, float *M, float *y,
+                                   const void *gate, const float *gamma, float eps,
+                                   int32_t act, float *o, int32_t *sel_out, sdm_shape shape,
+                                   void *stream);
 
 /*
  * Step 4 alone [paper.rainbus.top summary, method step 4]: for each of the B*T*H rows

@@ -53,6 +53,7 @@ def library():
         "sdm_state_init": ([P, P, S, P], I),
         "sdm_scan_forward": ([P, P, P, P, P, P, P, I, P, P, P, F, I, P, P, I, P, Z, S, P], I),
         "sdm_decode_step": ([P, P, P, P, P, P, P, P, P, F, I, P, P, S, P], I),
+        "sdm_decode_step_chained": ([P, P, P, P, P, P, P, P, P, F, I, P, P, S, P], I),
         "sdm_norm_gate": ([P, P, P, F, I, S, P, P], I),
         "sdm_get_device_status": ([P], I),
         "sdm_status_string": ([I], ctypes.c_char_p),
@@ -195,9 +196,12 @@ def sdm_scan_forward(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | Non
 
 def sdm_decode_step(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | None = None,
                     y=None, gate=None, gamma=None, eps: float = 1e-6, act: str = "silu", o=None,
-                    want_o: bool = True, sel_out=None, want_sel: bool = False, stream=None):
+                    want_o: bool = True, sel_out=None, want_sel: bool = False, stream=None,
+                    chained: bool = False):
     """One token for each (b, h).  kp, qp [B,H,S1+S2]; v, gate [B,H,d_v]; alpha, beta [B,H];
-    M [B,H,N,d_v] in/out.  Returns dict(y, o, sel)."""
+    M [B,H,N,d_v] in/out.  Returns dict(y, o, sel).  chained=True calls
+    sdm_decode_step_chained: only when the kernel launched right before on the stream writes
+    none of this step's inputs (a chain of steps over inputs already on the device)."""
     dev = kp.device
     _need(kp, "kp", device=dev)
     dt = kp.dtype
@@ -218,10 +222,10 @@ def sdm_decode_step(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | None
         o = torch.empty((B, H, d_v), dtype=torch.float32, device=dev)
     if sel_out is None and want_sel:
         sel_out = torch.empty(B * H * (W + R), dtype=torch.int32, device=dev)
-    _check(library().sdm_decode_step(
+    name = "sdm_decode_step_chained" if chained else "sdm_decode_step"
+    _check(getattr(library(), name)(
         _p(kp), _p(qp), _p(v), _p(alpha), _p(beta), _p(M), _p(y), _p(gate), _p(gamma),
-        float(eps), ACT[act], _p(o), _p(sel_out), shape, _stream(stream, dev)),
-        "sdm_decode_step")
+        float(eps), ACT[act], _p(o), _p(sel_out), shape, _stream(stream, dev)), name)
     return dict(y=y, o=o, sel=sel_out)
 
 

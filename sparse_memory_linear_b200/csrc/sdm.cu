@@ -36,7 +36,7 @@ constexpr size_t WS_ALIGN = 256;
     }                                            \
   } while (0)
 
-// SDM_NO_PDL=1 launches the decode step in plain stream order (for comparison).
+// SDM_NO_PDL=1 launches every kernel in plain stream order, sdm_decode_step_chained included.
 inline bool pdl_enabled() {
   static const bool on = [] {
     const char* e = getenv("SDM_NO_PDL");
@@ -746,10 +746,11 @@ sdm_status sdm_scan_forward(const void* kp, const void* qp, const void* v, const
   return SDM_OK;
 }
 
-sdm_status sdm_decode_step(const void* kp, const void* qp, const void* v, const float* alpha,
-                           const float* beta, float* M, float* y, const void* gate,
-                           const float* gamma, float eps, int32_t act, float* o,
-                           int32_t* sel_out, sdm_shape shape, void* stream) {
+// One decode step; `chained` launches it with programmatic stream serialisation.
+static sdm_status decode_step(const void* kp, const void* qp, const void* v, const float* alpha,
+                              const float* beta, float* M, float* y, const void* gate,
+                              const float* gamma, float eps, int32_t act, float* o,
+                              int32_t* sel_out, sdm_shape shape, void* stream, bool chained) {
   sdm_shape s = shape;
   s.T = 1;
   if (!shape_ok(s, false)) return SDM_ERR_INVALID_ARG;
@@ -793,9 +794,9 @@ sdm_status sdm_decode_step(const void* kp, const void* qp, const void* v, const 
   a.in_bf16 = s.in_dtype == SDM_BF16;
   ProfScope ps(SDM_KERNEL_DECODE, static_cast<cudaStream_t>(stream));
   bool launched = false;
-  // Programmatic stream serialisation: the step's selection (which reads only its inputs)
-  // may overlap the end of the kernel ahead of it; the kernel waits for that kernel before
-  // its first state access.
+  // Chained: programmatic stream serialisation.  The step's selection (which reads only its
+  // inputs) may then overlap the end of the kernel ahead of it; the kernel waits for that
+  // kernel before its first state access.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.BH);
   cfg.blockDim = dim3(DEC_THREADS);
@@ -805,7 +806,7 @@ sdm_status sdm_decode_step(const void* kp, const void* qp, const void* v, const 
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cfg.numAttrs = chained && pdl_enabled() ? 1 : 0;
 #define SDM_DEC_LAUNCH(E, KC, NQ)                                                        \
   if (!launched && SDM_DEC_FITS(E, KC, NQ)) {                                             \
     SDM_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_kernel<E, KC, NQ>, a, L));              \
@@ -818,6 +819,22 @@ sdm_status sdm_decode_step(const void* kp, const void* qp, const void* v, const 
   if (!launched) return SDM_ERR_UNSUPPORTED;
   SDM_CUDA_TRY(cudaGetLastError());
   return SDM_OK;
+}
+
+sdm_status sdm_decode_step(const void* kp, const void* qp, const void* v, const float* alpha,
+                           const float* beta, float* M, float* y, const void* gate,
+                           const float* gamma, float eps, int32_t act, float* o,
+                           int32_t* sel_out, sdm_shape shape, void* stream) {
+  return decode_step(kp, qp, v, alpha, beta, M, y, gate, gamma, eps, act, o, sel_out, shape,
+                     stream, false);
+}
+
+sdm_status sdm_decode_step_chained(const void* kp, const void* qp, const void* v,
+                                   const float* alpha, const float* beta, float* M, float* y,
+                                   const void* gate, const float* gamma, float eps, int32_t act,
+                                   float* o, int32_t* sel_out, sdm_shape shape, void* stream) {
+  return decode_step(kp, qp, v, alpha, beta, M, y, gate, gamma, eps, act, o, sel_out, shape,
+                     stream, true);
 }
 
 sdm_status sdm_get_device_status(void* stream) {

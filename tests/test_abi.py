@@ -103,11 +103,12 @@ def test_decode_and_select_and_norm_reject_bad_arguments(sdm):
     lib = sdm.library()
     P = ctypes.c_void_p
     s = good_shape(sdm)
-    # decode: missing M, then misaligned v
-    assert lib.sdm_decode_step(P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), None, P(FAKE),
-                               None, None, 1e-6, 0, None, None, s, None) == 1
-    assert lib.sdm_decode_step(P(FAKE), P(FAKE), P(FAKE + 4), P(FAKE), P(FAKE), P(FAKE),
-                               P(FAKE), None, None, 1e-6, 0, None, None, s, None) == 1
+    # decode, plain and chained: missing M, then misaligned v
+    for fn in (lib.sdm_decode_step, lib.sdm_decode_step_chained):
+        assert fn(P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), None, P(FAKE),
+                  None, None, 1e-6, 0, None, None, s, None) == 1
+        assert fn(P(FAKE), P(FAKE), P(FAKE + 4), P(FAKE), P(FAKE), P(FAKE),
+                  P(FAKE), None, None, 1e-6, 0, None, None, s, None) == 1
     # select: K out of range, null output
     assert lib.sdm_select(P(FAKE), s, 0, P(FAKE), P(FAKE), None) == 1
     assert lib.sdm_select(P(FAKE), s, 33, P(FAKE), P(FAKE), None) == 1

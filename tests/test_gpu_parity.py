@@ -253,13 +253,19 @@ def test_scan_long_skew_sampled(sdm, engine):
 
 
 # ------------------------------------------------------------------------- decode
-def decode_steps(sdm, wl, steps, M, gamma=None):
+def decode_steps(sdm, wl, steps, M, gamma=None, chained=False):
+    """One sdm_decode_step per step, or with chained=True one sdm_decode_step_chained per
+    step over inputs staged on the device before the first launch."""
     ys, os_, sels = [], [], []
-    for s in steps:
-        gs = {k: t.to(DEV) for k, t in s.items() if k != "M0"}
+    staged = [{k: t.to(DEV) for k, t in s.items() if k != "M0"} for s in steps] if chained \
+        else None
+    if chained:
+        torch.cuda.synchronize()
+    for i, s in enumerate(steps):
+        gs = staged[i] if chained else {k: t.to(DEV) for k, t in s.items() if k != "M0"}
         out = sdm.sdm_decode_step(gs["kp"], gs["qp"], gs["v"], gs["alpha"], gs["beta"], M,
                                   W=wl.W, R=wl.R, S1=wl.S1, gate=gs.get("gate"), gamma=gamma,
-                                  want_sel=True)
+                                  want_sel=True, chained=chained)
         ys.append(out["y"])
         os_.append(out["o"])
         sels.append(out["sel"])
@@ -346,8 +352,23 @@ def test_decode_equals_scan(sdm):
     assert_close(host(Md), host(Ms), "decode vs scan M", atol=1e-6, rtol=1e-5)
 
 
+def test_decode_chained_equals_plain(sdm):
+    """Chained launches (each step's selection overlapping the step before) give the plain
+    launches' results bit for bit."""
+    wl = sdm_synth.WORKLOADS["decode"].replace(B=16, T=12, S1=256, S2=256, seed=31)
+    steps = [sdm_synth.make_inputs(wl, step=s) for s in range(wl.T)]
+    M0 = steps[0]["M0"].to(DEV)
+    Mp = M0.unsqueeze(0).expand(wl.B, -1, -1, -1).contiguous()
+    Mc = Mp.clone()
+    y_p, o_p, sel_p = decode_steps(sdm, wl, steps, Mp)
+    y_c, o_c, sel_c = decode_steps(sdm, wl, steps, Mc, chained=True)
+    for a, b in zip(sel_p, sel_c):
+        assert torch.equal(a, b)
+    assert torch.equal(y_p, y_c) and torch.equal(o_p, o_c) and torch.equal(Mp, Mc)
+
+
 def test_decode_full_size_sampled(sdm):
-    """The batched-decode workload at full size (64 GB state), a few steps."""
+    """The batched-decode workload at full size (64 GB state), a few chained steps."""
     wl = sdm_synth.WORKLOADS["decode"]
     nsteps = 3
     steps = [{k: t.to(DEV) for k, t in sdm_synth.make_inputs(wl, step=s).items()}
@@ -355,7 +376,7 @@ def test_decode_full_size_sampled(sdm):
     M0 = steps[0]["M0"]
     M = torch.empty((wl.B, wl.H, wl.N, wl.d_v), dtype=F32, device=DEV)
     sdm.sdm_state_init(M0, M)
-    y, o, sels = decode_steps(sdm, wl, steps, M)
+    y, o, sels = decode_steps(sdm, wl, steps, M, chained=True)
     st = lambda k, b, h: np.stack([host(s[k][b, h]) for s in steps], 0)  # noqa: E731
     for (b, h) in [(0, 0), (63, 7), (17, 3)]:
         kp = st("kp", b, h)[None, :, None]

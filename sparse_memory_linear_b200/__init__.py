@@ -16,12 +16,14 @@ from ._binding import (  # noqa: F401
     library,
     library_path,
     sdm_decode_step,
+    sdm_decode_step_chained,
     sdm_get_device_status,
     sdm_launch_count,
     sdm_norm_gate,
     sdm_profile_enable,
     sdm_profile_read,
     sdm_scan_forward,
+    sdm_scan_forward_noalloc,
     sdm_select,
     sdm_state_init,
     sdm_status_string,

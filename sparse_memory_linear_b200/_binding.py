@@ -54,6 +54,7 @@ def library():
         "sdm_scan_forward": ([P, P, P, P, P, P, P, I, P, P, P, F, I, P, P, I, P, Z, S, P], I),
         "sdm_decode_step": ([P, P, P, P, P, P, P, P, P, F, I, P, P, S, P], I),
         "sdm_decode_step_chained": ([P, P, P, P, P, P, P, P, P, F, I, P, P, S, P], I),
+        "sdm_scan_forward_noalloc": ([P, P, P, P, P, P, P, I, P, P, P, F, I, P, P, S, P], I),
         "sdm_norm_gate": ([P, P, P, F, I, S, P, P], I),
         "sdm_get_device_status": ([P], I),
         "sdm_status_string": ([I], ctypes.c_char_p),
@@ -151,14 +152,10 @@ def sdm_state_init(M0: torch.Tensor, M: torch.Tensor, *, d_v: int | None = None,
     return M
 
 
-def sdm_scan_forward(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | None = None,
-                     M0=None, init: str = "m0", y=None, gate=None, gamma=None,
-                     eps: float = 1e-6, act: str = "silu", o=None, want_o: bool = True,
-                     sel_out=None, want_sel: bool = False, engine: str = "auto", ws=None,
-                     stream=None):
-    """Prefill over T tokens.  kp, qp [B,T,H,S1+S2]; v, gate [B,T,H,d_v]; alpha, beta
-    [B,T,H]; M [B,H,N,d_v] (in/out); M0 [H,N,d_v] (init="m0").
-    Returns dict(y, o, sel): sel holds [B,T,H,W] write slots then [B,T,H,R] read slots."""
+def _scan_outputs(kp, qp, v, alpha, beta, M, W, R, S1, M0, y, gate, gamma, o, want_o,
+                  sel_out, want_sel):
+    """Checks the prefill arguments and allocates the missing outputs; returns
+    (shape, y, o, sel_out)."""
     dev = kp.device
     _need(kp, "kp", device=dev)
     dt = kp.dtype
@@ -183,6 +180,20 @@ def sdm_scan_forward(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | Non
     _need(y, "y", torch.float32, dev)
     _need(o, "o", torch.float32, dev)
     _need(sel_out, "sel_out", torch.int32, dev)
+    return shape, y, o, sel_out
+
+
+def sdm_scan_forward(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | None = None,
+                     M0=None, init: str = "m0", y=None, gate=None, gamma=None,
+                     eps: float = 1e-6, act: str = "silu", o=None, want_o: bool = True,
+                     sel_out=None, want_sel: bool = False, engine: str = "auto", ws=None,
+                     stream=None):
+    """Prefill over T tokens.  kp, qp [B,T,H,S1+S2]; v, gate [B,T,H,d_v]; alpha, beta
+    [B,T,H]; M [B,H,N,d_v] (in/out); M0 [H,N,d_v] (init="m0").
+    Returns dict(y, o, sel): sel holds [B,T,H,W] write slots then [B,T,H,R] read slots."""
+    dev = kp.device
+    shape, y, o, sel_out = _scan_outputs(kp, qp, v, alpha, beta, M, W, R, S1, M0, y, gate,
+                                         gamma, o, want_o, sel_out, want_sel)
     need = sdm_workspace_size(shape, engine)
     if ws is None:
         ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
@@ -191,6 +202,25 @@ def sdm_scan_forward(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | Non
         _p(kp), _p(qp), _p(v), _p(alpha), _p(beta), _p(M0), _p(M), INIT[init], _p(y), _p(gate),
         _p(gamma), float(eps), ACT[act], _p(o), _p(sel_out), ENGINE[engine], _p(ws),
         ws.numel(), shape, _stream(stream, dev)), "sdm_scan_forward")
+    return dict(y=y, o=o, sel=sel_out)
+
+
+def sdm_scan_forward_noalloc(kp, qp, v, alpha, beta, M, *, W: int, R: int,
+                             S1: int | None = None, M0=None, init: str = "m0", y=None,
+                             gate=None, gamma=None, eps: float = 1e-6, act: str = "silu",
+                             o=None, want_o: bool = True, sel_out=None, want_sel: bool = False,
+                             stream=None):
+    """sdm_scan_forward with the sequential engine and the library's own fixed scratch array
+    instead of a workspace (no device allocation by the library; at most 16384 rows of
+    (sequence, token, head) with W = R = 64).  Outputs that are not given are allocated
+    here, before the call."""
+    dev = kp.device
+    shape, y, o, sel_out = _scan_outputs(kp, qp, v, alpha, beta, M, W, R, S1, M0, y, gate,
+                                         gamma, o, want_o, sel_out, want_sel)
+    _check(library().sdm_scan_forward_noalloc(
+        _p(kp), _p(qp), _p(v), _p(alpha), _p(beta), _p(M0), _p(M), INIT[init], _p(y), _p(gate),
+        _p(gamma), float(eps), ACT[act], _p(o), _p(sel_out), shape, _stream(stream, dev)),
+        "sdm_scan_forward_noalloc")
     return dict(y=y, o=o, sel=sel_out)
 
 
@@ -227,6 +257,12 @@ def sdm_decode_step(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | None
         _p(kp), _p(qp), _p(v), _p(alpha), _p(beta), _p(M), _p(y), _p(gate), _p(gamma),
         float(eps), ACT[act], _p(o), _p(sel_out), shape, _stream(stream, dev)), name)
     return dict(y=y, o=o, sel=sel_out)
+
+
+def sdm_decode_step_chained(kp, qp, v, alpha, beta, M, **kw):
+    """sdm_decode_step(..., chained=True): the launch may overlap the kernel ahead of it,
+    which must write none of this step's inputs."""
+    return sdm_decode_step(kp, qp, v, alpha, beta, M, chained=True, **kw)
 
 
 def sdm_norm_gate(y, *, gate=None, gamma=None, eps: float = 1e-6, act: str = "silu", o=None,

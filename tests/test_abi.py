@@ -33,6 +33,28 @@ def test_exports_every_declared_symbol(sdm):
         assert hasattr(lib, n), n
 
 
+def declared_parameter_counts():
+    src = open(os.path.join(ROOT, "include", "sdm.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for name, params in re.findall(r"\b(sdm_\w+)\s*\(([^)]*)\)\s*;", src):
+        params = params.strip()
+        out[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_has_every_declared_call_with_its_signature(sdm):
+    """Each call of the header has a Python function of the same name, and the ctypes
+    prototype the binding gives it has the header's number of parameters."""
+    import sparse_memory_linear_b200 as pkg
+    counts = declared_parameter_counts()
+    assert set(counts) == set(declared_functions())
+    lib = sdm.library()
+    for name, n in counts.items():
+        assert callable(getattr(pkg, name, None)), name
+        assert len(getattr(lib, name).argtypes) == n, name
+
+
 def test_library_is_the_in_tree_build(sdm):
     sdm.library()
     maps = open("/proc/self/maps").read()

@@ -60,11 +60,16 @@ def test_noalloc_equals_workspace_entry_point_twice(lib):
         y = torch.full_like(ref["y"], float("nan"))
         o = torch.full_like(ref["o"], float("nan"))
         sel = torch.full_like(ref["sel"], -1)
-        rc = L.sdm_scan_forward_noalloc(
-            _p(g["kp"]), _p(g["qp"]), _p(g["v"]), _p(g["alpha"]), _p(g["beta"]), _p(g["M0"]),
-            _p(M), 0, _p(y), _p(g["gate"]), _p(g["gamma"]), 1e-6, 0, _p(o), _p(sel), shape,
-            stream)
-        assert rc == 0, sdm.sdm_status_string(rc)
+        if call == 0:  # the C entry point itself
+            rc = L.sdm_scan_forward_noalloc(
+                _p(g["kp"]), _p(g["qp"]), _p(g["v"]), _p(g["alpha"]), _p(g["beta"]),
+                _p(g["M0"]), _p(M), 0, _p(y), _p(g["gate"]), _p(g["gamma"]), 1e-6, 0, _p(o),
+                _p(sel), shape, stream)
+            assert rc == 0, sdm.sdm_status_string(rc)
+        else:  # through the Python binding of the same name
+            sdm.sdm_scan_forward_noalloc(g["kp"], g["qp"], g["v"], g["alpha"], g["beta"], M,
+                                         W=wl.W, R=wl.R, M0=g["M0"], y=y, gate=g["gate"],
+                                         gamma=g["gamma"], o=o, sel_out=sel)
         torch.cuda.synchronize()
         assert sdm.sdm_get_device_status() == 0
         assert torch.equal(sel, ref["sel"]), f"call {call}: selected slots differ"

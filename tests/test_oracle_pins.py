@@ -132,6 +132,27 @@ def test_select_sample_tokens_of_tiny_and_small_workloads():
             np.testing.assert_array_equal(idx[r], want_idx)
 
 
+def test_select_route_when_sums_round():
+    """Hand-derived rows whose candidate sums round onto one another
+    (tests/golden/route_collisions.json): the oracle's product-key route keeps the top K of
+    every half, then the lowest slots among equal candidate sums; the definition mode takes
+    the top K of all sums.  The fixture also records what the rank-pair pruning alone gives,
+    which the selection kernels must not return."""
+    g = json.load(open(os.path.join(GOLDEN, "route_collisions.json")))
+    for c in g["cases"]:
+        a = np.array(c["a"], np.float32)
+        b = np.array(c["b"], np.float32)
+        row = np.concatenate([a, b])[None]
+        idx, wt = oracle.select(row, a.size, c["K"])
+        np.testing.assert_array_equal(idx[0], c["expect_route"])
+        np.testing.assert_array_equal(wt[0], c["expect_wt"])
+        idx_all, _ = oracle.select(row, a.size, c["K"], mode="brute_force")
+        np.testing.assert_array_equal(idx_all[0], c["expect_all_sums"])
+        want_all, _ = brute_force_topk(row[0], a.size, c["K"])
+        np.testing.assert_array_equal(idx_all[0], want_all)
+        assert c["expect_pruned_only"] != c["expect_route"]
+
+
 # -------------------------------------------------------------- slot weights (softmax)
 def test_weights_are_softmax_over_selected_set():
     rng = np.random.default_rng(11)

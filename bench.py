@@ -481,8 +481,8 @@ def run_reference(args, dist: Dist):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded counter-based generator)",
         "config": {"workload": wl.name, "shape": wl.note},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores,
+                         "host_cores": os.cpu_count(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -567,9 +567,12 @@ def main(argv=None):
         if not args.no_cpu_baseline and dist.world == 1 and dist.rank == 0:
             n, s, cores = oracle_sample_time(wl, args.cpu_tokens, os.cpu_count() or 1, g)
             line["cpu_baseline"] = {
-                "value": n / s, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "value": n / s, "unit": UNIT, "cores": cores, "host_cores": os.cpu_count(),
+                "kind": "oracle",
                 "sample": f"first {args.cpu_tokens} tokens of sequence 0, all {wl.H} heads "
-                          f"({n} token-heads, {s:.1f} s wall, one head per thread)"}
+                          f"({n} token-heads, {s:.1f} s wall, one head per thread: the "
+                          f"recurrence of a head is sequential, so {cores} of the "
+                          f"{os.cpu_count()} host cores have work)"}
         del g
         torch.cuda.empty_cache()
         if not args.no_decode:

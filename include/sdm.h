@@ -175,7 +175,7 @@ sdm_status sdm_decode_step(const void *kp, const void *qp, const void *v, const 
  * Precondition, which the library cannot check: the kernel launched right before this one
  * writes none of this step's inputs.  A kernel that produces them (a projection, for
  * instance) may let its dependents start before its own stores are visible; after such a
- * kernel call sdm_decode_step instead.  SDM_NO_PDL=1 in the environment makes this call
+ * kernel call sdm_decode_step instead.  sdm_set_option(SDM_OPT_NO_PDL, 1) makes this call
  * launch in plain stream order.
  */
 sdm_status sdm_decode_step_chained(const void *kp, const void *qp, const void *v,
@@ -214,6 +214,31 @@ sdm_status sdm_profile_enable(int32_t on);
  * sdm_kernel_kind, the summed device time in milliseconds (ms[SDM_KERNEL_KINDS]) and the
  * number of launches (launches[SDM_KERNEL_KINDS]); then forgets them. */
 sdm_status sdm_profile_read(double *ms, int64_t *launches);
+
+/* Process-wide launch options, for testing and tuning; every option defaults to 0, which
+ * is what normal use wants.  The library reads no environment variable: these calls are
+ * the only switches.  A value applies to the calls made after it is set, on every device
+ * and stream of the process; set options before any stream capture and not while another
+ * host thread is calling the library. */
+typedef enum {
+    SDM_OPT_NO_PDL = 1,             /* 1: every kernel in plain stream order, including
+                                       sdm_decode_step_chained                          */
+    SDM_OPT_SELECT_GENERAL = 2,     /* 1: bf16 rows also take the general selection path
+                                       (same results; compares the two paths)           */
+    SDM_OPT_SELECT_CTAS_PER_SM = 3, /* n > 0: at most n selection CTAs per SM           */
+    SDM_OPT_SLOT_CTAS_PER_SM = 4,   /* n > 0: at most n slot-engine scan CTAs per SM     */
+    SDM_OPT_SEQ_COLUMNS = 5,        /* 4, 8, 16 or 32: the sequential engine's column
+                                       slice (0: chosen by shape)                       */
+    SDM_OPT_SEQ_DEPTH = 6           /* 4 or 8: the sequential engine's gather-ahead
+                                       depth in tokens (0: chosen by slice)             */
+} sdm_option;
+
+/* Sets an option.  SDM_ERR_INVALID_ARG (and no change) for an unknown option or a value
+ * outside the ranges above. */
+sdm_status sdm_set_option(int32_t option, int32_t value);
+
+/* The option's current value, or -1 for an unknown option. */
+int32_t sdm_get_option(int32_t option);
 
 /* Number of kernels this library has launched in this process, on every device. */
 uint64_t sdm_launch_count(void);

@@ -9,6 +9,7 @@ behind the ABI.  There is no fallback: if the library is missing the calls raise
 from ._binding import (  # noqa: F401
     ACT,
     ENGINE,
+    OPTION,
     SDM_BF16,
     SDM_F32,
     SdmError,
@@ -18,6 +19,7 @@ from ._binding import (  # noqa: F401
     sdm_decode_step,
     sdm_decode_step_chained,
     sdm_get_device_status,
+    sdm_get_option,
     sdm_launch_count,
     sdm_norm_gate,
     sdm_profile_enable,
@@ -25,6 +27,7 @@ from ._binding import (  # noqa: F401
     sdm_scan_forward,
     sdm_scan_forward_noalloc,
     sdm_select,
+    sdm_set_option,
     sdm_state_init,
     sdm_status_string,
     sdm_workspace_size,

@@ -61,6 +61,8 @@ def library():
         "sdm_profile_enable": ([I], I),
         "sdm_profile_read": ([P, P], I),
         "sdm_launch_count": ([], ctypes.c_uint64),
+        "sdm_set_option": ([I, I], I),
+        "sdm_get_option": ([I], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -298,6 +300,19 @@ def sdm_profile_read() -> dict:
     _check(library().sdm_profile_read(ctypes.cast(ms, ctypes.c_void_p),
                                       ctypes.cast(n, ctypes.c_void_p)), "sdm_profile_read")
     return {k: (ms[i], n[i]) for i, k in enumerate(KERNEL_KINDS)}
+
+
+OPTION = {"no_pdl": 1, "select_general": 2, "select_ctas_per_sm": 3, "slot_ctas_per_sm": 4,
+          "seq_columns": 5, "seq_depth": 6}
+
+
+def sdm_set_option(option: str, value: int):
+    """Sets a process-wide launch option of include/sdm.h (sdm_option), by name."""
+    _check(library().sdm_set_option(OPTION[option], int(value)), f"sdm_set_option({option})")
+
+
+def sdm_get_option(option: str) -> int:
+    return int(library().sdm_get_option(OPTION[option]))
 
 
 def sdm_launch_count() -> int:

@@ -7,7 +7,9 @@
 //   step 1 (bf16 halves of up to 1024 scores, K <= 128): two warps per score half (write
 //   and read selection, first and second half) find the half's top K with the group
 //   selection of select_group.cuh; four warps per selection then take the top K of the
-//   rank-pair candidate sums the same way and write slot indices and softmax weights.
+//   rank-pair candidate sums the same way and write slot indices and softmax weights (when
+//   the halves' exponents span more than 15, the first of the four checks the ties at the
+//   K-th sum against all K*K pairs, as select.cuh describes).
 //   Other shapes: warps 0 and 1 run the warp-per-row selection of select.cuh.
 //   CTAs 0 .. 63 also prefetch into L2 the inputs of the CTAs dispatched after them;
 //   steps 2 and 3 issue every row load of the token at once: each warp's write rows go to
@@ -236,9 +238,29 @@ __device__ __forceinline__ void decode_select_group(const DecodeArgs& a, const D
           out_idx[r] = static_cast<int32_t>(flat);
           ev[r] = expf(key_score(static_cast<uint32_t>(c >> 32)) - s0);
           atomicOr(&bits[(flat >> 5) & 63u], 1u << (flat & 31u));
+          if (r == K - 1) cctl->kth = static_cast<uint32_t>(c >> 32);
         }
       });
   group_bar(5 + s, 128);
+  if (st < 32 && !warp_bf16_sums_exact(
+                     [&](int j) { return key16_value((j < K ? A[j] : B[j - K]) >> 16); }, K, st)) {
+    // fp32 rounding may have merged unequal sums: the ties at the K-th sum are checked
+    // against all K*K pairs (a refilled slot keeps the K-th key, so its weight is unchanged;
+    // a replaced slot's filter bit stays set, which the exact membership checks allow)
+    const uint32_t Tk = cctl->kth;
+    repair_ties_at_kth(
+        [&](int r1, int r2) {
+          return score_key(__fadd_rn(key16_value(A[r1] >> 16), key16_value(B[r2] >> 16)));
+        },
+        [&](int r1, int r2) {
+          return (0xffffu - (A[r1] & 0xffffu)) * static_cast<uint32_t>(a.S2) +
+                 (0xffffu - (B[r2] & 0xffffu));
+        },
+        K, Tk, st, [&](int r, uint32_t f) {
+          out_idx[r] = static_cast<int32_t>(f);
+          atomicOr(&bits[(f >> 5) & 63u], 1u << (f & 31u));
+        });
+  }
   if (st < K) {
     // the softmax denominator, the same sum in the same order on every thread (ev is zero
     // past K up to the next multiple of 4)

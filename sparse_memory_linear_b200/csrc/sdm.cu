@@ -36,14 +36,15 @@ constexpr size_t WS_ALIGN = 256;
     }                                            \
   } while (0)
 
-// SDM_NO_PDL=1 launches every kernel in plain stream order, sdm_decode_step_chained included.
-inline bool pdl_enabled() {
-  static const bool on = [] {
-    const char* e = getenv("SDM_NO_PDL");
-    return !(e && e[0] == '1');
-  }();
-  return on;
-}
+// Process-wide launch options (sdm_option); 0 everywhere by default.
+constexpr int OPT_SLOTS = 8;
+std::atomic<int> g_opt[OPT_SLOTS];
+
+inline int opt(int which) { return g_opt[which].load(std::memory_order_relaxed); }
+
+// SDM_OPT_NO_PDL = 1 launches every kernel in plain stream order, sdm_decode_step_chained
+// included.
+inline bool pdl_enabled() { return opt(SDM_OPT_NO_PDL) == 0; }
 
 // Launches `kernel` in stream order, or with PDL = true with programmatic stream
 // serialisation: scheduled while the kernel ahead of it finishes.  Every kernel of this
@@ -260,20 +261,10 @@ bool slot_engine_fits(const sdm_shape& s) {
 // slice) units to fill the GPU; below that the slot engine, whose parallelism is the
 // number of distinct slots touched, does better.
 int pick_engine(const sdm_shape& s, int requested, int sms) {
-  const char* env = getenv("SDM_ENGINE");
-  if (requested == SDM_ENGINE_AUTO && env) {
-    if (!strcmp(env, "seq")) requested = SDM_ENGINE_SEQ;
-    if (!strcmp(env, "slot")) requested = SDM_ENGINE_SLOT;
-  }
   if (requested != SDM_ENGINE_AUTO) return requested;
   if (!slot_engine_fits(s)) return SDM_ENGINE_SEQ;
   const long long units = (long long)s.B * s.H * (s.d_v / 32 > 0 ? s.d_v / 32 : 1);
   return (units < 2LL * sms && s.d_v >= 128) ? SDM_ENGINE_SLOT : SDM_ENGINE_SEQ;
-}
-
-int env_int(const char* name, int dflt) {
-  const char* v = getenv(name);
-  return v ? atoi(v) : dflt;
 }
 
 template <int R8, int KC>
@@ -288,7 +279,7 @@ sdm_status launch_select_fast_t(const SelJob& j0, const SelJob* j1, long long ro
                                                              warps * 32, smem));
   if (per_sm < 1) return SDM_ERR_UNSUPPORTED;
   const long long total_rows = rows * (j1 ? 2 : 1);
-  const int cap = env_int("SDM_SEL_CTAS", 0);
+  const int cap = opt(SDM_OPT_SELECT_CTAS_PER_SM);
   if (cap > 0 && cap < per_sm) per_sm = cap;
   long long grid = (long long)di->sms * per_sm;
   const long long need = (total_rows + warps - 1) / warps;
@@ -323,7 +314,7 @@ sdm_status launch_select(const SelJob& j0, const SelJob* j1, long long rows, int
   if (rows == 0) return SDM_OK;
   const int K1 = j1 ? j1->K : j0.K;
   const int kmax_all = j0.K > K1 ? j0.K : K1;
-  if (fast_select_ok(bf16, S1, S2, kmax_all) && env_int("SDM_SELECT_SLOW", 0) == 0)
+  if (fast_select_ok(bf16, S1, S2, kmax_all) && opt(SDM_OPT_SELECT_GENERAL) == 0)
     return launch_select_fast(j0, j1, rows, S1, S2, di, st);
   int warps = 8;
   size_t smem = sel_smem_bytes(S1, S2, j0.K, K1, warps);
@@ -336,7 +327,7 @@ sdm_status launch_select(const SelJob& j0, const SelJob* j1, long long rows, int
   SDM_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sel_kernel, warps * 32, smem));
   if (per_sm < 1) return SDM_ERR_UNSUPPORTED;
   const long long total_rows = rows * (j1 ? 2 : 1);
-  const int cap = env_int("SDM_SEL_CTAS", 0);
+  const int cap = opt(SDM_OPT_SELECT_CTAS_PER_SM);
   if (cap > 0 && cap < per_sm) per_sm = cap;
   long long grid = (long long)di->sms * per_sm;
   const long long need = (total_rows + warps - 1) / warps;
@@ -369,7 +360,7 @@ sdm_status launch_seq(const SeqArgs& a, cudaStream_t st) {
   const int bh = a.B * a.H;
   const int cws[4] = {32, 16, 8, 4};
   int CW = 0;
-  const int force_cw = env_int("SDM_SEQ_CW", 0);
+  const int force_cw = opt(SDM_OPT_SEQ_COLUMNS);
   for (int i = 0; i < 4; ++i) {
     const int c = cws[i];
     if (a.d_v % c != 0 || c * v_esz < 16) continue;
@@ -381,8 +372,8 @@ sdm_status launch_seq(const SeqArgs& a, cudaStream_t st) {
     if ((long long)bh * (a.d_v / c) * 5 >= (long long)di->sms * 4) break;
   }
   if (CW == 0) return SDM_ERR_UNSUPPORTED;
-  int D = env_int("SDM_SEQ_D", CW >= 32 ? 4 : 8);
-  if (D != 4 && D != 8) D = 4;
+  int D = opt(SDM_OPT_SEQ_DEPTH);
+  if (D != 4 && D != 8) D = CW >= 32 ? 4 : 8;
   SeqLayout L = seq_layout(a.ldw, a.ldr, CW, v_esz, D);
   if (L.total > (size_t)di->max_smem_optin && D == 8) {
     D = 4;
@@ -439,7 +430,7 @@ sdm_status launch_slot_chunk(const SlotArgs& a, const DeviceInfo* di, cudaStream
   SDM_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
       &per_sm, slot_chunk_kernel<NQ, G, PF>, SLOT_THREADS, smem));
   int ctas = per_sm > 0 ? per_sm : 1;
-  const int cap = env_int("SDM_SLOT_CTAS", 0);
+  const int cap = opt(SDM_OPT_SLOT_CTAS_PER_SM);
   if (cap > 0 && cap < ctas) ctas = cap;
   const int grid = di->sms * ctas;
   SDM_CUDA_TRY(launch_pdl(slot_chunk_kernel<NQ, G, PF>, dim3(grid), dim3(SLOT_THREADS), smem, st,
@@ -848,6 +839,27 @@ sdm_status sdm_get_device_status(void* stream) {
 }
 
 uint64_t sdm_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+sdm_status sdm_set_option(int32_t option, int32_t value) {
+  bool ok = false;
+  switch (option) {
+    case SDM_OPT_NO_PDL:
+    case SDM_OPT_SELECT_GENERAL: ok = value == 0 || value == 1; break;
+    case SDM_OPT_SELECT_CTAS_PER_SM:
+    case SDM_OPT_SLOT_CTAS_PER_SM: ok = value >= 0 && value <= 64; break;
+    case SDM_OPT_SEQ_COLUMNS: ok = value == 0 || value == 4 || value == 8 || value == 16 || value == 32; break;
+    case SDM_OPT_SEQ_DEPTH: ok = value == 0 || value == 4 || value == 8; break;
+    default: ok = false;
+  }
+  if (!ok) return SDM_ERR_INVALID_ARG;
+  g_opt[option].store(value, std::memory_order_relaxed);
+  return SDM_OK;
+}
+
+int32_t sdm_get_option(int32_t option) {
+  if (option < SDM_OPT_NO_PDL || option > SDM_OPT_SEQ_DEPTH) return -1;
+  return opt(option);
+}
 
 sdm_status sdm_profile_enable(int32_t on) {
   std::vector<ProfRec> drop;

@@ -12,12 +12,15 @@
 //   2. per half, a most-significant-digit radix select (8-bit digits, 256-bin histogram)
 //      finds the bin of the K-th key; keys above it and the lowest-index keys inside it
 //      form the half's top-K, then a bitonic sort gives their ranks;
-//   3. candidates are the rank pairs (r1, r2) with (r1+1)(r2+1) <= K: any other pair is
-//      preceded by at least K pairs with a larger-or-equal sum and a smaller slot index,
-//      so it cannot be among the top-K (exact whenever the fp32 sums are exact, which
-//      holds for bf16 halves of comparable magnitude);
+//   3. candidates are the rank pairs (r1, r2) with (r1+1)(r2+1) <= K: every other pair is
+//      preceded by at least K pairs with a larger-or-equal sum, so the pruned set holds all
+//      pairs above the K-th largest sum T and T itself;
 //   4. radix select over the candidate sums; ties at the threshold take the lowest flat
-//      slot indices; bitonic sort of the K winners; softmax weights.
+//      slot indices; bitonic sort of the K winners;
+//   5. ties at T beyond the pruning (repair_ties_at_kth): when fp32 rounding can merge
+//      unequal sums, a pair the pruning dropped may sum to T with a lower slot index than a
+//      tie it kept; if one does, the ties at T are refilled from all K*K pairs;
+//   6. softmax weights.
 #pragma once
 
 #include "common.cuh"
@@ -210,6 +213,103 @@ __device__ __forceinline__ uint64_t composite(uint32_t key, int32_t idx) {
   return (static_cast<uint64_t>(key) << 32) | static_cast<uint64_t>(0xffffffffu - static_cast<uint32_t>(idx));
 }
 
+// ------------------------------------------------------------------------------------
+// Ties at the K-th candidate sum beyond the rank-pair pruning.
+//
+// Let T be the K-th largest of the K*K candidate sums.  The pruned set P (rank pairs with
+// (r1+1)(r2+1) <= K) holds every pair whose sum is above T (such a pair has fewer than K
+// pairs at or above it, so its rank rectangle is smaller than K + 1) and at least K pairs at
+// or above T, so T and the pairs above it are found exactly from P.  Only the ties at T can
+// differ: with exact sums, a tie outside P has at least K pairs of its rank rectangle ahead
+// of it (equal sums there mean equal half scores, hence lower indices), but when fp32
+// rounding merges unequal sums, a dropped pair can sum to T with a lower slot index than a
+// tie P kept.  Sums fall weakly along a rank row and no dropped pair is above T, so such a
+// pair exists only if the first pair P drops in some rank row r1 >= 1, (r1, K/(r1+1)),
+// sums to T.  The result is then repaired: ranks from the first tie on are refilled with
+// the lowest slot indices among all K*K pairs whose sum is T.
+
+// Whether every fp32 sum of two of the bf16 values val(0 .. 2K) is exact: the nonzero values'
+// exponent fields (a subnormal's counted as 1) span at most 15 and stay below 254, so a sum
+// needs at most 24 significant bits and cannot overflow.  Warp-wide.
+template <typename Val>
+__device__ __forceinline__ bool warp_bf16_sums_exact(Val val, int K, int lane) {
+  uint32_t emin = 255u, emax = 0u;
+  for (int j = lane; j < 2 * K; j += 32) {
+    const uint32_t u = __float_as_uint(val(j)) & 0x7fffffffu;
+    if (u != 0u) {
+      const uint32_t e = max(u >> 23, 1u);
+      emin = min(emin, e);
+      emax = max(emax, e);
+    }
+  }
+  emin = __reduce_min_sync(FULL_MASK, emin);
+  emax = __reduce_max_sync(FULL_MASK, emax);
+  return emax == 0u || (emax - emin <= 15u && emax < 254u);
+}
+
+// Warp-wide repair of a selection whose K-th key is Tk.  sum_key(r1, r2) is the order key of
+// the fp32 sum of ranks r1, r2 (weakly decreasing in each), flat(r1, r2) the pair's slot
+// index.  If some rank row's first dropped pair sums to Tk, emit(r, flat) is called for the
+// ranks r = ngt .. K-1 (ngt: the pairs above Tk) with the lowest slot indices, ascending,
+// among all pairs whose key is Tk, and true is returned; otherwise nothing is emitted.
+// Emission happens on lane 0.
+template <typename SumKey, typename Flat, typename Emit>
+__device__ inline bool repair_ties_at_kth(SumKey sum_key, Flat flat, int K, uint32_t Tk,
+                                          int lane, Emit emit) {
+  bool hit = false;
+  for (int r1 = 1 + lane; r1 < K; r1 += 32)
+    if (sum_key(r1, K / (r1 + 1)) == Tk) hit = true;
+  if (!__any_sync(FULL_MASK, hit)) return false;
+  // per rank row, the columns [cs, ce) whose key is Tk, by binary search
+  constexpr int RPL = KMAX / 32;
+  int cs[RPL], ce[RPL];
+  int ngt = 0;
+#pragma unroll
+  for (int q = 0; q < RPL; ++q) {
+    const int r1 = lane + 32 * q;
+    cs[q] = 0;
+    ce[q] = 0;
+    if (r1 < K) {
+      int lo = 0, hi = K;
+      while (lo < hi) {
+        const int m = (lo + hi) >> 1;
+        if (sum_key(r1, m) > Tk) lo = m + 1;
+        else hi = m;
+      }
+      cs[q] = lo;
+      hi = K;
+      while (lo < hi) {
+        const int m = (lo + hi) >> 1;
+        if (sum_key(r1, m) >= Tk) lo = m + 1;
+        else hi = m;
+      }
+      ce[q] = lo;
+      ngt += cs[q];
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ngt += __shfl_xor_sync(FULL_MASK, ngt, o);
+  // the lowest slot indices among the ties, one per round (slot indices are below 2^24)
+  int floor_f = -1;
+  for (int r = ngt; r < K; ++r) {
+    uint32_t best = 0xffffffffu;
+#pragma unroll
+    for (int q = 0; q < RPL; ++q) {
+      const int r1 = lane + 32 * q;
+      for (int c = cs[q]; c < ce[q]; ++c) {
+        const uint32_t f = flat(r1, c);
+        if (static_cast<int>(f) > floor_f && f < best) best = f;
+      }
+    }
+    best = __reduce_min_sync(FULL_MASK, best);
+    if (best == 0xffffffffu) break;  // unreachable: P's own ties are among the pairs
+    if (lane == 0) emit(r, best);
+    floor_f = static_cast<int>(best);
+  }
+  __syncwarp();
+  return true;
+}
+
 // Top-K of one half (keys[0..n), index = position), written sorted to out_key/out_idx.
 __device__ inline void half_topk(const uint32_t* keys, int n, int K, int min_shift,
                                  SelScratch& sc, int lane, uint32_t* out_key,
@@ -321,6 +421,19 @@ __device__ inline void select_row(const void* row, bool bf16, int S1, int S2, in
   for (int j = K + lane; j < P; j += 32) sc.sortbuf[j] = 0ull;
   __syncwarp();
   warp_bitonic_desc(sc.sortbuf, P, lane);
+
+  // ties at the K-th sum beyond the pruning (exact bf16 sums cannot merge)
+  if (!bf16 || !warp_bf16_sums_exact(
+                   [&](int j) { return key_score(j < K ? sc.a_key[j] : sc.b_key[j - K]); }, K,
+                   lane)) {
+    const uint32_t Tk = static_cast<uint32_t>(sc.sortbuf[K - 1] >> 32);
+    repair_ties_at_kth(
+        [&](int r1, int r2) {
+          return score_key(__fadd_rn(key_score(sc.a_key[r1]), key_score(sc.b_key[r2])));
+        },
+        [&](int r1, int r2) { return static_cast<uint32_t>(sc.a_idx[r1] * S2 + sc.b_idx[r2]); },
+        K, Tk, lane, [&](int r, uint32_t f) { sc.sortbuf[r] = composite(Tk, static_cast<int32_t>(f)); });
+  }
 
   // softmax over the selected scores
   const float s0 = key_score(static_cast<uint32_t>(sc.sortbuf[0] >> 32));

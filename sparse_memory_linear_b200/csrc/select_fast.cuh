@@ -14,7 +14,9 @@
 //   4. a register bitonic sort (shuffles) orders them: (key desc, index asc).
 // Candidates: the rank pairs with (r1+1)(r2+1) <= K; their K-th largest sum is at least
 // both A[K-1] + B[0] and A[0] + B[K-1] (K candidate sums reach each), which brackets the same
-// histogram search; equal sums at the threshold take the lowest flat slot indices.
+// histogram search; equal sums at the threshold take the lowest flat slot indices.  When the
+// halves' exponents span more than 15, fp32 sums can round together and the ties at the K-th
+// sum are checked against all K*K pairs (repair_ties_at_kth, select.cuh).
 #pragma once
 
 #include "select.cuh"
@@ -400,6 +402,29 @@ __device__ __forceinline__ void cand_topk_bf16(const uint32_t* A, const uint32_t
     v[q] = p < K ? stage[p] : 0ull;
   }
   bitonic_desc_reg<uint64_t, NPL>(v, lane);
+  // ties at the K-th sum beyond the pruning: only when rounding can merge unequal sums
+  if (!warp_bf16_sums_exact([&](int j) { return j < K ? av[j] : bv[j - K]; }, K, lane)) {
+    uint64_t vk = 0ull;
+#pragma unroll
+    for (int q = 0; q < NPL; ++q)
+      if (q == ((K - 1) >> 5)) vk = v[q];
+    const uint32_t Tk = static_cast<uint32_t>(__shfl_sync(FULL_MASK, vk, (K - 1) & 31) >> 32);
+#pragma unroll
+    for (int q = 0; q < NPL; ++q)
+      if (q * 32 + lane < K) stage[q * 32 + lane] = v[q];
+    __syncwarp();
+    const bool fixed = repair_ties_at_kth(
+        [&](int r1, int r2) { return score_key(__fadd_rn(av[r1], bv[r2])); },
+        [&](int r1, int r2) { return static_cast<uint32_t>(ai[r1] + bi[r2]); }, K, Tk, lane,
+        [&](int r, uint32_t f) {
+          stage[r] = (static_cast<uint64_t>(Tk) << 32) | (0xffffffffu - f);
+        });
+    if (fixed) {
+#pragma unroll
+      for (int q = 0; q < NPL; ++q) v[q] = q * 32 + lane < K ? stage[q * 32 + lane] : 0ull;
+    }
+    __syncwarp();
+  }
   const float s0 = key_score(static_cast<uint32_t>(__shfl_sync(FULL_MASK, v[0], 0) >> 32));
   float e[NPL];
   float part = 0.0f;

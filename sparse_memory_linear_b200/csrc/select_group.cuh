@@ -44,6 +44,7 @@ struct GroupCtl {
   uint32_t wmin[4];  // per-warp bracket key
   uint32_t bin, run, cnt_bin;
   uint32_t count;    // list append counter, zero before the group starts
+  uint32_t kth;      // key of the K-th ranked composite (set by the caller's emit)
 };
 
 // Group-wide bracket [lo, hi]: hi is the largest key, lo the smallest of the warps' bracket

@@ -1,11 +1,20 @@
 """The C ABI without a GPU: the library loads, exports every entry point the header
-declares, sizes its scratch, and rejects bad arguments on the host before any launch."""
+declares, sizes its scratch, and rejects bad arguments on the host before any launch.
+
+The rejection tests pass made-up device addresses, which validation turns down before any
+launch; every one also checks that the library's launch counter did not move.  They run
+only where no CUDA device is visible, so that a regression in validation could never put a
+kernel on such an address.  The host code they exercise is the same on a GPU machine."""
 
 import ctypes
 import os
 import re
 
 import pytest
+import torch
+
+host_only = pytest.mark.skipif(torch.cuda.is_available(),
+                               reason="made-up device addresses are passed only without a GPU")
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -88,7 +97,25 @@ def test_workspace_size(sdm):
 FAKE = 0x10000  # aligned, never dereferenced: validation rejects the call first
 
 
+class no_launch:
+    """Asserts that the library launched no kernel inside the block."""
+
+    def __init__(self, sdm):
+        self.sdm = sdm
+
+    def __enter__(self):
+        self.n = self.sdm.sdm_launch_count()
+
+    def __exit__(self, *exc):
+        assert self.sdm.sdm_launch_count() == self.n, "a rejected call launched a kernel"
+
+
 def scan(sdm, shape, **over):
+    with no_launch(sdm):
+        return _scan(sdm, shape, **over)
+
+
+def _scan(sdm, shape, **over):
     args = dict(kp=FAKE, qp=FAKE, v=FAKE, alpha=FAKE, beta=FAKE, M0=FAKE + 0x100000000,
                 M=FAKE, init=0, y=FAKE, gate=None, gamma=None, eps=1e-6, act=0, o=None,
                 sel=None, engine=0, ws=FAKE, ws_bytes=1 << 40)
@@ -101,6 +128,7 @@ def scan(sdm, shape, **over):
         args["engine"], P(args["ws"]), args["ws_bytes"], shape, None)
 
 
+@host_only
 @pytest.mark.parametrize("bad", [
     dict(kp=None), dict(qp=None), dict(v=None), dict(alpha=None), dict(beta=None),
     dict(M=None), dict(y=None), dict(ws=None), dict(M0=None),
@@ -112,6 +140,7 @@ def test_scan_rejects_bad_arguments(sdm, bad):
     assert scan(sdm, good_shape(sdm), **bad) == 1
 
 
+@host_only
 @pytest.mark.parametrize("kw", [
     dict(W=0), dict(R=0), dict(W=33), dict(R=40), dict(S1=0), dict(S2=5000), dict(B=0),
     dict(H=0), dict(T=-1), dict(d_v=12), dict(d_v=0), dict(d_v=2048), dict(in_dtype=5),
@@ -121,7 +150,13 @@ def test_scan_rejects_bad_shapes(sdm, kw):
     assert scan(sdm, good_shape(sdm, **kw)) == 1
 
 
+@host_only
 def test_decode_and_select_and_norm_reject_bad_arguments(sdm):
+    with no_launch(sdm):
+        _decode_select_norm_reject(sdm)
+
+
+def _decode_select_norm_reject(sdm):
     lib = sdm.library()
     P = ctypes.c_void_p
     s = good_shape(sdm)
@@ -140,6 +175,49 @@ def test_decode_and_select_and_norm_reject_bad_arguments(sdm):
     assert lib.sdm_norm_gate(None, None, None, 1e-6, 0, s, P(FAKE), None) == 1
     # state init: overlapping M and M0
     assert lib.sdm_state_init(P(FAKE), P(FAKE), s, None) == 1
+
+
+@host_only
+def test_noalloc_rejects_shapes_beyond_its_scratch(sdm):
+    """4 x 8192 x 8 rows with W = R = 64 need 128 MiB of scratch, beyond the fixed 16 MiB
+    of sdm_scan_forward_noalloc: SDM_ERR_INVALID_ARG before any CUDA call or launch."""
+    lib = sdm.library()
+    big = sdm.shape_of(4, 8192, 8, 512, 512, 64, 64, 128, sdm.SDM_BF16)
+    assert sdm.sdm_workspace_size(big, "seq") > (16 << 20)
+    ok = sdm.shape_of(1, 1024, 8, 512, 512, 64, 64, 128, sdm.SDM_BF16)
+    assert sdm.sdm_workspace_size(ok, "seq") <= (16 << 20)
+    P = ctypes.c_void_p
+    with no_launch(sdm):
+        rc = lib.sdm_scan_forward_noalloc(P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE),
+                                          P(FAKE + 0x100000000), P(FAKE), 0, P(FAKE), None,
+                                          None, 1e-6, 0, None, None, big, None)
+    assert rc == 1
+
+
+def test_options_are_explicit_and_validated(sdm):
+    """Launch options come only from sdm_set_option: unknown options and values out of
+    range are refused and change nothing; every option reads back and resets to 0."""
+    lib = sdm.library()
+    for name, code in sdm.OPTION.items():
+        assert sdm.sdm_get_option(name) == 0
+    good = {"no_pdl": 1, "select_general": 1, "select_ctas_per_sm": 3, "slot_ctas_per_sm": 2,
+            "seq_columns": 16, "seq_depth": 8}
+    bad = {"no_pdl": 2, "select_general": -1, "select_ctas_per_sm": 65,
+           "slot_ctas_per_sm": -2, "seq_columns": 12, "seq_depth": 5}
+    try:
+        for name in sdm.OPTION:
+            assert lib.sdm_set_option(sdm.OPTION[name], bad[name]) == 1
+            assert sdm.sdm_get_option(name) == 0
+            sdm.sdm_set_option(name, good[name])
+            assert sdm.sdm_get_option(name) == good[name]
+    finally:
+        for name in sdm.OPTION:
+            sdm.sdm_set_option(name, 0)
+    assert lib.sdm_set_option(0, 0) == 1 and lib.sdm_set_option(99, 0) == 1
+    assert lib.sdm_get_option(0) == -1 and lib.sdm_get_option(99) == -1
+    csrc = os.path.join(ROOT, "sparse_memory_linear_b200", "csrc")
+    for f in os.listdir(csrc):
+        assert "getenv" not in open(os.path.join(csrc, f)).read(), f"{f} reads the environment"
 
 
 def test_status_strings(sdm):
@@ -183,6 +261,7 @@ int main(void) {
 """
 
 
+@host_only
 def test_plain_c_program_builds_links_and_calls_the_abi(sdm, tmp_path):
     """The boundary is usable from C alone: a C99 program including sdm.h links against
     libsdm.so and calls it (host-side calls only), and the header also parses as C++."""

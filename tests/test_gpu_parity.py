@@ -57,13 +57,16 @@ def test_select_matches_oracle(sdm, S1, S2, K, dt):
 
 @pytest.mark.parametrize("S1,S2,K", [(1024, 1024, 64), (512, 512, 64), (256, 200, 33),
                                      (1000, 24, 17), (8, 8, 8), (128, 130, 128)])
-def test_select_fast_path_equals_general_path(sdm, S1, S2, K, monkeypatch):
+def test_select_fast_path_equals_general_path(sdm, S1, S2, K):
     """bf16 rows take the register-resident path; forcing the general path must give the
     same slots bit for bit and the same weights."""
     x = sdm_synth.draw(5 + S1 + K, 1, (300, S1 + S2), BF16).to(DEV)
     idx_f, wt_f = sdm.sdm_select(x, K, S1=S1)
-    monkeypatch.setenv("SDM_SELECT_SLOW", "1")
-    idx_g, wt_g = sdm.sdm_select(x, K, S1=S1)
+    sdm.sdm_set_option("select_general", 1)
+    try:
+        idx_g, wt_g = sdm.sdm_select(x, K, S1=S1)
+    finally:
+        sdm.sdm_set_option("select_general", 0)
     torch.cuda.synchronize()
     assert torch.equal(idx_f, idx_g)
     assert_close(wt_f.cpu().numpy(), wt_g.cpu().numpy(), "weights", atol=1e-7, rtol=1e-6)

@@ -4,8 +4,9 @@ sdm_scan_forward_noalloc serves callers that cannot allocate device memory while
 runs (an engine that owns all device memory in its own pool, a plugin interface without a
 workspace argument, a loop that must not call the CUDA allocator once running): it takes
 its scratch from a fixed device array inside the library.  Its results must equal those of
-sdm_scan_forward with a caller workspace, call after call, even though every call reuses
-the same array.
+sdm_scan_forward with a caller workspace and those of the CPU oracle, call after call, even
+though every call reuses the same array; and once the first call on the device has looked
+up the array's address, a call must not change the memory the process holds on the device.
 """
 
 import ctypes
@@ -14,8 +15,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import sdm_synth
-from tests._parity import TOL_ABS, TOL_REL, assert_close
+from tests._parity import THREADS, TOL_ABS, TOL_REL, assert_close, host
 
 pytestmark = pytest.mark.gpu
 
@@ -81,13 +83,59 @@ def test_noalloc_equals_workspace_entry_point_twice(lib):
                      atol=TOL_ABS, rtol=TOL_REL)
 
 
-def test_noalloc_rejects_shapes_beyond_its_scratch(lib):
-    sdm, L = lib
-    # 4 x 8192 x 8 rows with W = R = 64 need 128 MiB of scratch, beyond the fixed 16 MiB
-    big = sdm.shape_of(4, 8192, 8, 512, 512, 64, 64, 128, sdm.SDM_BF16)
-    assert sdm.sdm_workspace_size(big, "seq") > (16 << 20)
-    fake = ctypes.c_void_p(0x10000)
-    rc = L.sdm_scan_forward_noalloc(fake, fake, fake, fake, fake, ctypes.c_void_p(0x2000000000),
-                                    fake, 0, fake, None, None, 1e-6, 0, None, None, big, None)
-    assert rc == 1  # SDM_ERR_INVALID_ARG, nothing launched
-    np.testing.assert_equal(sdm.sdm_get_device_status(), 0)
+def _noalloc(sdm, g, wl, M, y, o, sel):
+    sdm.sdm_scan_forward_noalloc(g["kp"], g["qp"], g["v"], g["alpha"], g["beta"], M, W=wl.W,
+                                 R=wl.R, M0=g["M0"], y=y, gate=g["gate"], gamma=g["gamma"],
+                                 o=o, sel_out=sel)
+
+
+def test_noalloc_matches_the_oracle_on_consecutive_calls(lib):
+    """Two calls in a row (the second over the first one's scratch) against the oracle."""
+    sdm, _ = lib
+    wl = sdm_synth.WORKLOADS["small"].replace(T=192, seed=78)
+    cpu = sdm_synth.make_inputs(wl, with_gamma=True)
+    g = {k: t.to(DEV) for k, t in cpu.items()}
+    ref = oracle.forward(host(cpu["kp"]), host(cpu["qp"]), host(cpu["v"]), host(cpu["alpha"]),
+                         host(cpu["beta"]), host(cpu["M0"]), S1=wl.S1, W=wl.W, R=wl.R,
+                         gate=host(cpu["gate"]), gamma=host(cpu["gamma"]), threads=THREADS)
+    n = wl.B * wl.T * wl.H
+    for call in range(2):
+        M = torch.full((wl.B, wl.H, wl.N, wl.d_v), float("nan"), device=DEV)
+        y = torch.full((wl.B, wl.T, wl.H, wl.d_v), float("nan"), device=DEV)
+        o = torch.full_like(y, float("nan"))
+        sel = torch.full((n * (wl.W + wl.R),), -1, dtype=torch.int32, device=DEV)
+        _noalloc(sdm, g, wl, M, y, o, sel)
+        torch.cuda.synchronize()
+        assert sdm.sdm_get_device_status() == 0
+        s = sel.cpu().numpy()
+        np.testing.assert_array_equal(s[: n * wl.W].reshape(ref["idx_w"].shape), ref["idx_w"])
+        np.testing.assert_array_equal(s[n * wl.W:].reshape(ref["idx_r"].shape), ref["idx_r"])
+        assert_close(host(y), ref["y"], f"call {call}: y")
+        assert_close(host(o), ref["o"], f"call {call}: o")
+        assert_close(host(M), ref["M"], f"call {call}: M")
+
+
+def test_noalloc_calls_hold_no_new_device_memory(lib):
+    """After the first call on the device (which looks up the array's address), further
+    calls leave torch's allocation count and the device's free memory where they were.
+    (The free-memory check assumes no other process allocates on this GPU meanwhile.)"""
+    sdm, _ = lib
+    wl = sdm_synth.WORKLOADS["small"].replace(T=512, seed=79)
+    g = {k: t.to(DEV) for k, t in sdm_synth.make_inputs(wl, with_gamma=True).items()}
+    M = torch.empty((wl.B, wl.H, wl.N, wl.d_v), device=DEV)
+    y = torch.empty((wl.B, wl.T, wl.H, wl.d_v), device=DEV)
+    o = torch.empty_like(y)
+    sel = torch.empty((wl.B * wl.T * wl.H * (wl.W + wl.R),), dtype=torch.int32, device=DEV)
+    _noalloc(sdm, g, wl, M, y, o, sel)
+    torch.cuda.synchronize()
+    held = torch.cuda.memory_allocated()
+    free0, _ = torch.cuda.mem_get_info()
+    launches = sdm.sdm_launch_count()
+    for _ in range(3):
+        _noalloc(sdm, g, wl, M, y, o, sel)
+    torch.cuda.synchronize()
+    assert sdm.sdm_launch_count() > launches  # the calls did run
+    assert torch.cuda.memory_allocated() == held
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 >= free0 - (1 << 20), (free0, free1)
+    assert sdm.sdm_get_device_status() == 0

@@ -111,6 +111,18 @@ def _need(t, name, dtype=None, device=None):
     return t
 
 
+def _expect(t, name, shape=None, numel=None):
+    """Raises ValueError unless tensor t (None passes) has this shape or element count.
+    The C ABI receives bare pointers and cannot see buffer sizes, so every tensor is
+    checked against the call's shape here, before any pointer reaches the library."""
+    if t is None:
+        return
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name} has {t.numel()} elements, expected {numel}")
+
+
 def shape_of(B, T, H, S1, S2, W, R, d_v, in_dtype) -> SdmShape:
     return SdmShape(int(B), int(T), int(H), int(S1), int(S2), int(W), int(R), int(d_v),
                     int(in_dtype))
@@ -128,11 +140,13 @@ def sdm_select(halves: torch.Tensor, K: int, *, S1: int | None = None, idx=None,
                stream=None):
     """Top-K product-key selection of every row of ``halves`` [..., S1+S2].
     Returns (idx int32 [..., K], wt float32 [..., K])."""
-    _need(halves, "halves")
     S = halves.shape[-1]
     S1 = S // 2 if S1 is None else int(S1)
     rows = halves.numel() // S if S else 0
     lead = tuple(halves.shape[:-1])
+    _expect(idx, "idx", lead + (K,))
+    _expect(wt, "wt", lead + (K,))
+    _need(halves, "halves")
     idx = torch.empty(lead + (K,), dtype=torch.int32, device=halves.device) if idx is None else idx
     wt = torch.empty(lead + (K,), dtype=torch.float32, device=halves.device) if wt is None else wt
     _need(idx, "idx", torch.int32, halves.device)
@@ -145,9 +159,12 @@ def sdm_select(halves: torch.Tensor, K: int, *, S1: int | None = None, idx=None,
 
 def sdm_state_init(M0: torch.Tensor, M: torch.Tensor, *, d_v: int | None = None, stream=None):
     """M[b, h] = M0[h] for every b.  M0 [H, N, d_v], M [B, H, N, d_v] float32."""
+    if M.dim() != 4:
+        raise ValueError(f"M has shape {tuple(M.shape)}, expected [B, H, N, d_v]")
+    B, H, N, dv = M.shape
+    _expect(M0, "M0", (H, N, dv))
     _need(M0, "M0", torch.float32)
     _need(M, "M", torch.float32, M0.device)
-    B, H, N, dv = M.shape
     shape = shape_of(B, 1, H, 1, N, 1, 1, dv, SDM_F32)
     _check(library().sdm_state_init(_p(M0), _p(M), shape, _stream(stream, M.device)),
            "sdm_state_init")
@@ -159,6 +176,19 @@ def _scan_outputs(kp, qp, v, alpha, beta, M, W, R, S1, M0, y, gate, gamma, o, wa
     """Checks the prefill arguments and allocates the missing outputs; returns
     (shape, y, o, sel_out)."""
     dev = kp.device
+    if kp.dim() != 4:
+        raise ValueError(f"kp has shape {tuple(kp.shape)}, expected [B, T, H, S1 + S2]")
+    B, T, H, S = kp.shape
+    S1 = S // 2 if S1 is None else int(S1)
+    d_v = v.shape[-1]
+    N = S1 * (S - S1)
+    for t, name, shp in ((qp, "qp", (B, T, H, S)), (v, "v", (B, T, H, d_v)),
+                         (gate, "gate", (B, T, H, d_v)), (alpha, "alpha", (B, T, H)),
+                         (beta, "beta", (B, T, H)), (M, "M", (B, H, N, d_v)),
+                         (M0, "M0", (H, N, d_v)), (gamma, "gamma", (d_v,)),
+                         (y, "y", (B, T, H, d_v)), (o, "o", (B, T, H, d_v))):
+        _expect(t, name, shp)
+    _expect(sel_out, "sel_out", numel=B * T * H * (W + R))
     _need(kp, "kp", device=dev)
     dt = kp.dtype
     _need(qp, "qp", dt, dev)
@@ -169,9 +199,6 @@ def _scan_outputs(kp, qp, v, alpha, beta, M, W, R, S1, M0, y, gate, gamma, o, wa
     _need(M, "M", torch.float32, dev)
     _need(M0, "M0", torch.float32, dev)
     _need(gamma, "gamma", torch.float32, dev)
-    B, T, H, S = kp.shape
-    S1 = S // 2 if S1 is None else int(S1)
-    d_v = v.shape[-1]
     shape = shape_of(B, T, H, S1, S - S1, W, R, d_v, _in_dtype(kp))
     if y is None:
         y = torch.empty((B, T, H, d_v), dtype=torch.float32, device=dev)
@@ -235,6 +262,18 @@ def sdm_decode_step(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | None
     sdm_decode_step_chained: only when the kernel launched right before on the stream writes
     none of this step's inputs (a chain of steps over inputs already on the device)."""
     dev = kp.device
+    if kp.dim() != 3:
+        raise ValueError(f"kp has shape {tuple(kp.shape)}, expected [B, H, S1 + S2]")
+    B, H, S = kp.shape
+    S1 = S // 2 if S1 is None else int(S1)
+    d_v = v.shape[-1]
+    N = S1 * (S - S1)
+    for t, name, shp in ((qp, "qp", (B, H, S)), (v, "v", (B, H, d_v)), (gate, "gate", (B, H, d_v)),
+                         (alpha, "alpha", (B, H)), (beta, "beta", (B, H)),
+                         (M, "M", (B, H, N, d_v)), (gamma, "gamma", (d_v,)),
+                         (y, "y", (B, H, d_v)), (o, "o", (B, H, d_v))):
+        _expect(t, name, shp)
+    _expect(sel_out, "sel_out", numel=B * H * (W + R))
     _need(kp, "kp", device=dev)
     dt = kp.dtype
     _need(qp, "qp", dt, dev)
@@ -244,9 +283,6 @@ def sdm_decode_step(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | None
     _need(beta, "beta", torch.float32, dev)
     _need(M, "M", torch.float32, dev)
     _need(gamma, "gamma", torch.float32, dev)
-    B, H, S = kp.shape
-    S1 = S // 2 if S1 is None else int(S1)
-    d_v = v.shape[-1]
     shape = shape_of(B, 1, H, S1, S - S1, W, R, d_v, _in_dtype(kp))
     if y is None:
         y = torch.empty((B, H, d_v), dtype=torch.float32, device=dev)
@@ -270,10 +306,13 @@ def sdm_decode_step_chained(kp, qp, v, alpha, beta, M, **kw):
 def sdm_norm_gate(y, *, gate=None, gamma=None, eps: float = 1e-6, act: str = "silu", o=None,
                   stream=None):
     """o = y * rsqrt(mean(y^2) + eps) * gamma * act(gate) over the last axis of y."""
+    d_v = y.shape[-1]
+    _expect(gate, "gate", tuple(y.shape))
+    _expect(o, "o", tuple(y.shape))
+    _expect(gamma, "gamma", (d_v,))
     _need(y, "y", torch.float32)
     _need(gate, "gate", device=y.device)
     _need(gamma, "gamma", torch.float32, y.device)
-    d_v = y.shape[-1]
     rows = y.numel() // d_v
     o = torch.empty_like(y) if o is None else o
     _need(o, "o", torch.float32, y.device)

@@ -281,3 +281,51 @@ def test_plain_c_program_builds_links_and_calls_the_abi(sdm, tmp_path):
     if shutil.which("g++"):
         subprocess.run(["g++", "-std=c++17", "-fsyntax-only", "-x", "c++", "-I",
                         os.path.join(ROOT, "include"), str(src)], check=True)
+
+
+def test_binding_refuses_tensors_that_do_not_match_the_call(sdm):
+    """The C ABI sees bare pointers, so the binding checks every tensor against the shape
+    of the call before anything reaches the library.  The first case is a decode run's
+    step-major stack [T, B, H, S] passed as a prefill's [B, T, H, S] with a state sized for
+    B sequences: the library would read it as T sequences and run off the end of the state."""
+    f = torch.float32
+    B, T, H, S1, d_v, W = 4, 16, 2, 16, 8, 4
+    N = S1 * S1
+    kp = torch.zeros(T, B, H, 2 * S1)
+    good = dict(qp=kp, v=torch.zeros(T, B, H, d_v), alpha=torch.zeros(T, B, H),
+                beta=torch.zeros(T, B, H))
+    with no_launch(sdm), pytest.raises(ValueError, match=r"M has shape"):
+        sdm.sdm_scan_forward(kp, good["qp"], good["v"], good["alpha"], good["beta"],
+                             torch.zeros(B, H, N, d_v), W=W, R=W)
+    kp = torch.zeros(B, T, H, 2 * S1)
+    args = dict(qp=kp, v=torch.zeros(B, T, H, d_v), alpha=torch.zeros(B, T, H),
+                beta=torch.zeros(B, T, H), M=torch.zeros(B, H, N, d_v))
+    bad = [("qp", torch.zeros(B, T, H, 2 * S1 + 2)), ("v", torch.zeros(B, T, H + 1, d_v)),
+           ("alpha", torch.zeros(B, T)), ("beta", torch.zeros(B, T, H, 1)),
+           ("M", torch.zeros(B, H, N + 1, d_v))]
+    for name, t in bad:
+        a = dict(args)
+        a[name] = t
+        with no_launch(sdm), pytest.raises(ValueError, match=name):
+            sdm.sdm_scan_forward(kp, a["qp"], a["v"], a["alpha"], a["beta"], a["M"], W=W, R=W)
+    for kw in (dict(y=torch.zeros(B, T, H, d_v + 1)), dict(o=torch.zeros(1)),
+               dict(M0=torch.zeros(H + 1, N, d_v)), dict(gate=torch.zeros(B, T, H, 2)),
+               dict(gamma=torch.zeros(d_v + 1)), dict(sel_out=torch.zeros(3, dtype=torch.int32))):
+        with no_launch(sdm), pytest.raises(ValueError, match="shape|elements"):
+            sdm.sdm_scan_forward(kp, args["qp"], args["v"], args["alpha"], args["beta"],
+                                 args["M"], W=W, R=W, **kw)
+    # consistent shapes get as far as the device check (no GPU tensors here)
+    with no_launch(sdm), pytest.raises(ValueError, match="CUDA"):
+        sdm.sdm_scan_forward(kp, args["qp"], args["v"], args["alpha"], args["beta"], args["M"],
+                             W=W, R=W)
+    # decode, state init, selection and norm/gate
+    dk = torch.zeros(B, H, 2 * S1)
+    with no_launch(sdm), pytest.raises(ValueError, match="M has shape"):
+        sdm.sdm_decode_step(dk, dk, torch.zeros(B, H, d_v), torch.zeros(B, H), torch.zeros(B, H),
+                            torch.zeros(2 * B, H, N, d_v), W=W, R=W)
+    with no_launch(sdm), pytest.raises(ValueError, match="M0 has shape"):
+        sdm.sdm_state_init(torch.zeros(H, N, 2 * d_v), torch.zeros(B, H, N, d_v))
+    with no_launch(sdm), pytest.raises(ValueError, match="idx has shape"):
+        sdm.sdm_select(torch.zeros(5, 2 * S1), W, idx=torch.zeros(5, W + 1, dtype=torch.int32))
+    with no_launch(sdm), pytest.raises(ValueError, match="o has shape"):
+        sdm.sdm_norm_gate(torch.zeros(5, d_v, dtype=f), o=torch.zeros(5, d_v + 4))

@@ -328,6 +328,75 @@ def bench_prefill(args, dist: Dist, dev):
     return res
 
 
+PREFILL_CONFIGS = ("small", "layer1p4b")
+
+
+def bench_prefill_configs(args, dist: Dist, dev):
+    """The other prefill workloads: the AUTO engine's step and both engines' steps, each
+    timed alone with CUDA events (median of the timed steps) after a write of twice the L2
+    size (the small workload's inputs and state fit in L2).  One step is one
+    sdm_scan_forward with SDM_CONTINUE, as in the headline."""
+    import sparse_memory_linear_b200 as sdm
+
+    stream = torch.cuda.current_stream(dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 64 << 20), dtype=torch.uint8, device=dev)
+    peak, peak_kind = hbm_peak()
+    out = []
+    for name in PREFILL_CONFIGS:
+        wl = sdm_synth.WORKLOADS[name]
+        g = {k: v.to(dev) for k, v in sdm_synth.make_inputs(wl, device=dev).items()}
+        M = torch.empty((wl.B, wl.H, wl.N, wl.d_v), dtype=torch.float32, device=dev)
+        sdm.sdm_state_init(g["M0"], M)
+        y = torch.empty((wl.B, wl.T, wl.H, wl.d_v), dtype=torch.float32, device=dev)
+        o = torch.empty_like(y)
+        ms = {}
+        for engine in ("auto", "seq", "slot"):
+            def step():
+                sdm.sdm_scan_forward(g["kp"], g["qp"], g["v"], g["alpha"], g["beta"], M,
+                                     W=wl.W, R=wl.R, S1=wl.S1, init="continue", gate=g["gate"],
+                                     y=y, o=o, engine=engine, stream=stream)
+            for _ in range(args.warmup):
+                step()
+            times = []
+            for _ in range(max(3, args.steps)):
+                flush.zero_()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                step()
+                b.record(stream)
+                torch.cuda.synchronize(dev)
+                times.append(a.elapsed_time(b))
+            ms[engine] = dist.max(statistics.median(times))
+        sdm.sdm_profile_enable(True)
+        sdm.sdm_scan_forward(g["kp"], g["qp"], g["v"], g["alpha"], g["beta"], M, W=wl.W,
+                             R=wl.R, S1=wl.S1, init="continue", gate=g["gate"], y=y, o=o,
+                             stream=stream)
+        torch.cuda.synchronize(dev)
+        prof = sdm.sdm_profile_read()
+        sdm.sdm_profile_enable(False)
+        if sdm.sdm_get_device_status() != 0:
+            raise RuntimeError("device status word set during the benchmark")
+        th = wl.B * wl.T * wl.H
+        step_s = ms["auto"] * 1e-3
+        out.append({
+            "workload": wl.name, "shape": wl.note, "metric": METRIC, "unit": UNIT,
+            "value": weak_scaling_value(th, step_s, dist.world), "ms_per_step": ms["auto"],
+            "engine": "slot" if prof["scan_slot"][1] else "seq",
+            "engine_ms_per_step": {"seq": ms["seq"], "slot": ms["slot"]},
+            "whole_step_hbm": {"bytes_per_token_head": algorithmic_bytes(wl),
+                               "GBps": th * algorithmic_bytes(wl) / step_s / 1e9,
+                               "frac": th * algorithmic_bytes(wl) / step_s / 1e9 / peak,
+                               "peak": peak, "peak_kind": peak_kind},
+            "kernels_ms_per_step": {k: v for k, (v, n) in prof.items() if n},
+            "l2": "flushed before every timed step (a write of twice the L2 size)",
+        })
+        del g, M, y, o
+        torch.cuda.empty_cache()
+    return out
+
+
 def step_bytes_of(wl) -> float:
     """Algorithmic bytes of one decode step of every (sequence, head)."""
     return wl.B * wl.H * algorithmic_bytes(wl)
@@ -501,6 +570,8 @@ def main(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the prefill lines of the small and 1.4B-like workloads")
     ap.add_argument("--cpu-tokens", type=int, default=8192,
                     help="tokens per head of the CPU-oracle sample")
     ap.add_argument("--reference-tokens", type=int, default=2048)
@@ -575,6 +646,8 @@ def main(argv=None):
                           f"{os.cpu_count()} host cores have work)"}
         del g
         torch.cuda.empty_cache()
+        if not args.no_configs and args.only is None:
+            line["prefill_configs"] = bench_prefill_configs(args, dist, dev)
         if not args.no_decode:
             line["decode"] = bench_decode(args, dist, dev)
         if dist.rank == 0:

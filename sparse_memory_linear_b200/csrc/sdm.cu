@@ -4,6 +4,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <cmath>
 #include <mutex>
 #include <utility>
 #include <vector>
@@ -257,14 +258,42 @@ bool slot_engine_fits(const sdm_shape& s) {
          rows < (1LL << 31) && s.T < (1 << 24);
 }
 
-// Engine of an AUTO request: the sequential engine needs enough (sequence, head, column
-// slice) units to fill the GPU; below that the slot engine, whose parallelism is the
-// number of distinct slots touched, does better.
+// Prefill times of both engines, measured on one B200 (CUDA events around one
+// sdm_scan_forward with SDM_CONTINUE: selection, engine and norm/gate; bf16 inputs, W = R =
+// 64).  AUTO takes the engine that was faster on the measured shape nearest to the request.
+struct EngineMeasure {
+  int B, H, T, N, d_v;
+  float seq_ms, slot_ms;
+};
+constexpr EngineMeasure kEngineTable[] = {
+    {2, 4, 2048, 65536, 64, 12.32f, 0.611f},          // small layer
+    {4, 8, 8192, 262144, 128, 28.80f, 11.98f},        // 1.4B-like layer
+    {1, 4, 262144, 1048576, 256, 1769.2f, 57.36f},    // long prefill, skewed slots
+    {64, 8, 256, 262144, 128, 12.82f, 6.34f},         // many short sequences
+};
+
+inline double log2d(double x) { return x > 1.0 ? std::log2(x) : 0.0; }
+
+// Engine of an AUTO request: the sequential engine when the slot engine cannot hold the
+// shape (its event keys and counts), otherwise the faster engine of the nearest measured
+// shape, by distance over log2 of the (sequence, head) units, tokens, slots and width.
 int pick_engine(const sdm_shape& s, int requested, int sms) {
+  (void)sms;
   if (requested != SDM_ENGINE_AUTO) return requested;
   if (!slot_engine_fits(s)) return SDM_ENGINE_SEQ;
-  const long long units = (long long)s.B * s.H * (s.d_v / 32 > 0 ? s.d_v / 32 : 1);
-  return (units < 2LL * sms && s.d_v >= 128) ? SDM_ENGINE_SLOT : SDM_ENGINE_SEQ;
+  double best = 1e30;
+  int engine = SDM_ENGINE_SLOT;
+  for (const EngineMeasure& m : kEngineTable) {
+    const double d = std::fabs(log2d((double)s.B * s.H) - log2d((double)m.B * m.H)) +
+                     std::fabs(log2d(s.T) - log2d(m.T)) +
+                     std::fabs(log2d((double)s.S1 * s.S2) - log2d(m.N)) +
+                     std::fabs(log2d(s.d_v) - log2d(m.d_v));
+    if (d < best) {
+      best = d;
+      engine = m.seq_ms < m.slot_ms ? SDM_ENGINE_SEQ : SDM_ENGINE_SLOT;
+    }
+  }
+  return engine;
 }
 
 template <int R8, int KC>

@@ -490,7 +490,18 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
       }
     }
   };
-  if (rows_smem) load_reads(warp);
+  if (rows_smem) {
+    // step 3 for this warp's first read rows, before the write loop: they are in flight with
+    // the write rows, and their registers are free again before the loop needs its own
+    load_reads(warp);
+    add_reads(warp);
+  }
+
+  // v of this lane's columns, held in registers for the write loop when it is one float4
+  // (wider rows read it from shared memory per row: registers are short there)
+  constexpr bool kVReg = NQ == 1;
+  float4 vreg = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (kVReg && lane < d4) vreg = reinterpret_cast<const float4*>(vs)[lane];
 
   // step 2 on one write row whose old value is `old`: store the new row, and add it to the
   // read sum if the token also reads the slot
@@ -507,12 +518,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
     const float kb = be * wt_w[j];
     const float ka = al * (1.0f - kb);
     float4* row = reinterpret_cast<float4*>(Mbh + (size_t)sl * a.d_v);
-    const float4* v4 = reinterpret_cast<const float4*>(vs);
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
       const int c = lane + 32 * q;
       if (c < d4) {
-        const float4 vv = v4[c];
+        const float4 vv = kVReg ? vreg : reinterpret_cast<const float4*>(vs)[c];
         float4 nw;
         nw.x = fmaf(ka, old[q].x, kb * vv.x);
         nw.y = fmaf(ka, old[q].y, kb * vv.y);
@@ -577,7 +587,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
     load_reads(warp);
   }
   // step 3 for the read rows this token does not write
-  add_reads(warp);
+  if (!rows_smem) add_reads(warp);
   for (int j0 = warp + DEC_WARPS * RB; j0 < a.R; j0 += DEC_WARPS * RB) {
     load_reads(j0);
     add_reads(j0);

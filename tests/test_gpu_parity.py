@@ -173,14 +173,22 @@ def test_scan_edge_shapes(sdm, kw, engine):
     full_check(wl, g, out, M, gamma=g["gamma"])
 
 
-def test_scan_without_gate_or_output(sdm):
+@pytest.mark.parametrize("engine", ENGINES)
+def test_scan_without_gate_or_output(sdm, engine):
+    """No gate, and no output o: y and the state are those of the run with o.  The state is
+    deterministic in both engines; the slot engine adds each read into y with float atomics,
+    whose order (and so y's last bits) may change from run to run."""
     wl = sdm_synth.WORKLOADS["tiny"].replace(B=2, T=20, seed=5)
     g = device_inputs(wl, with_gate=False)
-    out, M = run_scan(sdm, wl, g, eps=0.0)
+    out, M = run_scan(sdm, wl, g, eps=0.0, engine=engine)
     full_check(wl, g, out, M, eps=0.0)
-    out2, M2 = run_scan(sdm, wl, g, want_o=False)
+    out2, M2 = run_scan(sdm, wl, g, want_o=False, engine=engine)
     assert out2["o"] is None
-    assert torch.equal(out2["y"], out["y"]) and torch.equal(M2, M)
+    assert torch.equal(M2, M)
+    if engine == "seq":
+        assert torch.equal(out2["y"], out["y"])
+    else:
+        assert_close(host(out2["y"]), host(out["y"]), "y", atol=1e-7, rtol=1e-6)
 
 
 @pytest.mark.parametrize("engine", ENGINES)

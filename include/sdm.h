@@ -229,8 +229,10 @@ typedef enum {
     SDM_OPT_SLOT_CTAS_PER_SM = 4,   /* n > 0: at most n slot-engine scan CTAs per SM     */
     SDM_OPT_SEQ_COLUMNS = 5,        /* 4, 8, 16 or 32: the sequential engine's column
                                        slice (0: chosen by shape)                       */
-    SDM_OPT_SEQ_DEPTH = 6           /* 4 or 8: the sequential engine's gather-ahead
+    SDM_OPT_SEQ_DEPTH = 6,          /* 4 or 8: the sequential engine's gather-ahead
                                        depth in tokens (0: chosen by slice)             */
+    SDM_OPT_SLOT_CTA_STATS = 7      /* 1: the slot engine records per-CTA work
+                                       (sdm_slot_cta_stats)                             */
 } sdm_option;
 
 /* Sets an option.  SDM_ERR_INVALID_ARG (and no change) for an unknown option or a value
@@ -239,6 +241,18 @@ sdm_status sdm_set_option(int32_t option, int32_t value);
 
 /* The option's current value, or -1 for an unknown option. */
 int32_t sdm_get_option(int32_t option);
+
+/* Load balance of the slot engine.  While SDM_OPT_SLOT_CTA_STATS is 1, every launch of the
+ * engine's chunk kernel adds, for each of its CTAs (by block index, the first
+ * SDM_SLOT_STATS_CTAS of them), four counters to a table the library holds on each device:
+ * [0] events applied from short segments, [1] events of the long (hot-slot) segments it
+ * took, [2] spans of sorted events it took from the work queue, [3] the summed busy
+ * nanoseconds of its warps.  sdm_slot_cta_stats waits for the calling device to finish its
+ * work, copies the first max_ctas rows of that device's table to out[max_ctas][4] (host
+ * memory) and, when reset != 0, clears the table.  The counters use the device's global
+ * timer; nothing else changes with the option. */
+#define SDM_SLOT_STATS_CTAS 1024
+sdm_status sdm_slot_cta_stats(uint64_t *out, int32_t max_ctas, int32_t reset);
 
 /* Number of kernels this library has launched in this process, on every device. */
 uint64_t sdm_launch_count(void);

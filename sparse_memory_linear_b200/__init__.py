@@ -28,6 +28,7 @@ from ._binding import (  # noqa: F401
     sdm_scan_forward_noalloc,
     sdm_select,
     sdm_set_option,
+    sdm_slot_cta_stats,
     sdm_state_init,
     sdm_status_string,
     sdm_workspace_size,

@@ -63,6 +63,7 @@ def library():
         "sdm_launch_count": ([], ctypes.c_uint64),
         "sdm_set_option": ([I, I], I),
         "sdm_get_option": ([I], I),
+        "sdm_slot_cta_stats": ([P, I, I], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -342,7 +343,18 @@ def sdm_profile_read() -> dict:
 
 
 OPTION = {"no_pdl": 1, "select_general": 2, "select_ctas_per_sm": 3, "slot_ctas_per_sm": 4,
-          "seq_columns": 5, "seq_depth": 6}
+          "seq_columns": 5, "seq_depth": 6, "slot_cta_stats": 7}
+SLOT_STATS_CTAS = 1024
+
+
+def sdm_slot_cta_stats(max_ctas: int = SLOT_STATS_CTAS, reset: bool = True):
+    """Per-CTA work of the slot engine recorded while option "slot_cta_stats" is 1: an int64
+    array [max_ctas, 4] of (short-segment events, long-segment events, spans, busy warp-ns)."""
+    import numpy as np
+    out = np.zeros((int(max_ctas), 4), np.uint64)
+    _check(library().sdm_slot_cta_stats(ctypes.c_void_p(out.ctypes.data), int(max_ctas),
+                                        1 if reset else 0), "sdm_slot_cta_stats")
+    return out.astype(np.int64)
 
 
 def sdm_set_option(option: str, value: int):

@@ -261,20 +261,17 @@ __device__ __forceinline__ void decode_select_group(const DecodeArgs& a, const D
           atomicOr(&bits[(f >> 5) & 63u], 1u << (f & 31u));
         });
   }
-  if (st < K) {
-    // the softmax denominator, the same sum in the same order on every thread (ev is zero
-    // past K up to the next multiple of 4)
-    const float4* e4 = reinterpret_cast<const float4*>(ev);
-    float s_0 = 0.0f, s_1 = 0.0f, s_2 = 0.0f, s_3 = 0.0f;
-    for (int j = 0; j < (K + 3) / 4; ++j) {
-      const float4 e = e4[j];
-      s_0 += e.x;
-      s_1 += e.y;
-      s_2 += e.z;
-      s_3 += e.w;
-    }
-    out_wt[st] = ev[st] * (1.0f / ((s_0 + s_1) + (s_2 + s_3)));
-  }
+  // the softmax denominator: a butterfly sum within each of the group's four warps, then the
+  // four warp sums in a fixed order (the same sum on every thread)
+  const float e_own = st < K ? ev[st] : 0.0f;
+  float esum = e_own;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) esum += __shfl_xor_sync(FULL_MASK, esum, o);
+  if (lane == 0) cctl->wmin[st >> 5] = __float_as_uint(esum);
+  group_bar(5 + s, 128);
+  const float total = (__uint_as_float(cctl->wmin[0]) + __uint_as_float(cctl->wmin[1])) +
+                      (__uint_as_float(cctl->wmin[2]) + __uint_as_float(cctl->wmin[3]));
+  if (st < K) out_wt[st] = e_own * (1.0f / total);
 }
 
 // E == 0: warp-per-row selection (fp32 halves, halves longer than 1024 scores); otherwise
@@ -283,6 +280,9 @@ __device__ __forceinline__ void decode_select_group(const DecodeArgs& a, const D
 template <int E, int KC, int NQ>
 __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, DecLayout L) {
   extern __shared__ __align__(16) unsigned char smem[];
+  // the next step may be scheduled at once: its CTAs take the SM slots this step frees, and
+  // their selection overlaps this step's row traffic
+  grid_launch_dependents();
   const int bh = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool bf16 = a.in_bf16 != 0;
@@ -399,9 +399,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
     __syncthreads();
   }
 
-  // The selection is done: the next step may be scheduled now (its CTAs take the SM slots
-  // freed by this step, and their selection overlaps this step's row traffic).
-  grid_launch_dependents();
   // Everything above reads only this step's inputs.  A step launched with programmatic
   // stream serialisation may have started while the step before it still ran: wait for that
   // grid (and its memory) before touching anything it writes (sel_out, M, y, o).

@@ -357,7 +357,19 @@ struct SlotArgs {
   int hot_cap;
   int B, T, H, N, d_v, v_bf16;
   KeyBits kb;
+  unsigned long long* cta_stats;  // [SDM_SLOT_STATS_CTAS][4] work per CTA, or null
 };
+
+// Per-CTA work of the chunk kernel (load-balance analysis), added while enabled:
+// [0] events applied from short segments, [1] events of the long segments taken,
+// [2] spans taken, [3] summed busy nanoseconds of the CTA's warps.
+__device__ unsigned long long g_slot_cta_stats[SDM_SLOT_STATS_CTAS * 4];
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 constexpr int SLOT_THREADS = 256;
 constexpr int SLOT_WARPS = SLOT_THREADS / 32;
@@ -471,6 +483,10 @@ __global__ void __launch_bounds__(SLOT_THREADS, (NQ <= 2 ? 4 : 1)) slot_chunk_ke
   extern __shared__ __align__(16) unsigned char smem[];
   const uint32_t e0 = a.offs[chunk], e1 = a.offs[chunk + 1];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned long long* stats =
+      a.cta_stats && blockIdx.x < SDM_SLOT_STATS_CTAS ? a.cta_stats + 4 * blockIdx.x : nullptr;
+  const unsigned long long t_start = stats ? global_ns() : 0ull;
+  unsigned long long n_short = 0, n_long = 0, n_spans = 0;
   const int d4 = a.d_v / 4;
   const bool bf16 = a.v_bf16 != 0;
   const unsigned lt = lanemask_lt();
@@ -492,6 +508,7 @@ __global__ void __launch_bounds__(SLOT_THREADS, (NQ <= 2 ? 4 : 1)) slot_chunk_ke
     for (uint32_t hs = blockIdx.x; hs < nh; hs += gridDim.x) {
       const uint2 seg = a.hot_list[(size_t)chunk * a.hot_cap + hs];
       const uint32_t first = seg.x, n = seg.y;
+      if (warp == 0) n_long += n;
       int b, h;
       float* row = row_of(a.keys[first], b, h);
       const uint32_t per = (n + SLOT_WARPS - 1) / SLOT_WARPS;
@@ -552,6 +569,7 @@ __global__ void __launch_bounds__(SLOT_THREADS, (NQ <= 2 ? 4 : 1)) slot_chunk_ke
     if (lane == 0) span_id = atomicAdd(&a.span_next[chunk], 1u);
     span_id = __shfl_sync(FULL_MASK, span_id, 0);
     if (span_id >= (e1 - e0 + SLOT_SPAN - 1) / SLOT_SPAN) break;
+    ++n_spans;
     const uint32_t span = e0 + span_id * (uint32_t)SLOT_SPAN;
     const uint32_t span_end = min(e1, span + (uint32_t)SLOT_SPAN);
     // heads of the short segments starting in the span, in event order
@@ -587,6 +605,7 @@ __global__ void __launch_bounds__(SLOT_THREADS, (NQ <= 2 ? 4 : 1)) slot_chunk_ke
       }
     }
 
+    n_short += stop - first;
     auto issue = [&](int i) {
       if (i < nh) {
         int bb, hh;
@@ -717,6 +736,12 @@ __global__ void __launch_bounds__(SLOT_THREADS, (NQ <= 2 ? 4 : 1)) slot_chunk_ke
     close_segment();
     cp_async_wait<0>();
     __syncwarp();
+  }
+  if (stats && lane == 0) {
+    atomicAdd(stats + 0, n_short);
+    atomicAdd(stats + 1, n_long);
+    atomicAdd(stats + 2, n_spans);
+    atomicAdd(stats + 3, global_ns() - t_start);
   }
 }
 

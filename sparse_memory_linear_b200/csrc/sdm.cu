@@ -9,6 +9,8 @@
 #include <utility>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "decode.cuh"
 #include "norm_init.cuh"
@@ -36,6 +38,15 @@ constexpr size_t WS_ALIGN = 256;
       return SDM_ERR_CUDA;                       \
     }                                            \
   } while (0)
+
+// An NVTX range around one call of the ABI (visible in Nsight timelines; a few nanoseconds
+// when no tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Process-wide launch options (sdm_option); 0 everywhere by default.
 constexpr int OPT_SLOTS = 8;
@@ -510,6 +521,12 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
   a.d_v = s.d_v;
   a.v_bf16 = s.in_dtype == SDM_BF16;
   a.kb = WL.kb;
+  a.cta_stats = nullptr;
+  if (opt(SDM_OPT_SLOT_CTA_STATS)) {
+    void* p = nullptr;
+    SDM_CUDA_TRY(cudaGetSymbolAddress(&p, g_slot_cta_stats));
+    a.cta_stats = static_cast<unsigned long long*>(p);
+  }
   const int d4 = s.d_v / 4;
   for (int t0 = 0; t0 < s.T; t0 += WL.chunk) {
     const int ct = s.T - t0 < WL.chunk ? s.T - t0 : WL.chunk;
@@ -616,6 +633,7 @@ size_t sdm_workspace_size(sdm_shape shape, int32_t engine) {
 
 sdm_status sdm_select(const void* halves, sdm_shape shape, int32_t K, int32_t* idx, float* wt,
                       void* stream) {
+  NvtxRange nvtx_range("sdm_select");
   sdm_shape s = shape;  // only B, T, H, S1, S2 and in_dtype matter here
   s.W = s.R = 1;
   s.d_v = s.in_dtype == SDM_BF16 ? 8 : 4;
@@ -631,6 +649,7 @@ sdm_status sdm_select(const void* halves, sdm_shape shape, int32_t K, int32_t* i
 }
 
 sdm_status sdm_state_init(const float* M0, float* M, sdm_shape shape, void* stream) {
+  NvtxRange nvtx_range("sdm_state_init");
   // only B, H, N = S1*S2 and d_v matter here
   if (shape.B < 1 || shape.H < 1 || shape.S1 < 1 || shape.S2 < 1) return SDM_ERR_INVALID_ARG;
   if (shape.d_v < 4 || shape.d_v > 1024 || shape.d_v % 4 != 0) return SDM_ERR_INVALID_ARG;
@@ -644,6 +663,7 @@ sdm_status sdm_state_init(const float* M0, float* M, sdm_shape shape, void* stre
 
 sdm_status sdm_norm_gate(const float* y, const void* gate, const float* gamma, float eps,
                          int32_t act, sdm_shape shape, float* o, void* stream) {
+  NvtxRange nvtx_range("sdm_norm_gate");
   sdm_shape s = shape;  // only B, T, H, d_v and in_dtype matter here
   s.S1 = s.S2 = 1;
   s.W = s.R = 1;
@@ -663,6 +683,7 @@ sdm_status sdm_scan_forward(const void* kp, const void* qp, const void* v, const
                             float* y, const void* gate, const float* gamma, float eps,
                             int32_t act, float* o, int32_t* sel_out, int32_t engine, void* ws,
                             size_t ws_bytes, sdm_shape shape, void* stream) {
+  NvtxRange nvtx_range("sdm_scan_forward");
   const sdm_shape& s = shape;
   if (!shape_ok(s, true)) return SDM_ERR_INVALID_ARG;
   if (init != SDM_INIT_FROM_M0 && init != SDM_CONTINUE) return SDM_ERR_INVALID_ARG;
@@ -771,6 +792,7 @@ static sdm_status decode_step(const void* kp, const void* qp, const void* v, con
                               const float* beta, float* M, float* y, const void* gate,
                               const float* gamma, float eps, int32_t act, float* o,
                               int32_t* sel_out, sdm_shape shape, void* stream, bool chained) {
+  NvtxRange nvtx_range("sdm_decode_step");
   sdm_shape s = shape;
   s.T = 1;
   if (!shape_ok(s, false)) return SDM_ERR_INVALID_ARG;
@@ -878,6 +900,7 @@ sdm_status sdm_set_option(int32_t option, int32_t value) {
     case SDM_OPT_SLOT_CTAS_PER_SM: ok = value >= 0 && value <= 64; break;
     case SDM_OPT_SEQ_COLUMNS: ok = value == 0 || value == 4 || value == 8 || value == 16 || value == 32; break;
     case SDM_OPT_SEQ_DEPTH: ok = value == 0 || value == 4 || value == 8; break;
+    case SDM_OPT_SLOT_CTA_STATS: ok = value == 0 || value == 1; break;
     default: ok = false;
   }
   if (!ok) return SDM_ERR_INVALID_ARG;
@@ -886,8 +909,20 @@ sdm_status sdm_set_option(int32_t option, int32_t value) {
 }
 
 int32_t sdm_get_option(int32_t option) {
-  if (option < SDM_OPT_NO_PDL || option > SDM_OPT_SEQ_DEPTH) return -1;
+  if (option < SDM_OPT_NO_PDL || option > SDM_OPT_SLOT_CTA_STATS) return -1;
   return opt(option);
+}
+
+sdm_status sdm_slot_cta_stats(uint64_t* out, int32_t max_ctas, int32_t reset) {
+  if (!out || max_ctas < 1 || max_ctas > SDM_SLOT_STATS_CTAS) return SDM_ERR_INVALID_ARG;
+  SDM_CUDA_TRY(cudaDeviceSynchronize());
+  SDM_CUDA_TRY(cudaMemcpyFromSymbol(out, g_slot_cta_stats, (size_t)max_ctas * 4 * 8));
+  if (reset) {
+    void* p = nullptr;
+    SDM_CUDA_TRY(cudaGetSymbolAddress(&p, g_slot_cta_stats));
+    SDM_CUDA_TRY(cudaMemset(p, 0, sizeof(unsigned long long) * 4 * SDM_SLOT_STATS_CTAS));
+  }
+  return SDM_OK;
 }
 
 sdm_status sdm_profile_enable(int32_t on) {
@@ -979,6 +1014,7 @@ extern "C" sdm_status sdm_scan_forward_noalloc(const void* kp, const void* qp, c
                                                float eps, int32_t act, float* o,
                                                int32_t* sel_out, sdm_shape shape,
                                                void* stream) {
+  NvtxRange nvtx_range("sdm_scan_forward_noalloc");
   if (!shape_ok(shape, true)) return SDM_ERR_INVALID_ARG;
   if (sdm_workspace_size(shape, SDM_ENGINE_SEQ) > (size_t)SDM_NOALLOC_SCRATCH_BYTES)
     return SDM_ERR_INVALID_ARG;

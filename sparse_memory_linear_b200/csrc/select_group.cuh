@@ -41,7 +41,7 @@ __device__ __forceinline__ void group_bar(int id, int nthreads) {
 // Control words of one group, in shared memory.
 struct GroupCtl {
   uint32_t wmax[4];  // per-warp maximum key
-  uint32_t wmin[4];  // per-warp bracket key
+  uint32_t wmin[4];  // per-warp bracket key (candidate groups: per-warp softmax sums)
   uint32_t bin, run, cnt_bin;
   uint32_t count;    // list append counter, zero before the group starts
   uint32_t kth;      // key of the K-th ranked composite (set by the caller's emit)

@@ -201,9 +201,9 @@ def test_options_are_explicit_and_validated(sdm):
     for name, code in sdm.OPTION.items():
         assert sdm.sdm_get_option(name) == 0
     good = {"no_pdl": 1, "select_general": 1, "select_ctas_per_sm": 3, "slot_ctas_per_sm": 2,
-            "seq_columns": 16, "seq_depth": 8}
+            "seq_columns": 16, "seq_depth": 8, "slot_cta_stats": 1}
     bad = {"no_pdl": 2, "select_general": -1, "select_ctas_per_sm": 65,
-           "slot_ctas_per_sm": -2, "seq_columns": 12, "seq_depth": 5}
+           "slot_ctas_per_sm": -2, "seq_columns": 12, "seq_depth": 5, "slot_cta_stats": 3}
     try:
         for name in sdm.OPTION:
             assert lib.sdm_set_option(sdm.OPTION[name], bad[name]) == 1
@@ -214,6 +214,7 @@ def test_options_are_explicit_and_validated(sdm):
         for name in sdm.OPTION:
             sdm.sdm_set_option(name, 0)
     assert lib.sdm_set_option(0, 0) == 1 and lib.sdm_set_option(99, 0) == 1
+    assert lib.sdm_slot_cta_stats(None, 4, 0) == 1  # no output buffer: refused before any CUDA call
     assert lib.sdm_get_option(0) == -1 and lib.sdm_get_option(99) == -1
     csrc = os.path.join(ROOT, "sparse_memory_linear_b200", "csrc")
     for f in os.listdir(csrc):

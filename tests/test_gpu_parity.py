@@ -417,3 +417,23 @@ def test_norm_gate(sdm, act, dt):
     assert_close(host(o), ref, "o")
     o2 = sdm.sdm_norm_gate(y.to(DEV), eps=0.5)
     assert_close(host(o2), oracle.norm_gate(y.numpy(), None, None, 0.5), "o ungated")
+
+
+def test_slot_engine_cta_stats_account_for_every_event(sdm):
+    """With per-CTA statistics on, the slot engine's CTAs together apply every event of the
+    step exactly once (short segments plus long, hot-slot segments); with them off nothing is
+    recorded.  Skewed halves make hot slots, so both kinds occur."""
+    wl = sdm_synth.WORKLOADS["long_skew"].replace(T=4096, H=1, seed=41)
+    g = device_inputs(wl)
+    sdm.sdm_slot_cta_stats(reset=True)
+    sdm.sdm_set_option("slot_cta_stats", 1)
+    try:
+        out, M = run_scan(sdm, wl, g, engine="slot", want_o=False)
+    finally:
+        sdm.sdm_set_option("slot_cta_stats", 0)
+    st = sdm.sdm_slot_cta_stats(reset=True)
+    events = wl.B * wl.T * wl.H * (wl.W + wl.R)
+    assert int(st[:, 0].sum() + st[:, 1].sum()) == events
+    assert st[:, 1].sum() > 0 and st[:, 2].sum() > 0 and st[:, 3].sum() > 0
+    run_scan(sdm, wl, g, engine="slot", want_o=False)
+    assert int(sdm.sdm_slot_cta_stats(reset=True).sum()) == 0

@@ -397,6 +397,54 @@ def bench_prefill_configs(args, dist: Dist, dev):
     return out
 
 
+def bench_balance(args, dev):
+    """Load balance of the slot engine: one step of the prefill workload (with --override
+    applied) with the library's per-CTA work counters on (sdm_slot_cta_stats), after W
+    warm-up steps.  Reports events, spans and busy time per CTA (min, median, max, mean,
+    max/mean); busy time is the mean over a CTA's eight warps."""
+    import sparse_memory_linear_b200 as sdm
+
+    wl = sdm_synth.WORKLOADS[args.workload]
+    g = {k: v.to(dev) for k, v in sdm_synth.make_inputs(wl, device=dev).items()}
+    M = torch.empty((wl.B, wl.H, wl.N, wl.d_v), dtype=torch.float32, device=dev)
+    sdm.sdm_state_init(g["M0"], M)
+
+    def step():
+        sdm.sdm_scan_forward(g["kp"], g["qp"], g["v"], g["alpha"], g["beta"], M, W=wl.W,
+                             R=wl.R, S1=wl.S1, init="continue", gate=g["gate"], engine="slot")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    sdm.sdm_slot_cta_stats(reset=True)
+    sdm.sdm_set_option("slot_cta_stats", 1)
+    try:
+        step()
+    finally:
+        sdm.sdm_set_option("slot_cta_stats", 0)
+    st = sdm.sdm_slot_cta_stats(reset=True)
+    sdm.sdm_profile_enable(True)
+    step()
+    torch.cuda.synchronize(dev)
+    prof = sdm.sdm_profile_read()
+    sdm.sdm_profile_enable(False)
+    active = st[st[:, 3] > 0]
+    ev = active[:, 0] + active[:, 1]
+
+    def q(x):
+        x = np.asarray(x, np.float64)
+        return {"min": float(x.min()), "p50": float(np.median(x)), "max": float(x.max()),
+                "mean": float(x.mean()), "max_over_mean": float(x.max() / max(x.mean(), 1e-9))}
+
+    return {"workload": wl.name, "shape": wl.note, "ctas": int(active.shape[0]),
+            "chunk_launches": int(prof["scan_slot"][1]),
+            "scan_ms": prof["scan_slot"][0], "events_total": int(ev.sum()),
+            "events_in_long_segments": int(active[:, 1].sum()),
+            "events_per_cta": q(ev), "short_events_per_cta": q(active[:, 0]),
+            "long_events_per_cta": q(active[:, 1]), "spans_per_cta": q(active[:, 2]),
+            "busy_us_per_cta": q(active[:, 3] / 8.0 / 1e3)}
+
+
 def step_bytes_of(wl) -> float:
     """Algorithmic bytes of one decode step of every (sequence, head)."""
     return wl.B * wl.H * algorithmic_bytes(wl)
@@ -575,7 +623,7 @@ def main(argv=None):
     ap.add_argument("--cpu-tokens", type=int, default=8192,
                     help="tokens per head of the CPU-oracle sample")
     ap.add_argument("--reference-tokens", type=int, default=2048)
-    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "balance"], default=None,
                     help="run one part (profiling of a small case)")
     ap.add_argument("--override", default="",
                     help="workload fields to change, e.g. B=1,T=4096 (prefill workload)")
@@ -608,6 +656,11 @@ def main(argv=None):
         import sparse_memory_linear_b200 as sdm
         sdm.library()
 
+        if args.only == "balance":
+            out = bench_balance(args, dev)
+            if dist.rank == 0:
+                print(json.dumps({"balance": out}), flush=True)
+            return 0
         if args.only == "decode":
             out = bench_decode(args, dist, dev)
             if dist.rank == 0:

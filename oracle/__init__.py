@@ -62,6 +62,8 @@ def _load():
         lib.sdm_oracle_pass.argtypes = [I, I, I, I, I, P, P, P, P, P, L, P, P, L, I, P, P,
                                         P, P, P]
         lib.sdm_oracle_pass.restype = I
+        lib.sdm_oracle_pass_coupled.argtypes = lib.sdm_oracle_pass.argtypes
+        lib.sdm_oracle_pass_coupled.restype = I
         lib.sdm_oracle_norm_gate.argtypes = [L, I, P, P, P, ctypes.c_double, I, P]
         lib.sdm_oracle_norm_gate.restype = I
         _lib = lib
@@ -126,8 +128,12 @@ def norm_gate(y, g=None, gamma=None, eps: float = 1e-6, act: str | int = "silu")
 
 def run_unit(kp, qp, v, alpha, beta, M_init, b: int, h: int, *, S1: int, W: int, R: int,
              rows=None, want_y=None, t_end=None, select_mode: str = "product_key",
-             threads: int = 1, selection=None):
+             threads: int = 1, selection=None, coupled: bool = False):
     """Steps 1-3 for one (sequence b, head h) over tokens [0, t_end).
+
+    coupled: the coupled delta rule (one prediction shared by the token's written rows,
+    sdm_oracle_pass_coupled) instead of the per-slot write; every written row must then be
+    tracked.
 
     rows: tracked slot rows (int array) or None for all N rows.
     want_y: bool array [t_end] of tokens whose read result is wanted, or None (all).
@@ -186,9 +192,10 @@ def run_unit(kp, qp, v, alpha, beta, M_init, b: int, h: int, *, S1: int, W: int,
     wy = None if want_y is None else np.ascontiguousarray(want_y, dtype=np.uint8)
     y = np.full((t_end, d_v), np.nan, np.float64)
     M_out = np.empty((n_rows, d_v), np.float32)
-    rc = lib.sdm_oracle_pass(t_end, N, d_v, W, R, _ptr(idx_w), _ptr(wt_w), _ptr(idx_r),
-                             _ptr(wt_r), _ptr(v_u), d_v, _ptr(a_u), _ptr(be_u), 1, n_rows,
-                             _ptr(rows_arr), _ptr(M_in), _ptr(wy), _ptr(y), _ptr(M_out))
+    fn = lib.sdm_oracle_pass_coupled if coupled else lib.sdm_oracle_pass
+    rc = fn(t_end, N, d_v, W, R, _ptr(idx_w), _ptr(wt_w), _ptr(idx_r), _ptr(wt_r), _ptr(v_u),
+            d_v, _ptr(a_u), _ptr(be_u), 1, n_rows, _ptr(rows_arr), _ptr(M_in), _ptr(wy),
+            _ptr(y), _ptr(M_out))
     if rc != 0:
         raise ValueError(f"sdm_oracle_pass failed ({rc})")
     return dict(idx_w=idx_w, wt_w=wt_w, idx_r=idx_r, wt_r=wt_r, y=y, M=M_out, rows=rows_arr)
@@ -196,7 +203,7 @@ def run_unit(kp, qp, v, alpha, beta, M_init, b: int, h: int, *, S1: int, W: int,
 
 def forward(kp, qp, v, alpha, beta, M_init, *, S1: int, W: int, R: int, gate=None,
             gamma=None, eps: float = 1e-6, act="silu", select_mode: str = "product_key",
-            threads: int = 1):
+            threads: int = 1, coupled: bool = False):
     """The whole pass over every (b, h) and every token, all rows tracked.
 
     Returns dict(idx_w [B,T,H,W], idx_r [B,T,H,R], wt_w, wt_r, y [B,T,H,d_v] float64,
@@ -216,7 +223,7 @@ def forward(kp, qp, v, alpha, beta, M_init, *, S1: int, W: int, R: int, gate=Non
     def one(u):
         b, h = u
         r = run_unit(kp, qp, v, alpha, beta, M_init, b, h, S1=S1, W=W, R=R,
-                     select_mode=select_mode)
+                     select_mode=select_mode, coupled=coupled)
         idx_w[b, :, h], wt_w[b, :, h] = r["idx_w"], r["wt_w"]
         idx_r[b, :, h], wt_r[b, :, h] = r["idx_r"], r["wt_r"]
         y[b, :, h] = r["y"]

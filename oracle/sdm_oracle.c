@@ -25,7 +25,9 @@
  *     one, of the selected scores over the selected set only;
  *   - alpha_t and beta_t are per (token, head) scalars given as inputs;
  *   - the write of token t happens before its read (y_t reads M_t);
- *   - the delta prediction term is per slot (M~[i] of the slot being written);
+ *   - the delta prediction term is per slot (M~[i] of the slot being written); a second
+ *     entry point takes the coupled reading (one prediction shared by the token's written
+ *     rows), the one under which the method reduces to the gated delta rule;
  *   - RMSNorm is over d_v with epsilon eps and optional weight gamma; the output
  *     gate is act(g) with act in {silu, sigmoid, identity}.
  *
@@ -175,11 +177,11 @@ int sdm_oracle_select(const float *halves, long n, long row_stride, int S1, int 
  *   y     [T, d_v] read result (double); rows of unwanted tokens are left untouched
  *   M_out [n_rows, d_v] final values of the tracked rows (rounded to fp32)
  */
-int sdm_oracle_pass(int T, int N, int d_v, int W, int R, const int32_t *idx_w,
-                    const double *wt_w, const int32_t *idx_r, const double *wt_r,
-                    const float *v, long v_stride, const float *alpha, const float *beta,
-                    long ab_stride, int n_rows, const int32_t *rows, const float *M_in,
-                    const uint8_t *want_y, double *y, float *M_out) {
+static int pass_impl(int T, int N, int d_v, int W, int R, const int32_t *idx_w,
+                     const double *wt_w, const int32_t *idx_r, const double *wt_r,
+                     const float *v, long v_stride, const float *alpha, const float *beta,
+                     long ab_stride, int n_rows, const int32_t *rows, const float *M_in,
+                     const uint8_t *want_y, double *y, float *M_out, int coupled) {
     if (T < 0 || N < 1 || d_v < 1 || W < 1 || R < 1 || n_rows < 0) return ORACLE_ERR_ARG;
     if (!idx_w || !wt_w || !idx_r || !wt_r || !v || !alpha || !beta || !M_in || !M_out)
         return ORACLE_ERR_ARG;
@@ -188,15 +190,16 @@ int sdm_oracle_pass(int T, int N, int d_v, int W, int R, const int32_t *idx_w,
     int32_t *pos = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
     double *S = (double *)malloc(sizeof(double) * (size_t)n_rows * (size_t)d_v + 1);
     double *acc = (double *)malloc(sizeof(double) * (size_t)d_v);
-    if (!pos || !S || !acc) {
-        free(pos); free(S); free(acc);
+    double *pred = (double *)malloc(sizeof(double) * (size_t)d_v);
+    if (!pos || !S || !acc || !pred) {
+        free(pos); free(S); free(acc); free(pred);
         return ORACLE_ERR_NOMEM;
     }
     for (int i = 0; i < N; ++i) pos[i] = rows ? -1 : i;
     if (rows) {
         for (int p = 0; p < n_rows; ++p) {
             if (rows[p] < 0 || rows[p] >= N) {
-                free(pos); free(S); free(acc);
+                free(pos); free(S); free(acc); free(pred);
                 return ORACLE_ERR_ARG;
             }
             pos[rows[p]] = p;
@@ -209,8 +212,33 @@ int sdm_oracle_pass(int T, int N, int d_v, int W, int R, const int32_t *idx_w,
         const double a_t = (double)alpha[(long)t * ab_stride];
         const double b_t = (double)beta[(long)t * ab_stride];
         const float *v_t = v + (long)t * v_stride;
+        /* step 2, coupled reading: the token's written rows share one prediction,
+         * pred = sum over the write set of k_j * alpha_t * M[j]; then each written row
+         * becomes alpha_t * M[i] + beta_t * k_i * (v_t - pred).  Every written row must be
+         * tracked: the prediction reads them all. */
+        if (coupled) {
+            for (int c = 0; c < d_v; ++c) pred[c] = 0.0;
+            for (int j = 0; j < W && rc == ORACLE_OK; ++j) {
+                const int32_t i = idx_w[(long)t * W + j];
+                if (i < 0 || i >= N) rc = ORACLE_ERR_ARG;
+                else if (pos[i] < 0) rc = ORACLE_ERR_UNTRACKED;
+                else {
+                    const double kj = wt_w[(long)t * W + j];
+                    const double *row = S + (long)pos[i] * d_v;
+                    for (int c = 0; c < d_v; ++c) pred[c] += kj * (a_t * row[c]);
+                }
+            }
+            if (rc != ORACLE_OK) break;
+            for (int j = 0; j < W; ++j) {
+                const int32_t i = idx_w[(long)t * W + j];
+                const double kj = wt_w[(long)t * W + j];
+                double *row = S + (long)pos[i] * d_v;
+                for (int c = 0; c < d_v; ++c)
+                    row[c] = a_t * row[c] + b_t * kj * ((double)v_t[c] - pred[c]);
+            }
+        }
         /* step 2: gated delta write on the selected write slots */
-        for (int j = 0; j < W; ++j) {
+        for (int j = 0; j < W && !coupled; ++j) {
             const int32_t i = idx_w[(long)t * W + j];
             if (i < 0 || i >= N) { rc = ORACLE_ERR_ARG; break; }
             const int p = pos[i];
@@ -241,8 +269,34 @@ int sdm_oracle_pass(int T, int N, int d_v, int W, int R, const int32_t *idx_w,
     }
     if (rc == ORACLE_OK)
         for (long e = 0; e < (long)n_rows * d_v; ++e) M_out[e] = (float)S[e];
-    free(pos); free(S); free(acc);
+    free(pos); free(S); free(acc); free(pred);
     return rc;
+}
+
+int sdm_oracle_pass(int T, int N, int d_v, int W, int R, const int32_t *idx_w,
+                    const double *wt_w, const int32_t *idx_r, const double *wt_r,
+                    const float *v, long v_stride, const float *alpha, const float *beta,
+                    long ab_stride, int n_rows, const int32_t *rows, const float *M_in,
+                    const uint8_t *want_y, double *y, float *M_out) {
+    return pass_impl(T, N, d_v, W, R, idx_w, wt_w, idx_r, wt_r, v, v_stride, alpha, beta,
+                     ab_stride, n_rows, rows, M_in, want_y, y, M_out, 0);
+}
+
+/*
+ * Steps 2 and 3 with the coupled delta rule.  [P1] and [P3] state that SDM reduces exactly
+ * to the gated delta rule (GDN) when every slot is selected; the per-slot write of [P5]
+ * does not, while this one does: with the write set all N slots and key k (the slot
+ * weights), M_t = alpha_t (I - beta_t k k^T) M_{t-1} + beta_t k v_t^T.  Arguments as for
+ * sdm_oracle_pass; every written row must be tracked (ORACLE_ERR_UNTRACKED otherwise).
+ */
+int sdm_oracle_pass_coupled(int T, int N, int d_v, int W, int R, const int32_t *idx_w,
+                            const double *wt_w, const int32_t *idx_r, const double *wt_r,
+                            const float *v, long v_stride, const float *alpha,
+                            const float *beta, long ab_stride, int n_rows,
+                            const int32_t *rows, const float *M_in, const uint8_t *want_y,
+                            double *y, float *M_out) {
+    return pass_impl(T, N, d_v, W, R, idx_w, wt_w, idx_r, wt_r, v, v_stride, alpha, beta,
+                     ab_stride, n_rows, rows, M_in, want_y, y, M_out, 1);
 }
 
 /*

@@ -46,6 +46,10 @@ MUTANTS = {
     "write_weight_dropped": ("m[c] = m_tilde + b_t * k_i * (", "m[c] = m_tilde + b_t * ("),
     "beta_complemented": ("m[c] = m_tilde + b_t * k_i * (",
                           "m[c] = m_tilde + (1.0 - b_t) * k_i * ("),
+    # step 2, coupled reading: the shared prediction
+    "coupled_prediction_undecayed": ("pred[c] += kj * (a_t * row[c]);", "pred[c] += kj * row[c];"),
+    "coupled_prediction_unweighted": ("pred[c] += kj * (a_t * row[c]);",
+                                      "pred[c] += a_t * row[c];"),
     # step 3: the sparse read
     "read_weight_dropped": ("acc[c] += q_i * m[c];", "acc[c] += m[c];"),
     "read_uses_previous_tokens_slots": ("const int32_t i = idx_r[(long)t * R + j];",

@@ -153,6 +153,53 @@ def test_select_route_when_sums_round():
         assert c["expect_pruned_only"] != c["expect_route"]
 
 
+# ------------------------------------------------------- the coupled delta rule
+def test_coupled_rule_with_every_slot_selected_is_the_gated_delta_rule():
+    """SDM write-up on ai-paper-analysis.pages.dev and the m.163.com article: SDM reduces to
+    the gated delta rule when every slot is selected.  With the coupled prediction and
+    W = R = N, the pass must equal the dense recurrence M_t = alpha_t (I - beta_t k k^T)
+    M_{t-1} + beta_t k v_t^T, y_t = M_t^T q, written here with numpy matrices (k, q: the
+    slot weights scattered over all N slots).  The per-slot write does not reduce to it."""
+    rng = np.random.default_rng(12)
+    S1 = S2 = 4
+    N = S1 * S2
+    T, d_v = 9, 5
+    kp, qp, v, alpha, beta, M0 = rand_unit(rng, T, S1, S2, d_v)
+    M0 = (0.3 * rng.standard_normal((1, N, d_v))).astype(np.float32)
+    r = oracle.forward(kp, qp, v, alpha, beta, M0, S1=S1, W=N, R=N, coupled=True)
+    M = M0[0].astype(np.float64)
+    for t in range(T):
+        k = np.zeros(N)
+        q = np.zeros(N)
+        k[r["idx_w"][0, t, 0]] = r["wt_w"][0, t, 0]
+        q[r["idx_r"][0, t, 0]] = r["wt_r"][0, t, 0]
+        a_t, b_t = float(alpha[0, t, 0]), float(beta[0, t, 0])
+        M = a_t * (np.eye(N) - b_t * np.outer(k, k)) @ M + b_t * np.outer(k, v[0, t, 0])
+        np.testing.assert_allclose(r["y"][0, t, 0], M.T @ q, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(r["M"][0, 0], M.astype(np.float32), rtol=1e-6, atol=1e-7)
+    per_slot = oracle.forward(kp, qp, v, alpha, beta, M0, S1=S1, W=N, R=N)
+    assert np.abs(per_slot["y"] - r["y"]).max() > 1e-3
+
+
+def test_coupled_rule_with_one_write_slot_is_the_per_slot_rule():
+    """With W = 1 the shared prediction is the one written row, k alpha M[i] with k = 1:
+    the two readings coincide, bit for bit."""
+    rng = np.random.default_rng(13)
+    kp, qp, v, alpha, beta, M0 = rand_unit(rng, 30, 8, 8, 6)
+    a = oracle.forward(kp, qp, v, alpha, beta, M0, S1=8, W=1, R=5, coupled=True)
+    b = oracle.forward(kp, qp, v, alpha, beta, M0, S1=8, W=1, R=5)
+    np.testing.assert_array_equal(a["y"], b["y"])
+    np.testing.assert_array_equal(a["M"], b["M"])
+
+
+def test_coupled_rule_needs_every_written_row_tracked():
+    rng = np.random.default_rng(14)
+    kp, qp, v, alpha, beta, M0 = rand_unit(rng, 4, 8, 8, 4)
+    with pytest.raises(ValueError):
+        oracle.run_unit(kp, qp, v, alpha, beta, M0, 0, 0, S1=8, W=4, R=4, rows=[0, 1],
+                        want_y=np.zeros(4, bool), coupled=True)
+
+
 # -------------------------------------------------------------- slot weights (softmax)
 def test_weights_are_softmax_over_selected_set():
     rng = np.random.default_rng(11)

@@ -122,6 +122,26 @@ sdm_status sdm_scan_forward(const void *kp, const void *qp, const void *v, const
                             int32_t act, float *o, int32_t *sel_out, int32_t engine, void *ws,
                             size_t ws_bytes, sdm_shape shape, void *stream);
 
+/*
+ * Prefill with the coupled delta rule.  The write of [paper.rainbus.top summary, method step
+ * 2] predicts each written slot from its own row, M~[i]; the SDM write-up on
+ * ai-paper-analysis.pages.dev and the m.163.com article (section 二) also state that SDM
+ * reduces exactly to the gated delta rule when every slot is selected, which holds only when
+ * the token's written rows share one prediction:
+ *   p_t = sum_{j in I_w} k_j * alpha_t * M[j]
+ *   M[i] = alpha_t * M[i] + beta_t * k_i * (v_t - p_t)      for i in I_w
+ * (with I_w all N slots: M_t = alpha_t (I - beta_t k k^T) M_{t-1} + beta_t k v_t^T).  The
+ * read and step 4 are those of sdm_scan_forward, and so are the arguments.  The sequential
+ * engine computes it (SDM_ENGINE_AUTO takes it); the slot engine, which treats every slot as
+ * its own recurrence, cannot: SDM_ENGINE_SLOT returns SDM_ERR_UNSUPPORTED.
+ */
+sdm_status sdm_scan_forward_coupled(const void *kp, const void *qp, const void *v,
+                                    const float *alpha, const float *beta, const float *M0,
+                                    float *M, int32_t init, float *y, const void *gate,
+                                    const float *gamma, float eps, int32_t act, float *o,
+                                    int32_t *sel_out, int32_t engine, void *ws, size_t ws_bytes,
+                                    sdm_shape shape, void *stream);
+
 /* Size of the fixed scratch of sdm_scan_forward_noalloc (16 MiB per device). */
 #define SDM_NOALLOC_SCRATCH_BYTES (16u << 20)
 
@@ -183,6 +203,21 @@ sdm_status sdm_decode_step_chained(const void *kp, const void *qp, const void *v
                                    const void *gate, const float *gamma, float eps,
                                    int32_t act, float *o, int32_t *sel_out, sdm_shape shape,
                                    void *stream);
+
+/*
+ * One decode step with the coupled delta rule of sdm_scan_forward_coupled (arguments and
+ * launch as sdm_decode_step / sdm_decode_step_chained).  The write rows are summed in shared
+ * memory: shapes with W * d_v * 4 > 65536 bytes return SDM_ERR_UNSUPPORTED.
+ */
+sdm_status sdm_decode_step_coupled(const void *kp, const void *qp, const void *v,
+                                   const float *alpha, const float *beta, float *M, float *y,
+                                   const void *gate, const float *gamma, float eps, int32_t act,
+                                   float *o, int32_t *sel_out, sdm_shape shape, void *stream);
+sdm_status sdm_decode_step_coupled_chained(const void *kp, const void *qp, const void *v,
+                                           const float *alpha, const float *beta, float *M,
+                                           float *y, const void *gate, const float *gamma,
+                                           float eps, int32_t act, float *o, int32_t *sel_out,
+                                           sdm_shape shape, void *stream);
 
 /*
  * Step 4 alone [paper.rainbus.top summary, method step 4]: for each of the B*T*H rows

@@ -18,6 +18,8 @@ from ._binding import (  # noqa: F401
     library_path,
     sdm_decode_step,
     sdm_decode_step_chained,
+    sdm_decode_step_coupled,
+    sdm_decode_step_coupled_chained,
     sdm_get_device_status,
     sdm_get_option,
     sdm_launch_count,
@@ -25,6 +27,7 @@ from ._binding import (  # noqa: F401
     sdm_profile_enable,
     sdm_profile_read,
     sdm_scan_forward,
+    sdm_scan_forward_coupled,
     sdm_scan_forward_noalloc,
     sdm_select,
     sdm_set_option,

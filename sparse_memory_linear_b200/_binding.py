@@ -54,6 +54,10 @@ def library():
         "sdm_scan_forward": ([P, P, P, P, P, P, P, I, P, P, P, F, I, P, P, I, P, Z, S, P], I),
         "sdm_decode_step": ([P, P, P, P, P, P, P, P, P, F, I, P, P, S, P], I),
         "sdm_decode_step_chained": ([P, P, P, P, P, P, P, P, P, F, I, P, P, S, P], I),
+        "sdm_decode_step_coupled": ([P, P, P, P, P, P, P, P, P, F, I, P, P, S, P], I),
+        "sdm_decode_step_coupled_chained": ([P, P, P, P, P, P, P, P, P, F, I, P, P, S, P], I),
+        "sdm_scan_forward_coupled": ([P, P, P, P, P, P, P, I, P, P, P, F, I, P, P, I, P, Z, S, P],
+                                     I),
         "sdm_scan_forward_noalloc": ([P, P, P, P, P, P, P, I, P, P, P, F, I, P, P, S, P], I),
         "sdm_norm_gate": ([P, P, P, F, I, S, P, P], I),
         "sdm_get_device_status": ([P], I),
@@ -217,9 +221,10 @@ def sdm_scan_forward(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | Non
                      M0=None, init: str = "m0", y=None, gate=None, gamma=None,
                      eps: float = 1e-6, act: str = "silu", o=None, want_o: bool = True,
                      sel_out=None, want_sel: bool = False, engine: str = "auto", ws=None,
-                     stream=None):
+                     stream=None, coupled: bool = False):
     """Prefill over T tokens.  kp, qp [B,T,H,S1+S2]; v, gate [B,T,H,d_v]; alpha, beta
-    [B,T,H]; M [B,H,N,d_v] (in/out); M0 [H,N,d_v] (init="m0").
+    [B,T,H]; M [B,H,N,d_v] (in/out); M0 [H,N,d_v] (init="m0").  coupled=True calls
+    sdm_scan_forward_coupled (the coupled delta rule).
     Returns dict(y, o, sel): sel holds [B,T,H,W] write slots then [B,T,H,R] read slots."""
     dev = kp.device
     shape, y, o, sel_out = _scan_outputs(kp, qp, v, alpha, beta, M, W, R, S1, M0, y, gate,
@@ -228,11 +233,17 @@ def sdm_scan_forward(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | Non
     if ws is None:
         ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
     _need(ws, "ws", torch.uint8, dev)
-    _check(library().sdm_scan_forward(
+    name = "sdm_scan_forward_coupled" if coupled else "sdm_scan_forward"
+    _check(getattr(library(), name)(
         _p(kp), _p(qp), _p(v), _p(alpha), _p(beta), _p(M0), _p(M), INIT[init], _p(y), _p(gate),
         _p(gamma), float(eps), ACT[act], _p(o), _p(sel_out), ENGINE[engine], _p(ws),
-        ws.numel(), shape, _stream(stream, dev)), "sdm_scan_forward")
+        ws.numel(), shape, _stream(stream, dev)), name)
     return dict(y=y, o=o, sel=sel_out)
+
+
+def sdm_scan_forward_coupled(kp, qp, v, alpha, beta, M, **kw):
+    """sdm_scan_forward(..., coupled=True): the token's written rows share one prediction."""
+    return sdm_scan_forward(kp, qp, v, alpha, beta, M, coupled=True, **kw)
 
 
 def sdm_scan_forward_noalloc(kp, qp, v, alpha, beta, M, *, W: int, R: int,
@@ -257,7 +268,7 @@ def sdm_scan_forward_noalloc(kp, qp, v, alpha, beta, M, *, W: int, R: int,
 def sdm_decode_step(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | None = None,
                     y=None, gate=None, gamma=None, eps: float = 1e-6, act: str = "silu", o=None,
                     want_o: bool = True, sel_out=None, want_sel: bool = False, stream=None,
-                    chained: bool = False):
+                    chained: bool = False, coupled: bool = False):
     """One token for each (b, h).  kp, qp [B,H,S1+S2]; v, gate [B,H,d_v]; alpha, beta [B,H];
     M [B,H,N,d_v] in/out.  Returns dict(y, o, sel).  chained=True calls
     sdm_decode_step_chained: only when the kernel launched right before on the stream writes
@@ -291,11 +302,21 @@ def sdm_decode_step(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | None
         o = torch.empty((B, H, d_v), dtype=torch.float32, device=dev)
     if sel_out is None and want_sel:
         sel_out = torch.empty(B * H * (W + R), dtype=torch.int32, device=dev)
-    name = "sdm_decode_step_chained" if chained else "sdm_decode_step"
+    name = "sdm_decode_step" + ("_coupled" if coupled else "") + ("_chained" if chained else "")
     _check(getattr(library(), name)(
         _p(kp), _p(qp), _p(v), _p(alpha), _p(beta), _p(M), _p(y), _p(gate), _p(gamma),
         float(eps), ACT[act], _p(o), _p(sel_out), shape, _stream(stream, dev)), name)
     return dict(y=y, o=o, sel=sel_out)
+
+
+def sdm_decode_step_coupled(kp, qp, v, alpha, beta, M, **kw):
+    """sdm_decode_step(..., coupled=True): one step of the coupled delta rule."""
+    return sdm_decode_step(kp, qp, v, alpha, beta, M, coupled=True, **kw)
+
+
+def sdm_decode_step_coupled_chained(kp, qp, v, alpha, beta, M, **kw):
+    """sdm_decode_step(..., coupled=True, chained=True)."""
+    return sdm_decode_step(kp, qp, v, alpha, beta, M, coupled=True, chained=True, **kw)
 
 
 def sdm_decode_step_chained(kp, qp, v, alpha, beta, M, **kw):

@@ -57,6 +57,7 @@ struct DecLayout {
   // group selection
   uint32_t off_hist, off_ctl, off_list, list_stride, off_clist, clist_stride, off_sorted, off_ev;
   uint32_t off_bits;  // 2048-bit membership filters of the write and the read slots
+  uint32_t off_pred;  // coupled rule: per-warp shares of the prediction [DEC_WARPS][d_v]
   // warp-per-row selection
   uint32_t off_sel, sel_stride;
   // write rows staged over the selection scratch (dead once the selection is done)
@@ -69,7 +70,8 @@ struct DecLayout {
 // Shared-memory plan.  `group` selects the group selection (histograms, control words, four
 // half lists, two candidate lists, the sorted halves, softmax numerators); otherwise two
 // warp selection scratch areas.
-inline DecLayout dec_layout(int S1, int S2, int W, int R, int d_v, bool group) {
+inline DecLayout dec_layout(int S1, int S2, int W, int R, int d_v, bool group,
+                            bool coupled = false) {
   DecLayout L{};
   size_t p = 0;
   auto take = [&p](size_t bytes) {
@@ -85,6 +87,7 @@ inline DecLayout dec_layout(int S1, int S2, int W, int R, int d_v, bool group) {
   L.off_vec = take((2 * (size_t)d_v + 4) * 4);  // v, act(gate), alpha, beta
   L.off_part = take((size_t)DEC_WARPS * d_v * 4);
   L.off_bits = take(2 * 64 * 4);
+  L.off_pred = coupled ? take((size_t)DEC_WARPS * d_v * 4) : 0u;
   const size_t scratch = p;
   if (group) {
     L.off_hist = take(6 * 256 * 4);  // four halves, two candidate sets
@@ -277,7 +280,7 @@ __device__ __forceinline__ void decode_select_group(const DecodeArgs& a, const D
 // E == 0: warp-per-row selection (fp32 halves, halves longer than 1024 scores); otherwise
 // the group selection for bf16 halves of up to 512 E scores and K <= KC.  NQ float4
 // columns per lane: d_v <= 128 NQ.
-template <int E, int KC, int NQ>
+template <int E, int KC, int NQ, bool CP>
 __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, DecLayout L) {
   extern __shared__ __align__(16) unsigned char smem[];
   // the next step may be scheduled at once: its CTAs take the SM slots this step frees, and
@@ -500,8 +503,49 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
   float4 vreg = make_float4(0.f, 0.f, 0.f, 0.f);
   if (kVReg && lane < d4) vreg = reinterpret_cast<const float4*>(vs)[lane];
 
+  // coupled rule (CP): the prediction p = sum_j k_j alpha M[j] over the write rows, shared by
+  // all of them; each warp sums its rows' share, the shares meet in shared memory
+  float4 pred[NQ];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) pred[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if constexpr (CP) {
+    if (rows_smem) {
+      cp_async_wait<0>();  // this warp's write rows (its own lanes' chunks) have landed
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        const int c = lane + 32 * q;
+        float4 pp = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = warp; j < a.W; j += DEC_WARPS) {
+          if (static_cast<unsigned>(idx_w[j]) >= static_cast<unsigned>(a.N) || c >= d4) continue;
+          const float kw = wt_w[j] * al;
+          const float4 o4 = reinterpret_cast<const float4*>(wrow + (size_t)j * a.d_v)[c];
+          pp.x = fmaf(kw, o4.x, pp.x);
+          pp.y = fmaf(kw, o4.y, pp.y);
+          pp.z = fmaf(kw, o4.z, pp.z);
+          pp.w = fmaf(kw, o4.w, pp.w);
+        }
+        if (c < d4) reinterpret_cast<float4*>(smem + L.off_pred + (size_t)warp * a.d_v * 4)[c] = pp;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        const int c = lane + 32 * q;
+        if (c >= d4) continue;
+#pragma unroll
+        for (int w = 0; w < DEC_WARPS; ++w) {
+          const float4 t = reinterpret_cast<const float4*>(smem + L.off_pred + (size_t)w * a.d_v * 4)[c];
+          pred[q].x += t.x;
+          pred[q].y += t.y;
+          pred[q].z += t.z;
+          pred[q].w += t.w;
+        }
+      }
+    }
+  }
+
   // step 2 on one write row whose old value is `old`: store the new row, and add it to the
-  // read sum if the token also reads the slot
+  // read sum if the token also reads the slot.  Per-slot rule: alpha (1 - beta k) M[i] +
+  // beta k v; coupled rule: alpha M[i] + beta k (v - p).
   auto write_row = [&](int j, int sl, const float4 (&old)[NQ]) {
     int rpos = -1;
     const uint32_t us = static_cast<uint32_t>(sl);
@@ -513,13 +557,19 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) decode_kernel(DecodeArgs a, De
     }
     const float qr = rpos >= 0 ? wt_r[rpos] : 0.0f;
     const float kb = be * wt_w[j];
-    const float ka = al * (1.0f - kb);
+    const float ka = CP ? al : al * (1.0f - kb);
     float4* row = reinterpret_cast<float4*>(Mbh + (size_t)sl * a.d_v);
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
       const int c = lane + 32 * q;
       if (c < d4) {
-        const float4 vv = kVReg ? vreg : reinterpret_cast<const float4*>(vs)[c];
+        float4 vv = kVReg ? vreg : reinterpret_cast<const float4*>(vs)[c];
+        if constexpr (CP) {
+          vv.x -= pred[q].x;
+          vv.y -= pred[q].y;
+          vv.z -= pred[q].z;
+          vv.w -= pred[q].w;
+        }
         float4 nw;
         nw.x = fmaf(ka, old[q].x, kb * vv.x);
         nw.y = fmaf(ka, old[q].y, kb * vv.y);

@@ -34,6 +34,7 @@ struct SeqArgs {
   float* M;            // [B*H, N, d_v]
   float* y;            // [B*T*H, d_v]
   int B, T, H, N, W, R, ldw, ldr, d_v, v_bf16;
+  int coupled;  // 1: the coupled delta rule (one prediction shared by the written rows)
 };
 
 constexpr int SEQ_THREADS = 256;
@@ -210,8 +211,76 @@ __global__ void __launch_bounds__(SEQ_THREADS, 1) seq_scan_kernel(SeqArgs a) {
     }
     float* st = stage(u);
 
+    if (a.coupled) {
+      // step 2, coupled reading: pass 1 gathers this thread's old rows (forwarded where a
+      // token of the window wrote them) and its share of the prediction
+      // p = sum_j k_j alpha M[j]; the shares meet through shuffles and shared memory; pass 2
+      // writes alpha M[j] + beta k_j (v - p)
+      constexpr int RPT = (KMAX + NG - 1) / NG;  // write rows per thread
+      float4 olds[RPT];
+      float4 pp = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) {
+        const int j = g + i * NG;
+        olds[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (j >= a.W) continue;
+        const int s = iw[j];
+        if (static_cast<unsigned>(s) >= static_cast<unsigned>(a.N)) continue;
+        float4 old = reinterpret_cast<const float4*>(st + (size_t)j * CW)[lig];
+        if (tok_tab[seq_hash(s)] >= u - D) {
+          int tw, jw;
+          if (find_writer(s, u - 1, u - D, tw, jw))
+            old = reinterpret_cast<const float4*>(stage(tw) + (size_t)jw * CW)[lig];
+        }
+        olds[i] = old;
+        const float kw = ww[j] * al;
+        pp.x = fmaf(kw, old.x, pp.x);
+        pp.y = fmaf(kw, old.y, pp.y);
+        pp.z = fmaf(kw, old.z, pp.z);
+        pp.w = fmaf(kw, old.w, pp.w);
+      }
+#pragma unroll
+      for (int o = LPR; o < 32; o <<= 1) {
+        pp.x += __shfl_xor_sync(FULL_MASK, pp.x, o);
+        pp.y += __shfl_xor_sync(FULL_MASK, pp.y, o);
+        pp.z += __shfl_xor_sync(FULL_MASK, pp.z, o);
+        pp.w += __shfl_xor_sync(FULL_MASK, pp.w, o);
+      }
+      if (lane < LPR) reinterpret_cast<float4*>(red + warp * CW)[lane] = pp;
+      __syncthreads();
+      float4 pr = reinterpret_cast<const float4*>(red)[lig];
+#pragma unroll
+      for (int w = 1; w < NW; ++w) {
+        const float4 t = reinterpret_cast<const float4*>(red + w * CW)[lig];
+        pr.x += t.x;
+        pr.y += t.y;
+        pr.z += t.z;
+        pr.w += t.w;
+      }
+      const float4 dv = make_float4(vv.x - pr.x, vv.y - pr.y, vv.z - pr.z, vv.w - pr.w);
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) {
+        const int j = g + i * NG;
+        if (j >= a.W) continue;
+        const int s = iw[j];
+        if (static_cast<unsigned>(s) >= static_cast<unsigned>(a.N)) {
+          if (lig == 0) record_status(STATUS_BAD_INDEX);
+          continue;
+        }
+        const float kb = be * ww[j];
+        float4 nw;
+        nw.x = fmaf(al, olds[i].x, kb * dv.x);
+        nw.y = fmaf(al, olds[i].y, kb * dv.y);
+        nw.z = fmaf(al, olds[i].z, kb * dv.z);
+        nw.w = fmaf(al, olds[i].w, kb * dv.w);
+        reinterpret_cast<float4*>(st + (size_t)j * CW)[lig] = nw;
+        *reinterpret_cast<float4*>(Mbh + (size_t)s * a.d_v + col0 + 4 * lig) = nw;
+        if (lig == 0) tok_tab[seq_hash(s)] = u;
+      }
+    }
+
     // step 2: gated delta write
-    for (int j = g; j < a.W; j += NG) {
+    for (int j = g; j < a.W && !a.coupled; j += NG) {
       int s = iw[j];
       if (static_cast<unsigned>(s) >= static_cast<unsigned>(a.N)) {
         if (lig == 0) record_status(STATUS_BAD_INDEX);

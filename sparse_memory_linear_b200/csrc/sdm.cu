@@ -121,7 +121,8 @@ sdm_status device_info(DeviceInfo** out) {
     SDM_FAST_ATTR(4, 32) SDM_FAST_ATTR(4, 64) SDM_FAST_ATTR(4, 128)
 #undef SDM_FAST_ATTR
 #define SDM_DEC_ATTR(R8, KC, NQ) \
-  SDM_CUDA_TRY(allow_max_dynamic_smem(decode_kernel<R8, KC, NQ>, m));
+  SDM_CUDA_TRY(allow_max_dynamic_smem(decode_kernel<R8, KC, NQ, false>, m)); \
+  SDM_CUDA_TRY(allow_max_dynamic_smem(decode_kernel<R8, KC, NQ, true>, m));
     SDM_DEC_VARIANTS(SDM_DEC_ATTR)
 #undef SDM_DEC_ATTR
 #define SDM_SEQ_ATTR(CW, D) \
@@ -678,16 +679,19 @@ sdm_status sdm_norm_gate(const float* y, const void* gate, const float* gamma, f
                           static_cast<cudaStream_t>(stream));
 }
 
-sdm_status sdm_scan_forward(const void* kp, const void* qp, const void* v, const float* alpha,
-                            const float* beta, const float* M0, float* M, int32_t init,
-                            float* y, const void* gate, const float* gamma, float eps,
-                            int32_t act, float* o, int32_t* sel_out, int32_t engine, void* ws,
-                            size_t ws_bytes, sdm_shape shape, void* stream) {
-  NvtxRange nvtx_range("sdm_scan_forward");
+// Prefill; `coupled` selects the coupled delta rule (sequential engine only).
+static sdm_status scan_forward(const void* kp, const void* qp, const void* v, const float* alpha,
+                               const float* beta, const float* M0, float* M, int32_t init,
+                               float* y, const void* gate, const float* gamma, float eps,
+                               int32_t act, float* o, int32_t* sel_out, int32_t engine, void* ws,
+                               size_t ws_bytes, sdm_shape shape, void* stream, bool coupled) {
   const sdm_shape& s = shape;
   if (!shape_ok(s, true)) return SDM_ERR_INVALID_ARG;
   if (init != SDM_INIT_FROM_M0 && init != SDM_CONTINUE) return SDM_ERR_INVALID_ARG;
   if (engine < SDM_ENGINE_AUTO || engine > SDM_ENGINE_SLOT) return SDM_ERR_INVALID_ARG;
+  // the slot engine treats every slot as its own recurrence, which the shared prediction of
+  // the coupled rule breaks
+  if (coupled && engine == SDM_ENGINE_SLOT) return SDM_ERR_UNSUPPORTED;
   if (!act_ok(act) || !(eps >= 0.0f)) return SDM_ERR_INVALID_ARG;
   if (!M || !aligned16(M)) return SDM_ERR_INVALID_ARG;
   if (init == SDM_INIT_FROM_M0) {
@@ -711,7 +715,7 @@ sdm_status sdm_scan_forward(const void* kp, const void* qp, const void* v, const
   DeviceInfo* di;
   rc = device_info(&di);
   if (rc != SDM_OK) return rc;
-  engine = pick_engine(s, engine, di->sms);
+  engine = coupled ? SDM_ENGINE_SEQ : pick_engine(s, engine, di->sms);
   if (init == SDM_INIT_FROM_M0) {
     ProfScope ps(SDM_KERNEL_STATE_INIT, st);
     rc = launch_state_init(M0, M, s, st);
@@ -773,6 +777,7 @@ sdm_status sdm_scan_forward(const void* kp, const void* qp, const void* v, const
   a.ldr = WL.ldr;
   a.d_v = s.d_v;
   a.v_bf16 = bf16;
+  a.coupled = coupled ? 1 : 0;
   {
     ProfScope ps(SDM_KERNEL_SCAN_SEQ, st);
     rc = launch_seq(a, st);
@@ -787,11 +792,33 @@ sdm_status sdm_scan_forward(const void* kp, const void* qp, const void* v, const
   return SDM_OK;
 }
 
+sdm_status sdm_scan_forward(const void* kp, const void* qp, const void* v, const float* alpha,
+                            const float* beta, const float* M0, float* M, int32_t init,
+                            float* y, const void* gate, const float* gamma, float eps,
+                            int32_t act, float* o, int32_t* sel_out, int32_t engine, void* ws,
+                            size_t ws_bytes, sdm_shape shape, void* stream) {
+  NvtxRange nvtx_range("sdm_scan_forward");
+  return scan_forward(kp, qp, v, alpha, beta, M0, M, init, y, gate, gamma, eps, act, o,
+                      sel_out, engine, ws, ws_bytes, shape, stream, false);
+}
+
+sdm_status sdm_scan_forward_coupled(const void* kp, const void* qp, const void* v,
+                                    const float* alpha, const float* beta, const float* M0,
+                                    float* M, int32_t init, float* y, const void* gate,
+                                    const float* gamma, float eps, int32_t act, float* o,
+                                    int32_t* sel_out, int32_t engine, void* ws, size_t ws_bytes,
+                                    sdm_shape shape, void* stream) {
+  NvtxRange nvtx_range("sdm_scan_forward_coupled");
+  return scan_forward(kp, qp, v, alpha, beta, M0, M, init, y, gate, gamma, eps, act, o,
+                      sel_out, engine, ws, ws_bytes, shape, stream, true);
+}
+
 // One decode step; `chained` launches it with programmatic stream serialisation.
 static sdm_status decode_step(const void* kp, const void* qp, const void* v, const float* alpha,
                               const float* beta, float* M, float* y, const void* gate,
                               const float* gamma, float eps, int32_t act, float* o,
-                              int32_t* sel_out, sdm_shape shape, void* stream, bool chained) {
+                              int32_t* sel_out, sdm_shape shape, void* stream, bool chained,
+                              bool coupled) {
   NvtxRange nvtx_range("sdm_decode_step");
   sdm_shape s = shape;
   s.T = 1;
@@ -810,8 +837,10 @@ static sdm_status decode_step(const void* kp, const void* qp, const void* v, con
   const int need_nq = (s.d_v / 4 + 31) / 32;
 #define SDM_DEC_FITS(E, KC, NQ) \
   ((fast ? (E >= need_e && E > 0) : E == 0) && KC >= need_kc && NQ >= need_nq)
-  const DecLayout L = dec_layout(s.S1, s.S2, s.W, s.R, s.d_v, fast);
+  const DecLayout L = dec_layout(s.S1, s.S2, s.W, s.R, s.d_v, fast, coupled);
   if (L.total > (size_t)di->max_smem_optin) return SDM_ERR_UNSUPPORTED;
+  // the coupled rule sums the write rows staged in shared memory
+  if (coupled && !L.rows_smem) return SDM_ERR_UNSUPPORTED;
   DecodeArgs a;
   a.kp = kp;
   a.qp = qp;
@@ -851,7 +880,10 @@ static sdm_status decode_step(const void* kp, const void* qp, const void* v, con
   cfg.numAttrs = chained && pdl_enabled() ? 1 : 0;
 #define SDM_DEC_LAUNCH(E, KC, NQ)                                                        \
   if (!launched && SDM_DEC_FITS(E, KC, NQ)) {                                             \
-    SDM_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_kernel<E, KC, NQ>, a, L));              \
+    if (coupled)                                                                          \
+      SDM_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_kernel<E, KC, NQ, true>, a, L));      \
+    else                                                                                  \
+      SDM_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_kernel<E, KC, NQ, false>, a, L));     \
     g_launches.fetch_add(1, std::memory_order_relaxed);                                   \
     launched = true;                                                                      \
   }
@@ -868,7 +900,7 @@ sdm_status sdm_decode_step(const void* kp, const void* qp, const void* v, const 
                            const float* gamma, float eps, int32_t act, float* o,
                            int32_t* sel_out, sdm_shape shape, void* stream) {
   return decode_step(kp, qp, v, alpha, beta, M, y, gate, gamma, eps, act, o, sel_out, shape,
-                     stream, false);
+                     stream, false, false);
 }
 
 sdm_status sdm_decode_step_chained(const void* kp, const void* qp, const void* v,
@@ -876,7 +908,24 @@ sdm_status sdm_decode_step_chained(const void* kp, const void* qp, const void* v
                                    const void* gate, const float* gamma, float eps, int32_t act,
                                    float* o, int32_t* sel_out, sdm_shape shape, void* stream) {
   return decode_step(kp, qp, v, alpha, beta, M, y, gate, gamma, eps, act, o, sel_out, shape,
-                     stream, true);
+                     stream, true, false);
+}
+
+sdm_status sdm_decode_step_coupled(const void* kp, const void* qp, const void* v,
+                                   const float* alpha, const float* beta, float* M, float* y,
+                                   const void* gate, const float* gamma, float eps, int32_t act,
+                                   float* o, int32_t* sel_out, sdm_shape shape, void* stream) {
+  return decode_step(kp, qp, v, alpha, beta, M, y, gate, gamma, eps, act, o, sel_out, shape,
+                     stream, false, true);
+}
+
+sdm_status sdm_decode_step_coupled_chained(const void* kp, const void* qp, const void* v,
+                                           const float* alpha, const float* beta, float* M,
+                                           float* y, const void* gate, const float* gamma,
+                                           float eps, int32_t act, float* o, int32_t* sel_out,
+                                           sdm_shape shape, void* stream) {
+  return decode_step(kp, qp, v, alpha, beta, M, y, gate, gamma, eps, act, o, sel_out, shape,
+                     stream, true, true);
 }
 
 sdm_status sdm_get_device_status(void* stream) {

@@ -221,6 +221,18 @@ def test_options_are_explicit_and_validated(sdm):
         assert "getenv" not in open(os.path.join(csrc, f)).read(), f"{f} reads the environment"
 
 
+@host_only
+def test_coupled_prefill_refuses_the_slot_engine_before_any_launch(sdm):
+    lib = sdm.library()
+    P = ctypes.c_void_p
+    with no_launch(sdm):
+        rc = lib.sdm_scan_forward_coupled(P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE),
+                                          P(FAKE + 0x100000000), P(FAKE), 0, P(FAKE), None,
+                                          None, 1e-6, 0, None, None, 2, P(FAKE), 1 << 40,
+                                          good_shape(sdm), None)
+    assert rc == 2  # SDM_ERR_UNSUPPORTED
+
+
 def test_status_strings(sdm):
     assert sdm.sdm_status_string(0) == "SDM_OK"
     assert sdm.sdm_status_string(4) == "SDM_ERR_DEVICE_CHECK"

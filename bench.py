@@ -445,6 +445,67 @@ def bench_balance(args, dev):
             "busy_us_per_cta": q(active[:, 3] / 8.0 / 1e3)}
 
 
+def bench_coupled(args, dist: Dist, dev):
+    """The coupled delta rule: prefill of the 1.4B-like workload (sequential engine, the one
+    that computes it) and 256 chained decode steps of the batched-decode workload, timed as
+    the per-slot lines are."""
+    import sparse_memory_linear_b200 as sdm
+
+    stream = torch.cuda.current_stream(dev)
+    peak, peak_kind = hbm_peak()
+    wl = sdm_synth.WORKLOADS["layer1p4b"]
+    g = {k: v.to(dev) for k, v in sdm_synth.make_inputs(wl, device=dev).items()}
+    M = torch.empty((wl.B, wl.H, wl.N, wl.d_v), dtype=torch.float32, device=dev)
+    sdm.sdm_state_init(g["M0"], M)
+    y = torch.empty((wl.B, wl.T, wl.H, wl.d_v), dtype=torch.float32, device=dev)
+    o = torch.empty_like(y)
+
+    def step():
+        sdm.sdm_scan_forward_coupled(g["kp"], g["qp"], g["v"], g["alpha"], g["beta"], M,
+                                     W=wl.W, R=wl.R, S1=wl.S1, init="continue", gate=g["gate"],
+                                     y=y, o=o, stream=stream)
+
+    steps = max(3, args.steps)
+    secs = timed(step, steps, args.warmup, dist, stream)
+    th = wl.B * wl.T * wl.H
+    step_s = secs / steps
+    pre = {"workload": wl.name, "shape": wl.note, "engine": "seq",
+           "value": weak_scaling_value(th, step_s, dist.world), "unit": UNIT,
+           "ms_per_step": step_s * 1e3,
+           "whole_step_hbm_frac": th * algorithmic_bytes(wl) / step_s / 1e9 / peak}
+    del g, M, y, o
+    torch.cuda.empty_cache()
+
+    wl = sdm_synth.WORKLOADS[args.decode_workload]
+    steps_in = [{k: t.to(dev) for k, t in sdm_synth.make_inputs(wl, device=dev, step=s).items()}
+                for s in range(wl.T)]
+    M0 = steps_in[0].pop("M0")
+    M = torch.empty((wl.B, wl.H, wl.N, wl.d_v), dtype=torch.float32, device=dev)
+    sdm.sdm_state_init(M0, M)
+    yd = torch.empty((wl.B, wl.H, wl.d_v), dtype=torch.float32, device=dev)
+    od = torch.empty_like(yd)
+
+    def run_all():
+        for s in steps_in:
+            sdm.sdm_decode_step(s["kp"], s["qp"], s["v"], s["alpha"], s["beta"], M, W=wl.W,
+                                R=wl.R, S1=wl.S1, gate=s["gate"], y=yd, o=od, stream=stream,
+                                chained=True, coupled=True)
+
+    reps = max(1, args.steps // 2)
+    secs = timed(run_all, reps, 1, dist, stream)
+    per_step = secs / (reps * wl.T)
+    dec = {"workload": wl.note, "launch": "sdm_decode_step_coupled_chained",
+           "us_per_step": per_step * 1e6, "value": weak_scaling_value(wl.B * wl.H, per_step,
+                                                                       dist.world),
+           "unit": UNIT, "step_roofline_frac": step_bytes_of(wl) / per_step / 1e9 / peak}
+    if sdm.sdm_get_device_status() != 0:
+        raise RuntimeError("device status word set during the coupled benchmark")
+    del M, steps_in
+    torch.cuda.empty_cache()
+    return {"rule": "coupled delta (one prediction shared by the written rows)",
+            "prefill": pre, "decode": dec, "peak_kind": peak_kind}
+
+
 def step_bytes_of(wl) -> float:
     """Algorithmic bytes of one decode step of every (sequence, head)."""
     return wl.B * wl.H * algorithmic_bytes(wl)
@@ -703,6 +764,8 @@ def main(argv=None):
             line["prefill_configs"] = bench_prefill_configs(args, dist, dev)
         if not args.no_decode:
             line["decode"] = bench_decode(args, dist, dev)
+        if not args.no_configs and args.only is None:
+            line["coupled"] = bench_coupled(args, dist, dev)
         if dist.rank == 0:
             print(json.dumps(line), flush=True)
         return 0

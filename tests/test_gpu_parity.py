@@ -437,3 +437,14 @@ def test_slot_engine_cta_stats_account_for_every_event(sdm):
     assert st[:, 1].sum() > 0 and st[:, 2].sum() > 0 and st[:, 3].sum() > 0
     run_scan(sdm, wl, g, engine="slot", want_o=False)
     assert int(sdm.sdm_slot_cta_stats(reset=True).sum()) == 0
+
+
+def test_scan_slot_engine_over_several_chunks(sdm):
+    """Many wide (sequence, head) rows per token make the slot engine's time chunks short
+    (here 128 tokens), so the state carries over between chunks three times; the result is
+    the oracle's all the same."""
+    wl = sdm_synth.WORKLOADS["tiny"].replace(B=8, H=8, T=300, S1=16, S2=16, W=8, R=8,
+                                            d_v=1024, in_dtype=BF16, seed=61)
+    g = device_inputs(wl)
+    out, M = run_scan(sdm, wl, g, engine="slot")
+    full_check(wl, g, out, M)

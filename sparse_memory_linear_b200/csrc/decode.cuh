@@ -11,7 +11,7 @@
 //   the halves' exponents span more than 15, the first of the four checks the ties at the
 //   K-th sum against all K*K pairs, as select.cuh describes).
 //   Other shapes: warps 0 and 1 run the warp-per-row selection of select.cuh.
-//   CTAs 0 .. 63 also prefetch into L2 the inputs of the CTAs dispatched after them;
+//   CTAs 0 .. 127 also prefetch into L2 the inputs of the CTAs dispatched after them;
 //   steps 2 and 3 issue every row load of the token at once: each warp's write rows go to
 //   shared memory (over the dead selection scratch) by cp.async and its first read rows to
 //   registers, so the step waits for one memory latency;
@@ -110,9 +110,9 @@ inline DecLayout dec_layout(int S1, int S2, int W, int R, int d_v, bool group,
   return L;
 }
 
-// CTAs 0 .. DEC_PF_CTAS - 1 are dispatched first and prefetch for the others (a 64 x 8
-// batch at 4 CTAs per SM leaves 80 of the 592 slots free for the next step's first CTAs).
-constexpr int DEC_PF_CTAS = 64;
+// CTAs 0 .. DEC_PF_CTAS - 1 are dispatched first and prefetch for the others.  Measured on
+// a 64 x 8 batch (us per chained step): none 17.2, 32 CTAs 16.3, 64 16.5, 128 15.7.
+constexpr int DEC_PF_CTAS = 128;
 
 // L2 prefetch of the 128-byte lines of [p, p + bytes) by the lanes of one warp; every
 // address prefetched lies inside the span.
@@ -171,6 +171,16 @@ __device__ __forceinline__ void decode_select_group(const DecodeArgs& a, const D
   const int g = warp >> 1, gt = tid & 63;
   const int s = g >> 1, st = tid & 127;
   const int K = s ? a.R : a.W;
+  // this thread's rank pairs of the candidate table, loaded before the half selections so
+  // that the loads are long done when the candidates need them (read late, these loads of a
+  // table every CTA shares sat on the critical path, by up to 6 % of the step)
+  uint32_t tpre[CPT];
+  {
+    const uint16_t* tp = cand_table(K);
+    const int Cp = s ? L.C_r : L.C_w;
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) tpre[j] = st + 128 * j < Cp ? __ldg(tp + st + 128 * j) : 0u;
+  }
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L.off_hist);
   GroupCtl* ctl = reinterpret_cast<GroupCtl*>(smem + L.off_ctl);
   uint32_t* sorted = reinterpret_cast<uint32_t*>(smem + L.off_sorted);
@@ -203,7 +213,6 @@ __device__ __forceinline__ void decode_select_group(const DecodeArgs& a, const D
   // candidates of selection s
   const uint32_t* A = sorted + KMAX * (2 * s);
   const uint32_t* B = sorted + KMAX * (2 * s + 1);
-  const uint16_t* tab = cand_table(K);
   const int C = s ? L.C_r : L.C_w;
   uint32_t ck[CPT], cf[CPT];
 #pragma unroll
@@ -212,7 +221,7 @@ __device__ __forceinline__ void decode_select_group(const DecodeArgs& a, const D
     ck[j] = 0u;
     cf[j] = 0u;
     if (c < C) {
-      const int e = __ldg(tab + c);
+      const int e = static_cast<int>(tpre[j]);
       const uint32_t ca = A[e >> 7], cb = B[e & 127];
       ck[j] = score_key(__fadd_rn(key16_value(ca >> 16), key16_value(cb >> 16)));
       cf[j] = (0xffffu - (ca & 0xffffu)) * static_cast<uint32_t>(a.S2) + (0xffffu - (cb & 0xffffu));

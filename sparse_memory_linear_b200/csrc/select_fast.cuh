@@ -337,7 +337,7 @@ __device__ __forceinline__ void cand_topk_bf16(const uint32_t* A, const uint32_t
     ck[q] = 0u;  // no candidate (every real score has a key >= 1)
     cf[q] = 0u;
     if (c < C) {
-      const int e = __ldg(ctab + c);
+      const int e = ctab[c];
       const int r1 = e >> 7, r2 = e & 127;
       const float s = __fadd_rn(av[r1], bv[r2]);
       orbits |= __float_as_uint(s) & 0x7fffffffu;
@@ -476,9 +476,17 @@ __global__ void __launch_bounds__(256, 4) sel_fast_kernel(SelJob job0, SelJob jo
   grid_dependency_wait();
   grid_launch_dependents();
   extern __shared__ __align__(16) unsigned char smem[];
+  // the jobs' candidate tables, copied once per CTA: every row of a job reads the same one
+  __shared__ uint16_t ctab_s[2][cand_count(KC)];
+  const int K1 = njobs > 1 ? job1.K : job0.K;
+  for (int i = threadIdx.x; i < cand_count_dev(job0.K); i += blockDim.x)
+    ctab_s[0][i] = cand_table(job0.K)[i];
+  for (int i = threadIdx.x; i < cand_count_dev(K1); i += blockDim.x)
+    ctab_s[1][i] = cand_table(K1)[i];
+  __syncthreads();
   unsigned char* scratch_base = smem;
-  const uint16_t* tab0 = cand_table(job0.K);
-  const uint16_t* tab1 = cand_table(njobs > 1 ? job1.K : job0.K);
+  const uint16_t* tab0 = ctab_s[0];
+  const uint16_t* tab1 = ctab_s[1];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wpc = blockDim.x >> 5;
   FastScratch sc = carve_fast_scratch(scratch_base + (size_t)warp * fast_scratch_bytes(S1, S2, KC),

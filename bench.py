@@ -285,6 +285,10 @@ def bench_prefill(args, dist: Dist, dev):
         "kernels_ms_per_step": ms_step,
         "kernel_launches_per_step": n_step,
         "kernels_share": {k: ms_step[k] / sum(ms_step.values()) for k in ms_step},
+        "select_schedule": ("library default: with more than one time chunk, chunk c+1's "
+                            "selection runs on a low-priority stream beside chunk c's sort and "
+                            "scan, so the per-kernel times overlap and add up to more than the "
+                            "step"),
         "gpu_launches": int(launched),
         "roofline": {
             "kernel": f"seq_scan_kernel" if scan_kind == "scan_seq" else "slot_chunk_kernel",

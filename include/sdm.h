@@ -266,8 +266,16 @@ typedef enum {
                                        slice (0: chosen by shape)                       */
     SDM_OPT_SEQ_DEPTH = 6,          /* 4 or 8: the sequential engine's gather-ahead
                                        depth in tokens (0: chosen by slice)             */
-    SDM_OPT_SLOT_CTA_STATS = 7      /* 1: the slot engine records per-CTA work
+    SDM_OPT_SLOT_CTA_STATS = 7,     /* 1: the slot engine records per-CTA work
                                        (sdm_slot_cta_stats)                             */
+    SDM_OPT_SELECT_SCHEDULE = 8     /* the slot engine's selection, when T spans more
+                                       than one time chunk: 1 the whole selection first,
+                                       2 pipelined (chunk c + 1's selection on an
+                                       internal low-priority stream beside chunk c's
+                                       work on an internal high-priority one, joined
+                                       back to the caller's stream), 0 the library's
+                                       default; every schedule gives the same
+                                       selections and state                             */
 } sdm_option;
 
 /* Sets an option.  SDM_ERR_INVALID_ARG (and no change) for an unknown option or a value

@@ -364,7 +364,7 @@ def sdm_profile_read() -> dict:
 
 
 OPTION = {"no_pdl": 1, "select_general": 2, "select_ctas_per_sm": 3, "slot_ctas_per_sm": 4,
-          "seq_columns": 5, "seq_depth": 6, "slot_cta_stats": 7}
+          "seq_columns": 5, "seq_depth": 6, "slot_cta_stats": 7, "select_schedule": 8}
 SLOT_STATS_CTAS = 1024
 
 

@@ -49,7 +49,7 @@ struct NvtxRange {
 };
 
 // Process-wide launch options (sdm_option); 0 everywhere by default.
-constexpr int OPT_SLOTS = 8;
+constexpr int OPT_SLOTS = 16;
 std::atomic<int> g_opt[OPT_SLOTS];
 
 inline int opt(int which) { return g_opt[which].load(std::memory_order_relaxed); }
@@ -311,9 +311,22 @@ int pick_engine(const sdm_shape& s, int requested, int sms) {
   return engine;
 }
 
+// Grid of a selection launch over `total_rows` rows: one persistent wave at `per_sm` CTAs per
+// SM, or, with rows_per_warp > 0, short-lived CTAs whose warps take that many rows each (the
+// chunk-pipelined prefill, where the scan's CTAs take the SM slots that they free).
+long long select_grid(long long total_rows, int warps, int per_sm, int rows_per_warp,
+                      const DeviceInfo* di) {
+  const long long need = (total_rows + warps - 1) / warps;
+  if (rows_per_warp > 0) return (need + rows_per_warp - 1) / rows_per_warp;
+  const int cap = opt(SDM_OPT_SELECT_CTAS_PER_SM);
+  if (cap > 0 && cap < per_sm) per_sm = cap;
+  const long long grid = (long long)di->sms * per_sm;
+  return grid > need ? need : grid;
+}
+
 template <int R8, int KC>
 sdm_status launch_select_fast_t(const SelJob& j0, const SelJob* j1, long long rows, int S1, int S2,
-                                const DeviceInfo* di, cudaStream_t st) {
+                                int rows_per_warp, const DeviceInfo* di, cudaStream_t st) {
   const int K1 = j1 ? j1->K : j0.K;
   int warps = 8;
   size_t smem = sel_fast_smem_bytes(S1, S2, j0.K, K1, warps);
@@ -323,11 +336,7 @@ sdm_status launch_select_fast_t(const SelJob& j0, const SelJob* j1, long long ro
                                                              warps * 32, smem));
   if (per_sm < 1) return SDM_ERR_UNSUPPORTED;
   const long long total_rows = rows * (j1 ? 2 : 1);
-  const int cap = opt(SDM_OPT_SELECT_CTAS_PER_SM);
-  if (cap > 0 && cap < per_sm) per_sm = cap;
-  long long grid = (long long)di->sms * per_sm;
-  const long long need = (total_rows + warps - 1) / warps;
-  if (grid > need) grid = need;
+  const long long grid = select_grid(total_rows, warps, per_sm, rows_per_warp, di);
   SDM_CUDA_TRY(launch_pdl(sel_fast_kernel<R8, KC>, dim3((unsigned)grid), dim3(warps * 32), smem, st,
                           j0, j1 ? *j1 : j0, rows, j1 ? 2 : 1, S1, S2));
   g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -336,12 +345,13 @@ sdm_status launch_select_fast_t(const SelJob& j0, const SelJob* j1, long long ro
 }
 
 sdm_status launch_select_fast(const SelJob& j0, const SelJob* j1, long long rows, int S1, int S2,
-                              const DeviceInfo* di, cudaStream_t st) {
+                              int rows_per_warp, const DeviceInfo* di, cudaStream_t st) {
   const int K1 = j1 ? j1->K : j0.K;
   const int r8 = fast_r8(S1, S2);
   const int kc = fast_kc(j0.K > K1 ? j0.K : K1);
 #define SDM_FAST_CASE(R8, KC) \
-  if (r8 == R8 && kc == KC) return launch_select_fast_t<R8, KC>(j0, j1, rows, S1, S2, di, st);
+  if (r8 == R8 && kc == KC)      \
+    return launch_select_fast_t<R8, KC>(j0, j1, rows, S1, S2, rows_per_warp, di, st);
   SDM_FAST_CASE(1, 32) SDM_FAST_CASE(1, 64) SDM_FAST_CASE(1, 128)
   SDM_FAST_CASE(2, 32) SDM_FAST_CASE(2, 64) SDM_FAST_CASE(2, 128)
   SDM_FAST_CASE(4, 32) SDM_FAST_CASE(4, 64) SDM_FAST_CASE(4, 128)
@@ -349,9 +359,9 @@ sdm_status launch_select_fast(const SelJob& j0, const SelJob* j1, long long rows
   return SDM_ERR_UNSUPPORTED;
 }
 
-// Selection of one or two jobs over `rows` score rows.
+// Selection of one or two jobs over `rows` score rows (grid: select_grid).
 sdm_status launch_select(const SelJob& j0, const SelJob* j1, long long rows, int S1, int S2,
-                         int bf16, cudaStream_t st) {
+                         int bf16, cudaStream_t st, int rows_per_warp = 0) {
   DeviceInfo* di;
   sdm_status rc = device_info(&di);
   if (rc != SDM_OK) return rc;
@@ -359,7 +369,7 @@ sdm_status launch_select(const SelJob& j0, const SelJob* j1, long long rows, int
   const int K1 = j1 ? j1->K : j0.K;
   const int kmax_all = j0.K > K1 ? j0.K : K1;
   if (fast_select_ok(bf16, S1, S2, kmax_all) && opt(SDM_OPT_SELECT_GENERAL) == 0)
-    return launch_select_fast(j0, j1, rows, S1, S2, di, st);
+    return launch_select_fast(j0, j1, rows, S1, S2, rows_per_warp, di, st);
   int warps = 8;
   size_t smem = sel_smem_bytes(S1, S2, j0.K, K1, warps);
   while (warps > 1 && smem > (size_t)di->max_smem_optin / 2) {
@@ -371,11 +381,7 @@ sdm_status launch_select(const SelJob& j0, const SelJob* j1, long long rows, int
   SDM_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sel_kernel, warps * 32, smem));
   if (per_sm < 1) return SDM_ERR_UNSUPPORTED;
   const long long total_rows = rows * (j1 ? 2 : 1);
-  const int cap = opt(SDM_OPT_SELECT_CTAS_PER_SM);
-  if (cap > 0 && cap < per_sm) per_sm = cap;
-  long long grid = (long long)di->sms * per_sm;
-  const long long need = (total_rows + warps - 1) / warps;
-  if (grid > need) grid = need;
+  const long long grid = select_grid(total_rows, warps, per_sm, rows_per_warp, di);
   const int kmax = j0.K > K1 ? j0.K : K1;
   SDM_CUDA_TRY(launch_pdl(sel_kernel, dim3((unsigned)grid), dim3(warps * 32), smem, st,
                           j0, j1 ? *j1 : j0, rows, j1 ? 2 : 1, S1, S2, bf16, kmax));
@@ -484,12 +490,12 @@ sdm_status launch_slot_chunk(const SlotArgs& a, const DeviceInfo* di, cudaStream
   return SDM_OK;
 }
 
-// Steps 2-3 with the slot-parallel engine, one time chunk after another: the chunk's
-// events, their radix sort by (sequence, head, slot), its long segments, then the chunk's
-// segments.  A chunk's events and sort buffers (tens of MB) stay in L2 between the steps.
-sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
-                       const float* alpha, const float* beta, const void* v, float* M, float* y,
-                       const DeviceInfo* di, cudaStream_t st) {
+// One time chunk [t0, t0 + ct) of the slot engine on `st`: the chunk's events, their radix
+// sort by (sequence, head, slot), its long segments, then the chunk's segments.  The chunk's
+// selections must be complete in the workspace (stream order, or an event `st` waits on).
+sdm_status launch_slot_chunk_work(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
+                                  const SlotArgs& a, int t0, const DeviceInfo* di,
+                                  cudaStream_t st) {
   uint32_t* k0 = reinterpret_cast<uint32_t*>(w + WL.off_k0);
   uint32_t* k1 = reinterpret_cast<uint32_t*>(w + WL.off_k1);
   uint2* v0 = reinterpret_cast<uint2*>(w + WL.off_v0);
@@ -497,31 +503,110 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
   uint32_t* hist = reinterpret_cast<uint32_t*>(w + WL.off_hist);
   uint32_t* tot = reinterpret_cast<uint32_t*>(w + WL.off_tot);
   uint32_t* offs = reinterpret_cast<uint32_t*>(w + WL.off_offs);
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(w + WL.off_cnt);  // hot count | span queue
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(w + WL.off_cnt);
   uint2* hot = reinterpret_cast<uint2*>(w + WL.off_hot);
-  const int N = s.S1 * s.S2;
+  float* y = a.y;
+  const int N = a.N;
   const int bits = WL.kb.total();
-  // an even number of passes leaves the sorted events in k0 / v0
-  const int passes = (bits + 7) / 8;
-  uint32_t* ks = passes % 2 ? k1 : k0;
-  uint2* vs = passes % 2 ? v1 : v0;
-  SlotArgs a;
-  a.keys = ks;
-  a.vals = vs;
-  a.offs = offs;
+  const uint32_t* ks = a.keys;
+  const int d4 = s.d_v / 4;
+  const int ct = s.T - t0 < WL.chunk ? s.T - t0 : WL.chunk;
+  const long long E = (long long)ct * s.B * s.H * (s.W + s.R);
+  const int ntiles = (int)((E + RS_TILE - 1) / RS_TILE);
+  {
+    ProfScope ps(SDM_KERNEL_SLOT_SORT, st);
+    EventArgs ea;
+    ea.idx_w = reinterpret_cast<const int32_t*>(w + WL.off_idx_w);
+    ea.wt_w = reinterpret_cast<const float*>(w + WL.off_wt_w);
+    ea.idx_r = reinterpret_cast<const int32_t*>(w + WL.off_idx_r);
+    ea.wt_r = reinterpret_cast<const float*>(w + WL.off_wt_r);
+    ea.keys = k0;
+    ea.vals = v0;
+    ea.y = y;
+    ea.offs = offs;
+    ea.counters = cnt;
+    ea.B = s.B;
+    ea.T = s.T;
+    ea.H = s.H;
+    ea.N = N;
+    ea.W = s.W;
+    ea.R = s.R;
+    ea.ldw = WL.ldw;
+    ea.ldr = WL.ldr;
+    ea.d_v = s.d_v;
+    ea.t0 = t0;
+    ea.ct = ct;
+    ea.kb = WL.kb;
+    const long long crow = (long long)ct * s.B * s.H;
+    long long blocks = (crow + 7) / 8;  // a warp per chunk row
+    if (blocks > (long long)di->sms * 16) blocks = (long long)di->sms * 16;
+    SDM_CUDA_TRY(launch_pdl(slot_events_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
+                            ea));
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    SDM_CUDA_TRY(cudaGetLastError());
+    // LSD radix sort over the key bits in use
+    uint32_t* ka = k0;
+    uint32_t* kb = k1;
+    uint2* va = v0;
+    uint2* vb = v1;
+    for (int shift = 0; shift < bits; shift += 8) {
+      SDM_CUDA_TRY(launch_pdl<true>(radix_hist_kernel, dim3(ntiles), dim3(RS_THREADS), 0, st,
+                              ka, E, shift, hist, ntiles));
+      SDM_CUDA_TRY(launch_pdl<true>(radix_scan_kernel, dim3(RS_BINS), dim3(1024), 0, st,
+                              hist, ntiles, tot));
+      SDM_CUDA_TRY(launch_pdl<true>(radix_scatter_kernel, dim3(ntiles), dim3(RS_THREADS), RS_SCATTER_SMEM, st,
+                              ka, va, kb, vb, E, shift, hist, tot, ntiles));
+      g_launches.fetch_add(3, std::memory_order_relaxed);
+      SDM_CUDA_TRY(cudaGetLastError());
+      uint32_t* tk = ka;
+      ka = kb;
+      kb = tk;
+      uint2* tv = va;
+      va = vb;
+      vb = tv;
+    }
+    const long long nsamp = (E + 127) / 128;
+    long long lblocks = (nsamp + 255) / 256;
+    if (lblocks > (long long)di->sms * 8) lblocks = (long long)di->sms * 8;
+    if (lblocks < 1) lblocks = 1;
+    SDM_CUDA_TRY(launch_pdl<true>(slot_long_segments_kernel, dim3((unsigned)lblocks), dim3(256), 0, st,
+                            ks, E, cnt, hot, WL.hot_cap));
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    SDM_CUDA_TRY(cudaGetLastError());
+  }
+  ProfScope ps(SDM_KERNEL_SCAN_SLOT, st);
+  sdm_status rc;
+  if (d4 <= 32) rc = launch_slot_chunk<1, 4, 6>(a, di, st);
+  else if (d4 <= 64) rc = launch_slot_chunk<2, 2, 6>(a, di, st);
+  else if (d4 <= 128) rc = launch_slot_chunk<4, 4, 4>(a, di, st);
+  else rc = launch_slot_chunk<8, 2, 2>(a, di, st);
+  return rc;
+}
+
+// The slot engine's arguments for one call: sorted events in k0 / v0 after an even number of
+// radix passes, else in k1 / v1.
+sdm_status make_slot_args(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
+                          const float* alpha, const float* beta, const void* v, float* M,
+                          float* y, SlotArgs* out) {
+  const int passes = (WL.kb.total() + 7) / 8;
+  SlotArgs& a = *out;
+  a.keys = reinterpret_cast<uint32_t*>(w + (passes % 2 ? WL.off_k1 : WL.off_k0));
+  a.vals = reinterpret_cast<uint2*>(w + (passes % 2 ? WL.off_v1 : WL.off_v0));
+  a.offs = reinterpret_cast<uint32_t*>(w + WL.off_offs);
   a.alpha = alpha;
   a.beta = beta;
   a.v = v;
   a.M = M;
   a.y = y;
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(w + WL.off_cnt);  // hot count | span queue
   a.hot_count = cnt;
-  a.hot_list = hot;
+  a.hot_list = reinterpret_cast<uint2*>(w + WL.off_hot);
   a.span_next = cnt + 1;
   a.hot_cap = WL.hot_cap;
   a.B = s.B;
   a.T = s.T;
   a.H = s.H;
-  a.N = N;
+  a.N = s.S1 * s.S2;
   a.d_v = s.d_v;
   a.v_bf16 = s.in_dtype == SDM_BF16;
   a.kb = WL.kb;
@@ -531,80 +616,118 @@ sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
     SDM_CUDA_TRY(cudaGetSymbolAddress(&p, g_slot_cta_stats));
     a.cta_stats = static_cast<unsigned long long*>(p);
   }
-  const int d4 = s.d_v / 4;
-  for (int t0 = 0; t0 < s.T; t0 += WL.chunk) {
-    const int ct = s.T - t0 < WL.chunk ? s.T - t0 : WL.chunk;
-    const long long E = (long long)ct * s.B * s.H * (s.W + s.R);
-    const int ntiles = (int)((E + RS_TILE - 1) / RS_TILE);
-    {
-      ProfScope ps(SDM_KERNEL_SLOT_SORT, st);
-      EventArgs ea;
-      ea.idx_w = reinterpret_cast<const int32_t*>(w + WL.off_idx_w);
-      ea.wt_w = reinterpret_cast<const float*>(w + WL.off_wt_w);
-      ea.idx_r = reinterpret_cast<const int32_t*>(w + WL.off_idx_r);
-      ea.wt_r = reinterpret_cast<const float*>(w + WL.off_wt_r);
-      ea.keys = k0;
-      ea.vals = v0;
-      ea.y = y;
-      ea.offs = offs;
-      ea.counters = cnt;
-      ea.B = s.B;
-      ea.T = s.T;
-      ea.H = s.H;
-      ea.N = N;
-      ea.W = s.W;
-      ea.R = s.R;
-      ea.ldw = WL.ldw;
-      ea.ldr = WL.ldr;
-      ea.d_v = s.d_v;
-      ea.t0 = t0;
-      ea.ct = ct;
-      ea.kb = WL.kb;
-      const long long crow = (long long)ct * s.B * s.H;
-      long long blocks = (crow + 7) / 8;  // a warp per chunk row
-      if (blocks > (long long)di->sms * 16) blocks = (long long)di->sms * 16;
-      SDM_CUDA_TRY(launch_pdl(slot_events_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
-                              ea));
-      g_launches.fetch_add(1, std::memory_order_relaxed);
-      SDM_CUDA_TRY(cudaGetLastError());
-      // LSD radix sort over the key bits in use
-      uint32_t* ka = k0;
-      uint32_t* kb = k1;
-      uint2* va = v0;
-      uint2* vb = v1;
-      for (int shift = 0; shift < bits; shift += 8) {
-        SDM_CUDA_TRY(launch_pdl<true>(radix_hist_kernel, dim3(ntiles), dim3(RS_THREADS), 0, st,
-                                ka, E, shift, hist, ntiles));
-        SDM_CUDA_TRY(launch_pdl<true>(radix_scan_kernel, dim3(RS_BINS), dim3(1024), 0, st,
-                                hist, ntiles, tot));
-        SDM_CUDA_TRY(launch_pdl<true>(radix_scatter_kernel, dim3(ntiles), dim3(RS_THREADS), RS_SCATTER_SMEM, st,
-                                ka, va, kb, vb, E, shift, hist, tot, ntiles));
-        g_launches.fetch_add(3, std::memory_order_relaxed);
-        SDM_CUDA_TRY(cudaGetLastError());
-        uint32_t* tk = ka;
-        ka = kb;
-        kb = tk;
-        uint2* tv = va;
-        va = vb;
-        vb = tv;
-      }
-      const long long nsamp = (E + 127) / 128;
-      long long lblocks = (nsamp + 255) / 256;
-      if (lblocks > (long long)di->sms * 8) lblocks = (long long)di->sms * 8;
-      if (lblocks < 1) lblocks = 1;
-      SDM_CUDA_TRY(launch_pdl<true>(slot_long_segments_kernel, dim3((unsigned)lblocks), dim3(256), 0, st,
-                              ks, E, cnt, hot, WL.hot_cap));
-      g_launches.fetch_add(1, std::memory_order_relaxed);
-      SDM_CUDA_TRY(cudaGetLastError());
+  return SDM_OK;
+}
+
+// Steps 2-3 with the slot-parallel engine, one time chunk after another on `st`, after the
+// whole selection.  A chunk's events and sort buffers (tens of MB) stay in L2 between the
+// steps.
+sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
+                       const float* alpha, const float* beta, const void* v, float* M, float* y,
+                       const DeviceInfo* di, cudaStream_t st) {
+  SlotArgs a;
+  sdm_status rc = make_slot_args(s, WL, w, alpha, beta, v, M, y, &a);
+  for (int t0 = 0; rc == SDM_OK && t0 < s.T; t0 += WL.chunk)
+    rc = launch_slot_chunk_work(s, WL, w, a, t0, di, st);
+  return rc;
+}
+
+// Whether SDM_OPT_SELECT_SCHEDULE = 0 pipelines the slot engine's selection with its chunks.
+// Long skewed step (32 chunks), ms: whole selection first 52.9, pipelined 46.6.
+constexpr bool PIPELINE_BY_DEFAULT = true;
+
+// Rows per warp of a chunk's selection launch in the pipelined schedule: CTAs that live one
+// selection per warp, so that the scan's CTAs (on the higher-priority stream) take the SM
+// slots they free.  Long skewed step, ms: 1 row 46.6, 2 rows 47.7, 8 rows 49.4, one
+// persistent wave 48.8; 2 rows with both streams at the same priority 50.2.
+constexpr int PIPE_SEL_ROWS_PER_WARP = 1;
+
+// Streams and events of one device for the pipelined slot engine: chunk work on `hi`
+// (greatest priority), selections on `lo` (least priority).  Created on first use; the
+// mutex serialises the enqueueing of pipelined calls, whose event ring it protects.
+struct PipeStreams {
+  bool ready = false;
+  cudaStream_t hi = nullptr, lo = nullptr;
+  cudaEvent_t fork = nullptr, done = nullptr, sel[2] = {nullptr, nullptr};
+};
+std::mutex g_pipe_mu;
+PipeStreams g_pipe[MAX_DEVICES];
+
+sdm_status pipe_streams(PipeStreams** out) {
+  int dev = 0;
+  SDM_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= MAX_DEVICES) return SDM_ERR_UNSUPPORTED;
+  PipeStreams& P = g_pipe[dev];
+  if (!P.ready) {
+    int least = 0, greatest = 0;
+    SDM_CUDA_TRY(cudaDeviceGetStreamPriorityRange(&least, &greatest));
+    SDM_CUDA_TRY(cudaStreamCreateWithPriority(&P.hi, cudaStreamNonBlocking, greatest));
+    SDM_CUDA_TRY(cudaStreamCreateWithPriority(&P.lo, cudaStreamNonBlocking, least));
+    cudaEvent_t* evs[] = {&P.fork, &P.done, &P.sel[0], &P.sel[1]};
+    for (cudaEvent_t* e : evs) SDM_CUDA_TRY(cudaEventCreateWithFlags(e, cudaEventDisableTiming));
+    P.ready = true;
+  }
+  *out = &P;
+  return SDM_OK;
+}
+
+// The selection of time chunk [t0, t0 + ct) of every sequence, both jobs, on `q`.
+sdm_status launch_select_chunk(const sdm_shape& s, const WsLayout& WL, const SelJob& jw,
+                               const SelJob& jr, int bf16, int t0, cudaStream_t q) {
+  const int ct = s.T - t0 < WL.chunk ? s.T - t0 : WL.chunk;
+  const long long first = (long long)t0 * s.H;  // the chunk's first row of sequence 0
+  const size_t row_bytes = (size_t)(s.S1 + s.S2) * (bf16 ? 2 : 4);
+  SelJob cw = jw, cr = jr;
+  for (SelJob* j : {&cw, &cr}) {
+    j->halves = static_cast<const unsigned char*>(j->halves) + first * row_bytes;
+    j->idx += first * j->ld;
+    j->wt += first * j->ld;
+    j->seg_rows = ct * s.H;
+    j->seg_stride = (long long)s.T * s.H;
+  }
+  ProfScope ps(SDM_KERNEL_SELECT, q);
+  return launch_select(cw, &cr, (long long)s.B * ct * s.H, s.S1, s.S2, bf16, q,
+                       PIPE_SEL_ROWS_PER_WARP);
+}
+
+// Steps 1-3 with the slot engine, pipelined: chunk c + 1's selection runs on a
+// low-priority stream while chunk c's sort and scan run on a high-priority one; its CTAs
+// take the SM slots that the chunk work leaves (the scan's load-imbalance tail, the
+// sort's narrow kernels).  Forked from and joined back to `st` with events, so `st` sees the
+// same order as the serial schedule; a chunk's work waits for its own selection only.
+sdm_status launch_slot_pipelined(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
+                                 const SelJob& jw, const SelJob& jr, int bf16,
+                                 const float* alpha, const float* beta, const void* v,
+                                 float* M, float* y, const DeviceInfo* di, cudaStream_t st) {
+  SlotArgs a;
+  sdm_status rc = make_slot_args(s, WL, w, alpha, beta, v, M, y, &a);
+  if (rc != SDM_OK) return rc;
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  PipeStreams* P;
+  rc = pipe_streams(&P);
+  if (rc != SDM_OK) return rc;
+  SDM_CUDA_TRY(cudaEventRecord(P->fork, st));
+  SDM_CUDA_TRY(cudaStreamWaitEvent(P->hi, P->fork, 0));
+  SDM_CUDA_TRY(cudaStreamWaitEvent(P->lo, P->fork, 0));
+  // chunk c's selection is recorded in sel[c & 1]; chunk c + 1's record is enqueued before
+  // `hi` waits for chunk c, and chunk c + 2's (the same event) only after that wait, which
+  // keeps the record it saw
+  rc = launch_select_chunk(s, WL, jw, jr, bf16, 0, P->lo);
+  if (rc != SDM_OK) return rc;
+  SDM_CUDA_TRY(cudaEventRecord(P->sel[0], P->lo));
+  for (int c = 0; c < WL.n_chunks; ++c) {
+    if (c + 1 < WL.n_chunks) {
+      rc = launch_select_chunk(s, WL, jw, jr, bf16, (c + 1) * WL.chunk, P->lo);
+      if (rc != SDM_OK) return rc;
+      SDM_CUDA_TRY(cudaEventRecord(P->sel[(c + 1) & 1], P->lo));
     }
-    ProfScope ps(SDM_KERNEL_SCAN_SLOT, st);
-    sdm_status rc;
-    if (d4 <= 32) rc = launch_slot_chunk<1, 4, 6>(a, di, st);
-    else if (d4 <= 64) rc = launch_slot_chunk<2, 2, 6>(a, di, st);
-    else if (d4 <= 128) rc = launch_slot_chunk<4, 4, 4>(a, di, st);
-    else rc = launch_slot_chunk<8, 2, 2>(a, di, st);
+    SDM_CUDA_TRY(cudaStreamWaitEvent(P->hi, P->sel[c & 1], 0));
+    rc = launch_slot_chunk_work(s, WL, w, a, c * WL.chunk, di, P->hi);
     if (rc != SDM_OK) return rc;
   }
+  // `hi` has waited for every selection, so `done` covers both streams
+  SDM_CUDA_TRY(cudaEventRecord(P->done, P->hi));
+  SDM_CUDA_TRY(cudaStreamWaitEvent(st, P->done, 0));
   return SDM_OK;
 }
 
@@ -646,7 +769,7 @@ sdm_status sdm_select(const void* halves, sdm_shape shape, int32_t K, int32_t* i
   if (K < 1 || K > smin || K > KMAX) return SDM_ERR_INVALID_ARG;
   if (!halves || !idx || !wt) return SDM_ERR_INVALID_ARG;
   if (!aligned16(halves) || !aligned16(idx) || !aligned16(wt)) return SDM_ERR_INVALID_ARG;
-  SelJob j{halves, idx, wt, K, K};
+  SelJob j{halves, idx, wt, K, K, 0, 0};
   ProfScope ps(SDM_KERNEL_SELECT, static_cast<cudaStream_t>(stream));
   return launch_select(j, nullptr, (long long)s.B * s.T * s.H, s.S1, s.S2,
                        s.in_dtype == SDM_BF16, static_cast<cudaStream_t>(stream));
@@ -735,13 +858,19 @@ static sdm_status scan_forward(const void* kp, const void* qp, const void* v, co
   const long long rows = (long long)s.B * s.T * s.H;
   const int bf16 = s.in_dtype == SDM_BF16;
 
-  SelJob jw{kp, idx_w, wt_w, s.W, WL.ldw};
-  SelJob jr{qp, idx_r, wt_r, s.R, WL.ldr};
-  {
+  SelJob jw{kp, idx_w, wt_w, s.W, WL.ldw, 0, 0};
+  SelJob jr{qp, idx_r, wt_r, s.R, WL.ldr, 0, 0};
+  const int sched = opt(SDM_OPT_SELECT_SCHEDULE);
+  const bool pipelined = engine == SDM_ENGINE_SLOT && WL.n_chunks > 1 &&
+                         (sched == 2 || (sched == 0 && PIPELINE_BY_DEFAULT));
+  if (pipelined) {
+    rc = launch_slot_pipelined(s, WL, w, jw, jr, bf16, alpha, beta, v, M, y, di, st);
+    if (rc != SDM_OK) return rc;
+  } else {
     ProfScope ps(SDM_KERNEL_SELECT, st);
     rc = launch_select(jw, &jr, rows, s.S1, s.S2, bf16, st);
+    if (rc != SDM_OK) return rc;
   }
-  if (rc != SDM_OK) return rc;
   if (sel_out) {
     SDM_CUDA_TRY(cudaMemcpy2DAsync(sel_out, (size_t)s.W * 4, idx_w, (size_t)WL.ldw * 4,
                                    (size_t)s.W * 4, (size_t)rows, cudaMemcpyDeviceToDevice, st));
@@ -751,8 +880,10 @@ static sdm_status scan_forward(const void* kp, const void* qp, const void* v, co
   }
 
   if (engine == SDM_ENGINE_SLOT) {
-    rc = launch_slot(s, WL, w, alpha, beta, v, M, y, di, st);
-    if (rc != SDM_OK) return rc;
+    if (!pipelined) {
+      rc = launch_slot(s, WL, w, alpha, beta, v, M, y, di, st);
+      if (rc != SDM_OK) return rc;
+    }
     if (o) {
       ProfScope ps(SDM_KERNEL_NORM_GATE, st);
       rc = launch_norm_gate(y, gate, bf16, gamma, eps, act, rows, s.d_v, o, st);
@@ -953,6 +1084,7 @@ sdm_status sdm_set_option(int32_t option, int32_t value) {
     case SDM_OPT_SEQ_COLUMNS: ok = value == 0 || value == 4 || value == 8 || value == 16 || value == 32; break;
     case SDM_OPT_SEQ_DEPTH: ok = value == 0 || value == 4 || value == 8; break;
     case SDM_OPT_SLOT_CTA_STATS: ok = value == 0 || value == 1; break;
+    case SDM_OPT_SELECT_SCHEDULE: ok = value >= 0 && value <= 2; break;
     default: ok = false;
   }
   if (!ok) return SDM_ERR_INVALID_ARG;
@@ -961,7 +1093,7 @@ sdm_status sdm_set_option(int32_t option, int32_t value) {
 }
 
 int32_t sdm_get_option(int32_t option) {
-  if (option < SDM_OPT_NO_PDL || option > SDM_OPT_SLOT_CTA_STATS) return -1;
+  if (option < SDM_OPT_NO_PDL || option > SDM_OPT_SELECT_SCHEDULE) return -1;
   return opt(option);
 }
 

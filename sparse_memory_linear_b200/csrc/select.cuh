@@ -471,7 +471,18 @@ struct SelJob {
   float* wt;
   int K;
   int ld;
+  // Rows of a strided window (0: none).  Row r of the job is row
+  // (r / seg_rows) * seg_stride + r % seg_rows of halves, idx and wt: a time chunk of every
+  // sequence, when the pointers start at the chunk's first row of sequence 0.
+  int seg_rows;
+  long long seg_stride;
 };
+
+__device__ __forceinline__ long long sel_job_row(const SelJob& J, long long r) {
+  if (J.seg_rows == 0) return r;
+  const long long q = r / J.seg_rows;
+  return q * J.seg_stride + (r - q * J.seg_rows);
+}
 
 // Persistent selection kernel over rows of job0 followed by rows of job1.
 __global__ void __launch_bounds__(256) sel_kernel(SelJob job0, SelJob job1, long long n_rows,
@@ -495,7 +506,7 @@ __global__ void __launch_bounds__(256) sel_kernel(SelJob job0, SelJob job1, long
        r += (long long)gridDim.x * wpc) {
     const bool second = r >= n_rows;
     const SelJob& J = second ? job1 : job0;
-    const long long row = second ? r - n_rows : r;
+    const long long row = sel_job_row(J, second ? r - n_rows : r);
     const void* src = reinterpret_cast<const unsigned char*>(J.halves) + (size_t)row * S * esz;
     select_row(src, bf16 != 0, S1, S2, J.K, second ? tab1 : tab0, sc, lane,
                J.idx + (size_t)row * J.ld, J.wt + (size_t)row * J.ld);

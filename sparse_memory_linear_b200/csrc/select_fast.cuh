@@ -210,7 +210,9 @@ __device__ __forceinline__ void half_topk_bf16(const __nv_bfloat16* src, int S, 
   for (int r = 0; r < R8; ++r) {
     const int e0 = r * 256 + lane * 8;
     if (vec && e0 + 8 <= S) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(src + e0);
+      // read once: streamed (evict-first), so that a selection running beside the slot
+      // engine's scan leaves the scan's L2-resident rows in place
+      const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(src + e0));
       const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -500,7 +502,7 @@ __global__ void __launch_bounds__(256, 4) sel_fast_kernel(SelJob job0, SelJob jo
        r += (long long)gridDim.x * wpc) {
     const bool second = r >= n_rows;
     const SelJob& J = second ? job1 : job0;
-    const long long row = second ? r - n_rows : r;
+    const long long row = sel_job_row(J, second ? r - n_rows : r);
     const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(J.halves) + (size_t)row * S;
     select_row_fast<R8, KC>(src, S1, S2, J.K, second ? tab1 : tab0, sc, lane,
                             J.idx + (size_t)row * J.ld, J.wt + (size_t)row * J.ld);

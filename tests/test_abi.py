@@ -201,9 +201,10 @@ def test_options_are_explicit_and_validated(sdm):
     for name, code in sdm.OPTION.items():
         assert sdm.sdm_get_option(name) == 0
     good = {"no_pdl": 1, "select_general": 1, "select_ctas_per_sm": 3, "slot_ctas_per_sm": 2,
-            "seq_columns": 16, "seq_depth": 8, "slot_cta_stats": 1}
+            "seq_columns": 16, "seq_depth": 8, "slot_cta_stats": 1, "select_schedule": 2}
     bad = {"no_pdl": 2, "select_general": -1, "select_ctas_per_sm": 65,
-           "slot_ctas_per_sm": -2, "seq_columns": 12, "seq_depth": 5, "slot_cta_stats": 3}
+           "slot_ctas_per_sm": -2, "seq_columns": 12, "seq_depth": 5, "slot_cta_stats": 3,
+           "select_schedule": 3}
     try:
         for name in sdm.OPTION:
             assert lib.sdm_set_option(sdm.OPTION[name], bad[name]) == 1

@@ -439,12 +439,45 @@ def test_slot_engine_cta_stats_account_for_every_event(sdm):
     assert int(sdm.sdm_slot_cta_stats(reset=True).sum()) == 0
 
 
-def test_scan_slot_engine_over_several_chunks(sdm):
+@pytest.mark.parametrize("schedule", ["serial", "pipelined"])
+@pytest.mark.parametrize("dt", [BF16, F32])
+def test_scan_slot_engine_over_several_chunks(sdm, dt, schedule):
     """Many wide (sequence, head) rows per token make the slot engine's time chunks short
-    (here 128 tokens), so the state carries over between chunks three times; the result is
-    the oracle's all the same."""
+    (here 128 tokens: 128 + 128 + 44), so the state carries over between chunks; the result
+    is the oracle's all the same, with the whole selection first and with each chunk's
+    selection pipelined beside the chunk before (bf16 rows take the fast selection, fp32 rows
+    the general one; both select a chunk of all 8 sequences through a strided window)."""
     wl = sdm_synth.WORKLOADS["tiny"].replace(B=8, H=8, T=300, S1=16, S2=16, W=8, R=8,
-                                            d_v=1024, in_dtype=BF16, seed=61)
+                                            d_v=1024, in_dtype=dt, seed=61)
     g = device_inputs(wl)
-    out, M = run_scan(sdm, wl, g, engine="slot")
+    sdm.sdm_set_option("select_schedule", 1 if schedule == "serial" else 2)
+    try:
+        out, M = run_scan(sdm, wl, g, engine="slot")
+    finally:
+        sdm.sdm_set_option("select_schedule", 0)
     full_check(wl, g, out, M)
+
+
+def test_pipelined_schedule_equals_serial_schedule(sdm):
+    """Both schedules of the slot engine's selection on the long skewed shape at 1/32 of its
+    tokens (4 time chunks): the same selections and final state bit for bit, y within
+    rounding (reads are added with float atomics), and again on a second call that
+    continues from the first call's state."""
+    wl = sdm_synth.WORKLOADS["long_skew"].replace(T=32768)
+    g = device_inputs(wl)
+    res = {}
+    for sched in (1, 2):
+        M = torch.empty((wl.B, wl.H, wl.N, wl.d_v), dtype=F32, device=DEV)
+        sdm.sdm_set_option("select_schedule", sched)
+        try:
+            out1, M = run_scan(sdm, wl, g, engine="slot", want_o=False, M=M)
+            sel1, y1 = out1["sel"].clone(), out1["y"].clone()
+            out2, M = run_scan(sdm, wl, g, engine="slot", want_o=False, M=M, init="continue")
+        finally:
+            sdm.sdm_set_option("select_schedule", 0)
+        res[sched] = (sel1, y1, out2["sel"], out2["y"], M)
+    a, b = res[1], res[2]
+    assert torch.equal(a[0], b[0]) and torch.equal(a[2], b[2])
+    assert torch.equal(a[4], b[4])
+    for ya, yb in ((a[1], b[1]), (a[3], b[3])):
+        assert_close(host(yb), host(ya).astype(np.float64), "y", atol=1e-5, rtol=1e-5)

@@ -285,10 +285,11 @@ def bench_prefill(args, dist: Dist, dev):
         "kernels_ms_per_step": ms_step,
         "kernel_launches_per_step": n_step,
         "kernels_share": {k: ms_step[k] / sum(ms_step.values()) for k in ms_step},
-        "select_schedule": ("library default: with more than one time chunk, chunk c+1's "
-                            "selection runs on a low-priority stream beside chunk c's sort and "
-                            "scan, so the per-kernel times overlap and add up to more than the "
-                            "step"),
+        "select_schedule": (
+            "serial: the whole selection, then the chunks" if args.select_schedule == "serial"
+            else "pipelined (the library's default): with more than one time chunk, chunk "
+                 "c+1's selection runs on a low-priority stream beside chunk c's sort and scan, "
+                 "so the per-kernel times overlap and add up to more than the step"),
         "gpu_launches": int(launched),
         "roofline": {
             "kernel": f"seq_scan_kernel" if scan_kind == "scan_seq" else "slot_chunk_kernel",
@@ -688,6 +689,9 @@ def main(argv=None):
     ap.add_argument("--cpu-tokens", type=int, default=8192,
                     help="tokens per head of the CPU-oracle sample")
     ap.add_argument("--reference-tokens", type=int, default=2048)
+    ap.add_argument("--select-schedule", choices=["default", "serial", "pipelined"],
+                    default="default",
+                    help="the slot engine's selection schedule (SDM_OPT_SELECT_SCHEDULE)")
     ap.add_argument("--only", choices=["prefill", "decode", "balance"], default=None,
                     help="run one part (profiling of a small case)")
     ap.add_argument("--override", default="",
@@ -720,6 +724,8 @@ def main(argv=None):
         torch.cuda.set_device(dev)
         import sparse_memory_linear_b200 as sdm
         sdm.library()
+        sdm.sdm_set_option("select_schedule",
+                           {"default": 0, "serial": 1, "pipelined": 2}[args.select_schedule])
 
         if args.only == "balance":
             out = bench_balance(args, dev)

@@ -281,9 +281,9 @@ struct EngineMeasure {
   float seq_ms, slot_ms;
 };
 constexpr EngineMeasure kEngineTable[] = {
-    {2, 4, 2048, 65536, 64, 12.32f, 0.611f},          // small layer
-    {4, 8, 8192, 262144, 128, 28.80f, 11.98f},        // 1.4B-like layer
-    {1, 4, 262144, 1048576, 256, 1769.2f, 57.36f},    // long prefill, skewed slots
+    {2, 4, 2048, 65536, 64, 12.67f, 0.597f},          // small layer
+    {4, 8, 8192, 262144, 128, 29.69f, 10.29f},        // 1.4B-like layer
+    {1, 4, 262144, 1048576, 256, 1769.2f, 46.30f},    // long prefill, skewed slots
     {64, 8, 256, 262144, 128, 12.82f, 6.34f},         // many short sequences
 };
 

@@ -450,6 +450,53 @@ def bench_balance(args, dev):
             "busy_us_per_cta": q(active[:, 3] / 8.0 / 1e3)}
 
 
+def bench_state_rows(args, dist: Dist, dev):
+    """State checkpoints of the long skewed layer (M: 4 heads x 2^20 slots x 256 fp32, 4 GB,
+    larger than L2): sdm_state_pack and sdm_state_unpack per format, each timed alone with
+    CUDA events (median of 5 after 3 warm-ups).  HBM bytes per call: the fp32 rows plus the
+    codes plus the per-row scales, each once."""
+    import sparse_memory_linear_b200 as sdm
+
+    stream = torch.cuda.current_stream(dev)
+    peak, peak_kind = hbm_peak()
+    wl = sdm_synth.WORKLOADS[args.workload]
+    gen = torch.Generator(device=dev).manual_seed(0x5D3)
+    M = torch.randn((wl.B * wl.H * wl.N, wl.d_v), generator=gen, device=dev) * 0.02
+    back = torch.empty_like(M)
+    rows = M.shape[0]
+    out = {"workload": f"{wl.name} state, {rows} rows x {wl.d_v} fp32 ({M.numel() * 4 >> 20} MiB)"}
+    for fmt in ("bf16", "e4m3", "int4"):
+        codes, scales = sdm.sdm_state_pack(M, fmt)
+        code_bytes = codes.numel() * codes.element_size()
+        scale_bytes = 0 if scales is None else rows * 4
+        io = M.numel() * 4 + code_bytes + scale_bytes
+        res = {"code_bytes": code_bytes, "scale_bytes": scale_bytes}
+        for name, fn in (("pack", lambda: sdm.sdm_state_pack(M, fmt, codes=codes, scales=scales)),
+                         ("unpack", lambda: sdm.sdm_state_unpack(codes, scales, wl.d_v, fmt,
+                                                                 out=back))):
+            ts = []
+            for i in range(8):
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                torch.cuda.synchronize(dev)
+                if i >= 3:
+                    ts.append(a.elapsed_time(b))
+            ms = float(np.median(ts))
+            gbps = io / (ms * 1e-3) / 1e9
+            res[name] = {"ms": ms, "GBps": gbps, "frac": gbps / peak}
+        out[fmt] = res
+    out["peak"] = peak
+    out["peak_kind"] = f"{peak_kind} (burst copy)"
+    if sdm.sdm_get_device_status() != 0:
+        raise RuntimeError("device status word set during the checkpoint benchmark")
+    del M, back
+    torch.cuda.empty_cache()
+    return out
+
+
 def bench_coupled(args, dist: Dist, dev):
     """The coupled delta rule: prefill of the 1.4B-like workload (sequential engine, the one
     that computes it) and 256 chained decode steps of the batched-decode workload, timed as
@@ -692,7 +739,7 @@ def main(argv=None):
     ap.add_argument("--select-schedule", choices=["default", "serial", "pipelined"],
                     default="default",
                     help="the slot engine's selection schedule (SDM_OPT_SELECT_SCHEDULE)")
-    ap.add_argument("--only", choices=["prefill", "decode", "balance"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "balance", "rows"], default=None,
                     help="run one part (profiling of a small case)")
     ap.add_argument("--override", default="",
                     help="workload fields to change, e.g. B=1,T=4096 (prefill workload)")
@@ -731,6 +778,11 @@ def main(argv=None):
             out = bench_balance(args, dev)
             if dist.rank == 0:
                 print(json.dumps({"balance": out}), flush=True)
+            return 0
+        if args.only == "rows":
+            out = bench_state_rows(args, dist, dev)
+            if dist.rank == 0:
+                print(json.dumps({"state_rows": out}), flush=True)
             return 0
         if args.only == "decode":
             out = bench_decode(args, dist, dev)
@@ -776,6 +828,7 @@ def main(argv=None):
             line["decode"] = bench_decode(args, dist, dev)
         if not args.no_configs and args.only is None:
             line["coupled"] = bench_coupled(args, dist, dev)
+            line["state_rows"] = bench_state_rows(args, dist, dev)
         if dist.rank == 0:
             print(json.dumps(line), flush=True)
         return 0

@@ -227,6 +227,42 @@ sdm_status sdm_decode_step_coupled_chained(const void *kp, const void *qp, const
 sdm_status sdm_norm_gate(const float *y, const void *gate, const float *gamma, float eps,
                          int32_t act, sdm_shape shape, float *o, void *stream);
 
+/*
+ * Low-precision state rows (state checkpoints) [m.163.com article on SDM, section 八, the
+ * memory-efficiency paragraph: the state checkpoints of 128k fine-tuning stored as fp8 or
+ * int4, with no loss in training loss or final quality].  A checkpoint row holds one row of
+ * d_v fp32 state values as
+ *   SDM_ROWS_BF16: d_v 16-bit codes, each value rounded to nearest-even bf16; no scale;
+ *   SDM_ROWS_E4M3: d_v 8-bit OCP FP8 E4M3 codes of x / s and one fp32 scale s = amax / 448
+ *                  (amax: the row's largest |x|), rounded to nearest-even and saturating at
+ *                  +-448; a zero result is the code 0x00;
+ *   SDM_ROWS_INT4: d_v / 2 bytes of 4-bit two's-complement codes, element 2i in the low
+ *                  nibble of byte i, of x / s rounded to nearest-even and clamped to [-7, 7],
+ *                  and one fp32 scale s = amax / 7.
+ * s, x / s and the unpacked code * s are single fp32 operations rounded to nearest; s = 0
+ * gives all-zero codes.  The live state of the pass stays fp32: these calls make and read
+ * checkpoints of it (any `rows` rows of d_v values, e.g. M [B,H,N,d_v] as B*H*N rows).
+ */
+typedef enum { SDM_ROWS_BF16 = 1, SDM_ROWS_E4M3 = 2, SDM_ROWS_INT4 = 3 } sdm_row_format;
+
+/* Bytes of the codes of `rows` rows of d_v values in `format`; 0 for invalid arguments
+ * (rows < 0, d_v outside [4, 512] or not a multiple of 4, unknown format). */
+size_t sdm_state_rows_bytes(int64_t rows, int32_t d_v, int32_t format);
+
+/* Packs M [rows, d_v] (fp32, device) into codes (device, sdm_state_rows_bytes bytes) and, for
+ * E4M3 and INT4, scales [rows] (fp32, device; ignored for BF16).  M and codes 16-byte
+ * aligned, scales 4-byte aligned; none may overlap.  Invalid arguments return
+ * SDM_ERR_INVALID_ARG before anything is launched; rows = 0 launches nothing.  One launch,
+ * asynchronous on `stream`. */
+sdm_status sdm_state_pack(const float *M, int64_t rows, int32_t d_v, int32_t format,
+                          void *codes, float *scales, void *stream);
+
+/* Unpacks codes (+ scales) made by sdm_state_pack into M [rows, d_v] (fp32): each value is
+ * its code's value times the row's scale (BF16: the code widened).  Same rules as
+ * sdm_state_pack. */
+sdm_status sdm_state_unpack(const void *codes, const float *scales, int64_t rows, int32_t d_v,
+                            int32_t format, float *M, void *stream);
+
 /* Kinds of kernel launch reported by the timing calls below. */
 typedef enum {
     SDM_KERNEL_STATE_INIT = 0, /* M0 broadcast into M                         */
@@ -236,6 +272,7 @@ typedef enum {
     SDM_KERNEL_NORM_GATE = 4,  /* step 4                                      */
     SDM_KERNEL_DECODE = 5,     /* fused decode step                           */
     SDM_KERNEL_SLOT_SORT = 6,  /* slot engine: event build and radix sort      */
+    SDM_KERNEL_STATE_ROWS = 7, /* state checkpoint pack / unpack              */
     SDM_KERNEL_KINDS = 8
 } sdm_kernel_kind;
 

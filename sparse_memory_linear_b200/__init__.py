@@ -10,6 +10,7 @@ from ._binding import (  # noqa: F401
     ACT,
     ENGINE,
     OPTION,
+    ROW_FORMAT,
     SDM_BF16,
     SDM_F32,
     SdmError,
@@ -33,6 +34,9 @@ from ._binding import (  # noqa: F401
     sdm_set_option,
     sdm_slot_cta_stats,
     sdm_state_init,
+    sdm_state_pack,
+    sdm_state_rows_bytes,
+    sdm_state_unpack,
     sdm_status_string,
     sdm_workspace_size,
     shape_of,

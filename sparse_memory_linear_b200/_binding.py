@@ -68,6 +68,9 @@ def library():
         "sdm_set_option": ([I, I], I),
         "sdm_get_option": ([I], I),
         "sdm_slot_cta_stats": ([P, I, I], I),
+        "sdm_state_rows_bytes": ([ctypes.c_int64, I, I], Z),
+        "sdm_state_pack": ([P, ctypes.c_int64, I, I, P, P, P], I),
+        "sdm_state_unpack": ([P, P, ctypes.c_int64, I, I, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -345,8 +348,69 @@ def sdm_norm_gate(y, *, gate=None, gamma=None, eps: float = 1e-6, act: str = "si
     return o
 
 
+ROW_FORMAT = {"bf16": 1, "e4m3": 2, "int4": 3}
+
+
+def _row_codes_shape(rows: int, d_v: int, fmt: str):
+    if fmt == "bf16":
+        return (rows, d_v), torch.int16
+    if fmt == "e4m3":
+        return (rows, d_v), torch.uint8
+    if fmt == "int4":
+        return (rows, d_v // 2), torch.uint8
+    raise ValueError(f"unknown row format {fmt!r}; one of {sorted(ROW_FORMAT)}")
+
+
+def sdm_state_rows_bytes(rows: int, d_v: int, fmt: str = "e4m3") -> int:
+    """Bytes of the checkpoint codes of `rows` rows of d_v values (0: invalid arguments)."""
+    return int(library().sdm_state_rows_bytes(int(rows), int(d_v), ROW_FORMAT[fmt]))
+
+
+def sdm_state_pack(M, fmt: str = "e4m3", *, codes=None, scales=None, stream=None):
+    """Checkpoint rows of M [..., d_v] (fp32): (codes, scales).  codes: int16 [rows, d_v]
+    (bf16 bit patterns), uint8 [rows, d_v] (E4M3) or uint8 [rows, d_v / 2] (int4, two per
+    byte); scales: fp32 [rows] (None for bf16)."""
+    d_v = M.shape[-1]
+    rows = M.numel() // d_v if d_v else 0
+    cshape, cdt = _row_codes_shape(rows, d_v, fmt)
+    _expect(codes, "codes", cshape)
+    _expect(scales, "scales", (rows,))
+    _need(M, "M", torch.float32)
+    if codes is None:
+        codes = torch.empty(cshape, dtype=cdt, device=M.device)
+    _need(codes, "codes", cdt, M.device)
+    if fmt != "bf16":
+        if scales is None:
+            scales = torch.empty(rows, dtype=torch.float32, device=M.device)
+        _need(scales, "scales", torch.float32, M.device)
+    else:
+        scales = None
+    _check(library().sdm_state_pack(_p(M), rows, d_v, ROW_FORMAT[fmt], _p(codes), _p(scales),
+                                    _stream(stream, M.device)), "sdm_state_pack")
+    return codes, scales
+
+
+def sdm_state_unpack(codes, scales, d_v: int, fmt: str = "e4m3", *, out=None, stream=None):
+    """fp32 rows [rows, d_v] from checkpoint codes (+ scales) made by sdm_state_pack."""
+    rows = codes.shape[0]
+    cshape, cdt = _row_codes_shape(rows, d_v, fmt)
+    _expect(codes, "codes", cshape)
+    _expect(out, "out", None, rows * d_v)
+    _need(codes, "codes", cdt)
+    if fmt != "bf16":
+        _expect(scales, "scales", (rows,))
+        _need(scales, "scales", torch.float32, codes.device)
+    out = torch.empty((rows, d_v), dtype=torch.float32, device=codes.device) if out is None \
+        else out
+    _need(out, "out", torch.float32, codes.device)
+    _check(library().sdm_state_unpack(_p(codes), _p(scales if fmt != "bf16" else None), rows,
+                                      d_v, ROW_FORMAT[fmt], _p(out),
+                                      _stream(stream, codes.device)), "sdm_state_unpack")
+    return out
+
+
 KERNEL_KINDS = ("state_init", "select", "scan_seq", "scan_slot", "norm_gate", "decode",
-                "slot_sort")
+                "slot_sort", "state_rows")
 
 
 def sdm_profile_enable(on: bool = True):

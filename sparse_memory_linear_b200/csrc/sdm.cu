@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "norm_init.cuh"
+#include "rows.cuh"
 #include "scan_seq.cuh"
 #include "scan_slot.cuh"
 #include "select.cuh"
@@ -803,6 +804,95 @@ sdm_status sdm_norm_gate(const float* y, const void* gate, const float* gamma, f
   return launch_norm_gate(y, gate, s.in_dtype == SDM_BF16, gamma, eps, act,
                           (long long)s.B * s.T * s.H, s.d_v, o,
                           static_cast<cudaStream_t>(stream));
+}
+
+// Bytes of the codes of `rows` state rows in `format` (0: invalid arguments).
+static size_t rows_code_bytes(int64_t rows, int32_t d_v, int32_t format) {
+  if (rows < 0 || d_v < 4 || d_v > 512 || d_v % 4 != 0) return 0;
+  switch (format) {
+    case SDM_ROWS_BF16: return (size_t)rows * d_v * 2;
+    case SDM_ROWS_E4M3: return (size_t)rows * d_v;
+    case SDM_ROWS_INT4: return (size_t)rows * d_v / 2;
+  }
+  return 0;
+}
+
+static unsigned rows_grid(int64_t rows, const DeviceInfo* di) {
+  long long blocks = (rows + 7) / 8;  // a warp per row
+  if (blocks > (long long)di->sms * 16) blocks = (long long)di->sms * 16;
+  return (unsigned)(blocks > 0 ? blocks : 1);
+}
+
+// Host checks shared by the pack and unpack calls.
+static sdm_status rows_check(const void* M, int64_t rows, int32_t d_v, int32_t format,
+                             const void* codes, const void* scales) {
+  if (rows == 0 && format >= SDM_ROWS_BF16 && format <= SDM_ROWS_INT4 && d_v >= 4 &&
+      d_v <= 512 && d_v % 4 == 0)
+    return SDM_OK;
+  const size_t nc = rows_code_bytes(rows, d_v, format);
+  if (nc == 0 || !M || !codes || !aligned16(M) || !aligned16(codes)) return SDM_ERR_INVALID_ARG;
+  const size_t nm = (size_t)rows * d_v * 4;
+  if (overlaps(M, nm, codes, nc)) return SDM_ERR_INVALID_ARG;
+  if (format != SDM_ROWS_BF16) {
+    if (!scales || (reinterpret_cast<uintptr_t>(scales) & 3u) != 0) return SDM_ERR_INVALID_ARG;
+    if (overlaps(M, nm, scales, (size_t)rows * 4) || overlaps(codes, nc, scales, (size_t)rows * 4))
+      return SDM_ERR_INVALID_ARG;
+  }
+  return SDM_OK;
+}
+
+size_t sdm_state_rows_bytes(int64_t rows, int32_t d_v, int32_t format) {
+  return rows_code_bytes(rows, d_v, format);
+}
+
+sdm_status sdm_state_pack(const float* M, int64_t rows, int32_t d_v, int32_t format,
+                          void* codes, float* scales, void* stream) {
+  NvtxRange nvtx_range("sdm_state_pack");
+  sdm_status rc = rows_check(M, rows, d_v, format, codes, scales);
+  if (rc != SDM_OK || rows == 0) return rc;
+  DeviceInfo* di;
+  rc = device_info(&di);
+  if (rc != SDM_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProfScope ps(SDM_KERNEL_STATE_ROWS, st);
+  const dim3 grid(rows_grid(rows, di)), block(256);
+  if (format == SDM_ROWS_BF16)
+    SDM_CUDA_TRY(launch_pdl(rows_pack_kernel<ROWS_FMT_BF16>, grid, block, 0, st, M,
+                            (long long)rows, (int)d_v, codes, scales));
+  else if (format == SDM_ROWS_E4M3)
+    SDM_CUDA_TRY(launch_pdl(rows_pack_kernel<ROWS_FMT_E4M3>, grid, block, 0, st, M,
+                            (long long)rows, (int)d_v, codes, scales));
+  else
+    SDM_CUDA_TRY(launch_pdl(rows_pack_kernel<ROWS_FMT_INT4>, grid, block, 0, st, M,
+                            (long long)rows, (int)d_v, codes, scales));
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  SDM_CUDA_TRY(cudaGetLastError());
+  return SDM_OK;
+}
+
+sdm_status sdm_state_unpack(const void* codes, const float* scales, int64_t rows, int32_t d_v,
+                            int32_t format, float* M, void* stream) {
+  NvtxRange nvtx_range("sdm_state_unpack");
+  sdm_status rc = rows_check(M, rows, d_v, format, codes, scales);
+  if (rc != SDM_OK || rows == 0) return rc;
+  DeviceInfo* di;
+  rc = device_info(&di);
+  if (rc != SDM_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProfScope ps(SDM_KERNEL_STATE_ROWS, st);
+  const dim3 grid(rows_grid(rows, di)), block(256);
+  if (format == SDM_ROWS_BF16)
+    SDM_CUDA_TRY(launch_pdl(rows_unpack_kernel<ROWS_FMT_BF16>, grid, block, 0, st, codes,
+                            scales, (long long)rows, (int)d_v, M));
+  else if (format == SDM_ROWS_E4M3)
+    SDM_CUDA_TRY(launch_pdl(rows_unpack_kernel<ROWS_FMT_E4M3>, grid, block, 0, st, codes,
+                            scales, (long long)rows, (int)d_v, M));
+  else
+    SDM_CUDA_TRY(launch_pdl(rows_unpack_kernel<ROWS_FMT_INT4>, grid, block, 0, st, codes,
+                            scales, (long long)rows, (int)d_v, M));
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  SDM_CUDA_TRY(cudaGetLastError());
+  return SDM_OK;
 }
 
 // Prefill; `coupled` selects the coupled delta rule (sequential engine only).

@@ -177,6 +177,39 @@ def _decode_select_norm_reject(sdm):
     assert lib.sdm_state_init(P(FAKE), P(FAKE), s, None) == 1
 
 
+def test_state_rows_bytes(sdm):
+    assert sdm.sdm_state_rows_bytes(1000, 256, "bf16") == 512000
+    assert sdm.sdm_state_rows_bytes(1000, 256, "e4m3") == 256000
+    assert sdm.sdm_state_rows_bytes(1000, 256, "int4") == 128000
+    assert sdm.sdm_state_rows_bytes(0, 4, "int4") == 0
+    lib = sdm.library()
+    for rows, d_v, fmt in ((-1, 64, 2), (10, 2, 2), (10, 6, 2), (10, 516, 3), (10, 64, 0),
+                           (10, 64, 4)):
+        assert lib.sdm_state_rows_bytes(rows, d_v, fmt) == 0
+
+
+@host_only
+def test_state_pack_and_unpack_reject_bad_arguments(sdm):
+    """Unknown format, d_v out of range, missing or misaligned buffers, a missing scale
+    array, overlapping buffers: SDM_ERR_INVALID_ARG before any launch; rows = 0 is a no-op."""
+    lib = sdm.library()
+    P = ctypes.c_void_p
+    big = FAKE + (1 << 30)
+    with no_launch(sdm):
+        for fn, args in ((lib.sdm_state_pack, lambda M, r, d, f, c, s: (M, r, d, f, c, s, None)),
+                         (lib.sdm_state_unpack, lambda M, r, d, f, c, s: (c, s, r, d, f, M, None))):
+            assert fn(*args(P(FAKE), 8, 64, 0, P(big), P(big * 2))) == 1      # format
+            assert fn(*args(P(FAKE), 8, 66, 2, P(big), P(big * 2))) == 1      # d_v % 4
+            assert fn(*args(P(FAKE), 8, 1024, 2, P(big), P(big * 2))) == 1    # d_v > 512
+            assert fn(*args(None, 8, 64, 2, P(big), P(big * 2))) == 1         # no M
+            assert fn(*args(P(FAKE), 8, 64, 2, None, P(big * 2))) == 1        # no codes
+            assert fn(*args(P(FAKE), 8, 64, 2, P(big + 4), P(big * 2))) == 1  # misaligned
+            assert fn(*args(P(FAKE), 8, 64, 3, P(big), None)) == 1            # no scales
+            assert fn(*args(P(FAKE), 8, 64, 2, P(FAKE + 256), P(big * 2))) == 1  # overlap
+            assert fn(*args(P(FAKE), -1, 64, 2, P(big), P(big * 2))) == 1     # rows < 0
+            assert fn(*args(None, 0, 64, 2, None, None)) == 0                 # nothing to do
+
+
 @host_only
 def test_noalloc_rejects_shapes_beyond_its_scratch(sdm):
     """4 x 8192 x 8 rows with W = R = 64 need 128 MiB of scratch, beyond the fixed 16 MiB

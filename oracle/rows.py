@@ -7,16 +7,19 @@ module states, from the formats' definitions, what a checkpoint row holds:
     bf16  one 16-bit code per value: the fp32 value rounded to nearest, ties to even, to
           8 significand bits (no scale);
     e4m3  one 8-bit code per value and one fp32 scale per row, s = amax / 448: the code is
-          the OCP FP8 E4M3 value nearest to x / s (ties to even, saturating at +-448); a
-          value that rounds to zero takes the code of +0;
+          the OCP FP8 E4M3 value nearest to q = x * (1 / s) (ties to even, saturating at
+          +-448); a value that rounds to zero takes the code of +0;
     int4  one 4-bit two's-complement code per value (two per byte, the even element in the
-          low nibble) and one fp32 scale per row, s = amax / 7: the code is x / s rounded to
-          nearest, ties to even, clamped to [-7, 7].
+          low nibble) and one fp32 scale per row, s = amax / 7: the code is q = x * (1 / s)
+          rounded to nearest, ties to even, clamped to [-7, 7].
 
-amax is the row's largest |x|.  The scale, the quotient x / s and the decoded value code * s
-are each one fp32 operation rounded to nearest; a row with amax = 0 (or a scale that
-underflows to 0) gets scale 0 and all-zero codes.  Those fp32 steps decide the codes, so the
-oracle takes them in fp32 as the kernels do; everything else is exact.  Inputs are finite.
+amax is the row's largest |x|.  The value coded is q = x * r with r = 1 / s; the scale s,
+its reciprocal r, the product q and the decoded value code * s are each one fp32 operation
+rounded to nearest.  A scale below the smallest normal fp32, 2^-126 (amax below about
+5.3e-36 for E4M3 and 8.2e-38 for int4, or zero), is stored as 0 with all-zero codes, so that r
+stays finite.  Those fp32
+steps decide the codes, so the oracle takes them in fp32 as the kernels do; everything else
+is exact.  Inputs are finite.
 
 Only the test-suite, the smoke check and the benchmark's CPU-baseline leg may import this
 module; the product path never does.
@@ -84,10 +87,14 @@ def bf16_decode(c: np.ndarray) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------- rows
+FLT_MIN = np.float32(2.0 ** -126)
+
+
 def row_scale(row: np.ndarray, fmt: str) -> np.float32:
     amax = np.float32(np.max(np.abs(row.astype(np.float32)))) if row.size else np.float32(0)
     top = np.float32(E4M3_MAX if fmt == "e4m3" else INT4_MAX)
-    return np.float32(amax / top)
+    s = np.float32(amax / top)
+    return s if s >= FLT_MIN else np.float32(0)
 
 
 def pack(M: np.ndarray, fmt: str):
@@ -111,7 +118,7 @@ def pack(M: np.ndarray, fmt: str):
         scales[r] = s
         if s == 0:
             continue
-        q = M[r] / s  # fp32 / fp32 -> fp32, rounded to nearest
+        q = M[r] * np.float32(np.float32(1) / s)  # fp32 reciprocal, fp32 product
         if fmt == "e4m3":
             codes[r] = [e4m3_encode(float(v)) for v in q]
         else:

@@ -96,8 +96,12 @@ def test_hand_worked_int4_row():
 
 
 def test_zero_row_has_zero_scale_and_codes():
-    row = np.zeros((2, 8), np.float32)
+    """All-zero rows, and rows so small that their scale would fall below the smallest
+    normal fp32 (whose reciprocal would overflow), are stored as zero."""
+    row = np.zeros((4, 8), np.float32)
     row[1, 3] = -0.0
+    row[2, :] = np.float32(1e-38)
+    row[3, 5] = np.float32(-5e-38)
     for fmt in ("e4m3", "int4"):
         codes, scales = R.pack(row, fmt)
         assert not codes.any() and not scales.any()
@@ -107,8 +111,8 @@ def test_zero_row_has_zero_scale_and_codes():
 @pytest.mark.parametrize("fmt", ["e4m3", "int4"])
 def test_round_trip_error_is_within_half_a_code_step(fmt):
     """|unpack(pack(x)) - x| is at most half the spacing of the code grid at x / s, times s
-    (plus the fp32 roundings of x / s and code * s), and the row's largest |x| comes back
-    within one fp32 rounding."""
+    (plus the fp32 roundings of 1 / s, x * (1 / s) and code * s), and the row's largest |x|
+    comes back within the same roundings."""
     rng = np.random.default_rng(7)
     M = (rng.standard_normal((64, 32)) * 10.0 ** rng.integers(-3, 3, (64, 1))).astype(np.float32)
     codes, scales = R.pack(M, fmt)
@@ -122,7 +126,7 @@ def test_round_trip_error_is_within_half_a_code_step(fmt):
         i = np.clip(np.searchsorted(grid, q, side="right") - 1, 0, 125)
         step = grid[i + 1] - grid[i]
     err = np.abs(back.astype(np.float64) - M)
-    assert np.all(err <= s * step / 2 + 4e-7 * np.abs(M) + 1e-30)
+    assert np.all(err <= s * step / 2 + 5e-7 * np.abs(M) + 1e-30)
     amax = np.abs(M).max(axis=1)
     got = np.abs(back).max(axis=1)
-    assert np.all(np.abs(got - amax) <= 4e-7 * amax)
+    assert np.all(np.abs(got - amax) <= 5e-7 * amax)

@@ -5,12 +5,13 @@
 // A row of d_v fp32 values becomes
 //   bf16: d_v codes, each the value rounded to nearest-even bf16 (no scale);
 //   E4M3: d_v codes and one fp32 scale s = amax / 448: the OCP FP8 E4M3 value nearest to
-//         x / s (ties to even, saturating; a zero result is the code of +0);
+//         q = x * (1 / s) (ties to even, saturating; a zero result is the code of +0);
 //   int4: d_v / 2 bytes of 4-bit two's-complement codes (element 2i in the low nibble) and
-//         one fp32 scale s = amax / 7: x / s rounded to nearest-even, clamped to [-7, 7];
-// amax being the row's largest |x|.  s, x / s and code * s are single fp32 operations rounded
-// to nearest (IEEE division, no approximations); s = 0 gives all-zero codes.  Both kernels
-// stream: each row is read and written once, one warp per row, 16-byte loads.
+//         one fp32 scale s = amax / 7: q rounded to nearest-even, clamped to [-7, 7];
+// amax being the row's largest |x|.  s, 1 / s, q and code * s are single fp32 operations
+// rounded to nearest (IEEE division for s and 1 / s, once per row); a scale below the
+// smallest normal fp32 is stored as 0 with all-zero codes, which keeps 1 / s finite.  Both
+// kernels stream: each row is read and written once, one warp per row, 16-byte loads.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -87,19 +88,17 @@ __global__ void __launch_bounds__(256) rows_pack_kernel(const float* __restrict_
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      const float s = amax / (FMT == ROWS_FMT_E4M3 ? 448.0f : 7.0f);
+      const float s0 = amax / (FMT == ROWS_FMT_E4M3 ? 448.0f : 7.0f);
+      const float s = s0 >= 1.17549435e-38f ? s0 : 0.0f;  // 2^-126, the smallest normal
+      const float inv = s != 0.0f ? 1.0f / s : 0.0f;
       if (lane == 0) scales[r] = s;
 #pragma unroll
       for (int k = 0; k < ROWS_MAX_Q; ++k) {
         const int c = lane + 32 * k;
         if (c >= d4) continue;
-        float q[4] = {0.f, 0.f, 0.f, 0.f};
-        if (s != 0.0f) {
-          q[0] = x[k].x / s;
-          q[1] = x[k].y / s;
-          q[2] = x[k].z / s;
-          q[3] = x[k].w / s;
-        }
+        // inv = 0 for a zero row: every q is +-0 and codes to 0
+        const float q[4] = {__fmul_rn(x[k].x, inv), __fmul_rn(x[k].y, inv),
+                            __fmul_rn(x[k].z, inv), __fmul_rn(x[k].w, inv)};
         if constexpr (FMT == ROWS_FMT_E4M3) {
           const uint32_t w = e4m3_code(q[0]) | (e4m3_code(q[1]) << 8) |
                              (e4m3_code(q[2]) << 16) | (e4m3_code(q[3]) << 24);

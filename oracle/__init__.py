@@ -64,6 +64,8 @@ def _load():
         lib.sdm_oracle_pass.restype = I
         lib.sdm_oracle_pass_coupled.argtypes = lib.sdm_oracle_pass.argtypes
         lib.sdm_oracle_pass_coupled.restype = I
+        lib.sdm_oracle_pass_logged.argtypes = lib.sdm_oracle_pass.argtypes + [P]
+        lib.sdm_oracle_pass_logged.restype = I
         lib.sdm_oracle_norm_gate.argtypes = [L, I, P, P, P, ctypes.c_double, I, P]
         lib.sdm_oracle_norm_gate.restype = I
         _lib = lib
@@ -128,8 +130,13 @@ def norm_gate(y, g=None, gamma=None, eps: float = 1e-6, act: str | int = "silu")
 
 def run_unit(kp, qp, v, alpha, beta, M_init, b: int, h: int, *, S1: int, W: int, R: int,
              rows=None, want_y=None, t_end=None, select_mode: str = "product_key",
-             threads: int = 1, selection=None, coupled: bool = False):
+             threads: int = 1, selection=None, coupled: bool = False,
+             want_log: bool = False):
     """Steps 1-3 for one (sequence b, head h) over tokens [0, t_end).
+
+    want_log: also return "wlog" [t_end, W, d_v] float64, the undo log of the in-place
+    update: written slot j of token t as the write found it (sdm_oracle_pass_logged; NaN for
+    untracked rows).
 
     coupled: the coupled delta rule (one prediction shared by the token's written rows,
     sdm_oracle_pass_coupled) instead of the per-slot write; every written row must then be
@@ -192,22 +199,33 @@ def run_unit(kp, qp, v, alpha, beta, M_init, b: int, h: int, *, S1: int, W: int,
     wy = None if want_y is None else np.ascontiguousarray(want_y, dtype=np.uint8)
     y = np.full((t_end, d_v), np.nan, np.float64)
     M_out = np.empty((n_rows, d_v), np.float32)
-    fn = lib.sdm_oracle_pass_coupled if coupled else lib.sdm_oracle_pass
-    rc = fn(t_end, N, d_v, W, R, _ptr(idx_w), _ptr(wt_w), _ptr(idx_r), _ptr(wt_r), _ptr(v_u),
+    args = (t_end, N, d_v, W, R, _ptr(idx_w), _ptr(wt_w), _ptr(idx_r), _ptr(wt_r), _ptr(v_u),
             d_v, _ptr(a_u), _ptr(be_u), 1, n_rows, _ptr(rows_arr), _ptr(M_in), _ptr(wy),
             _ptr(y), _ptr(M_out))
+    wlog = None
+    if want_log:
+        if coupled:
+            raise ValueError("the undo log is kept for the per-slot rule")
+        wlog = np.empty((t_end, W, d_v), np.float64)
+        rc = lib.sdm_oracle_pass_logged(*args, _ptr(wlog))
+    else:
+        rc = (lib.sdm_oracle_pass_coupled if coupled else lib.sdm_oracle_pass)(*args)
     if rc != 0:
         raise ValueError(f"sdm_oracle_pass failed ({rc})")
-    return dict(idx_w=idx_w, wt_w=wt_w, idx_r=idx_r, wt_r=wt_r, y=y, M=M_out, rows=rows_arr)
+    out = dict(idx_w=idx_w, wt_w=wt_w, idx_r=idx_r, wt_r=wt_r, y=y, M=M_out, rows=rows_arr)
+    if want_log:
+        out["wlog"] = wlog
+    return out
 
 
 def forward(kp, qp, v, alpha, beta, M_init, *, S1: int, W: int, R: int, gate=None,
             gamma=None, eps: float = 1e-6, act="silu", select_mode: str = "product_key",
-            threads: int = 1, coupled: bool = False):
+            threads: int = 1, coupled: bool = False, want_log: bool = False):
     """The whole pass over every (b, h) and every token, all rows tracked.
 
     Returns dict(idx_w [B,T,H,W], idx_r [B,T,H,R], wt_w, wt_r, y [B,T,H,d_v] float64,
-    o [B,T,H,d_v] float64, M [B,H,N,d_v] float32).
+    o [B,T,H,d_v] float64, M [B,H,N,d_v] float32), and with want_log the undo log
+    wlog [B,T,H,W,d_v] float64 (run_unit).
     """
     B, T, H, S = kp.shape
     N = S1 * (S - S1)
@@ -218,12 +236,15 @@ def forward(kp, qp, v, alpha, beta, M_init, *, S1: int, W: int, R: int, gate=Non
     wt_r = np.empty((B, T, H, R), np.float64)
     y = np.empty((B, T, H, d_v), np.float64)
     M = np.empty((B, H, N, d_v), np.float32)
+    wlog = np.empty((B, T, H, W, d_v), np.float64) if want_log else None
     units = [(b, h) for b in range(B) for h in range(H)]
 
     def one(u):
         b, h = u
         r = run_unit(kp, qp, v, alpha, beta, M_init, b, h, S1=S1, W=W, R=R,
-                     select_mode=select_mode, coupled=coupled)
+                     select_mode=select_mode, coupled=coupled, want_log=want_log)
+        if want_log:
+            wlog[b, :, h] = r["wlog"]
         idx_w[b, :, h], wt_w[b, :, h] = r["idx_w"], r["wt_w"]
         idx_r[b, :, h], wt_r[b, :, h] = r["idx_r"], r["wt_r"]
         y[b, :, h] = r["y"]
@@ -237,4 +258,25 @@ def forward(kp, qp, v, alpha, beta, M_init, *, S1: int, W: int, R: int, gate=Non
             one(u)
     g = None if gate is None else np.asarray(gate, dtype=np.float32)
     o = norm_gate(y, g, gamma, eps, act)
-    return dict(idx_w=idx_w, idx_r=idx_r, wt_w=wt_w, wt_r=wt_r, y=y, o=o, M=M)
+    out = dict(idx_w=idx_w, idx_r=idx_r, wt_w=wt_w, wt_r=wt_r, y=y, o=o, M=M)
+    if want_log:
+        out["wlog"] = wlog
+    return out
+
+
+def undo(M, idx_w, wlog):
+    """Undoes a pass's in-place writes [m.163.com article on SDM, section 八, the
+    memory-efficiency paragraph]: replays the undo log backwards, from the last token to the
+    first, putting back each written row as its write found it.
+
+    M [B,H,N,d_v] the state after the pass; idx_w [B,T,H,W]; wlog [B,T,H,W,d_v].  Returns the
+    restored state (float64).
+    """
+    out = np.array(M, dtype=np.float64, copy=True)
+    B, T, H, W = idx_w.shape
+    for b in range(B):
+        for h in range(H):
+            for t in range(T - 1, -1, -1):
+                for j in range(W):
+                    out[b, h, idx_w[b, t, h, j]] = wlog[b, t, h, j]
+    return out

@@ -181,7 +181,8 @@ static int pass_impl(int T, int N, int d_v, int W, int R, const int32_t *idx_w,
                      const double *wt_w, const int32_t *idx_r, const double *wt_r,
                      const float *v, long v_stride, const float *alpha, const float *beta,
                      long ab_stride, int n_rows, const int32_t *rows, const float *M_in,
-                     const uint8_t *want_y, double *y, float *M_out, int coupled) {
+                     const uint8_t *want_y, double *y, float *M_out, int coupled,
+                     double *wlog) {
     if (T < 0 || N < 1 || d_v < 1 || W < 1 || R < 1 || n_rows < 0) return ORACLE_ERR_ARG;
     if (!idx_w || !wt_w || !idx_r || !wt_r || !v || !alpha || !beta || !M_in || !M_out)
         return ORACLE_ERR_ARG;
@@ -233,6 +234,8 @@ static int pass_impl(int T, int N, int d_v, int W, int R, const int32_t *idx_w,
                 const int32_t i = idx_w[(long)t * W + j];
                 const double kj = wt_w[(long)t * W + j];
                 double *row = S + (long)pos[i] * d_v;
+                if (wlog)
+                    for (int c = 0; c < d_v; ++c) wlog[((long)t * W + j) * d_v + c] = row[c];
                 for (int c = 0; c < d_v; ++c)
                     row[c] = a_t * row[c] + b_t * kj * ((double)v_t[c] - pred[c]);
             }
@@ -242,9 +245,16 @@ static int pass_impl(int T, int N, int d_v, int W, int R, const int32_t *idx_w,
             const int32_t i = idx_w[(long)t * W + j];
             if (i < 0 || i >= N) { rc = ORACLE_ERR_ARG; break; }
             const int p = pos[i];
-            if (p < 0) continue; /* untracked row: cannot influence tracked ones */
+            if (p < 0) { /* untracked row: cannot influence tracked ones */
+                if (wlog)
+                    for (int c = 0; c < d_v; ++c) wlog[((long)t * W + j) * d_v + c] = NAN;
+                continue;
+            }
             const double k_i = wt_w[(long)t * W + j];
             double *m = S + (long)p * d_v;
+            /* the undo log: the row as the write found it */
+            if (wlog)
+                for (int c = 0; c < d_v; ++c) wlog[((long)t * W + j) * d_v + c] = m[c];
             for (int c = 0; c < d_v; ++c) {
                 const double m_tilde = a_t * m[c];
                 m[c] = m_tilde + b_t * k_i * ((double)v_t[c] - m_tilde);
@@ -279,7 +289,25 @@ int sdm_oracle_pass(int T, int N, int d_v, int W, int R, const int32_t *idx_w,
                     long ab_stride, int n_rows, const int32_t *rows, const float *M_in,
                     const uint8_t *want_y, double *y, float *M_out) {
     return pass_impl(T, N, d_v, W, R, idx_w, wt_w, idx_r, wt_r, v, v_stride, alpha, beta,
-                     ab_stride, n_rows, rows, M_in, want_y, y, M_out, 0);
+                     ab_stride, n_rows, rows, M_in, want_y, y, M_out, 0, NULL);
+}
+
+/*
+ * sdm_oracle_pass that also keeps the undo log of the in-place update [m.163.com article on
+ * SDM, section 八, the memory-efficiency paragraph: training updates the state in place and
+ * undoes the updates during backpropagation]: wlog[(t * W + j) * d_v + c] is written slot j
+ * of token t as that token's write found it, before the write (NaN for an untracked row).
+ * Replaying the log backwards restores the state the pass started from.
+ */
+int sdm_oracle_pass_logged(int T, int N, int d_v, int W, int R, const int32_t *idx_w,
+                           const double *wt_w, const int32_t *idx_r, const double *wt_r,
+                           const float *v, long v_stride, const float *alpha,
+                           const float *beta, long ab_stride, int n_rows, const int32_t *rows,
+                           const float *M_in, const uint8_t *want_y, double *y, float *M_out,
+                           double *wlog) {
+    if (!wlog) return ORACLE_ERR_ARG;
+    return pass_impl(T, N, d_v, W, R, idx_w, wt_w, idx_r, wt_r, v, v_stride, alpha, beta,
+                     ab_stride, n_rows, rows, M_in, want_y, y, M_out, 0, wlog);
 }
 
 /*
@@ -296,7 +324,7 @@ int sdm_oracle_pass_coupled(int T, int N, int d_v, int W, int R, const int32_t *
                             const int32_t *rows, const float *M_in, const uint8_t *want_y,
                             double *y, float *M_out) {
     return pass_impl(T, N, d_v, W, R, idx_w, wt_w, idx_r, wt_r, v, v_stride, alpha, beta,
-                     ab_stride, n_rows, rows, M_in, want_y, y, M_out, 1);
+                     ab_stride, n_rows, rows, M_in, want_y, y, M_out, 1, NULL);
 }
 
 /*

@@ -17,6 +17,8 @@ import subprocess
 import sys
 from concurrent.futures import ThreadPoolExecutor
 
+import pytest
+
 import oracle
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -50,6 +52,9 @@ MUTANTS = {
     "coupled_prediction_undecayed": ("pred[c] += kj * (a_t * row[c]);", "pred[c] += kj * row[c];"),
     "coupled_prediction_unweighted": ("pred[c] += kj * (a_t * row[c]);",
                                       "pred[c] += a_t * row[c];"),
+    # the undo log of the in-place update: the row as the write found it
+    "undo_log_of_decayed_row": ("wlog[((long)t * W + j) * d_v + c] = m[c];",
+                                "wlog[((long)t * W + j) * d_v + c] = a_t * m[c];"),
     # step 3: the sparse read
     "read_weight_dropped": ("acc[c] += q_i * m[c];", "acc[c] += m[c];"),
     "read_uses_previous_tokens_slots": ("const int32_t i = idx_r[(long)t * R + j];",
@@ -99,3 +104,35 @@ def test_every_mutant_fails_a_pin_and_the_unmodified_copy_passes(tmp_path):
     # a detection is a failed pin (exit code 1), not a build error or a crash
     other = {n: r.returncode for n, r in results.items() if r.returncode != 1}
     assert not other, f"mutants that did not run to a failed pin: {other}"
+
+
+# Mistakes planted in the Python undo (a replay of the log): each must fail an undo pin.
+UNDO_MUTANTS = {
+    "replayed_forwards": ("for t in range(T - 1, -1, -1):", "for t in range(T):"),
+    "last_token_skipped": ("for t in range(T - 1, -1, -1):", "for t in range(T - 2, -1, -1):"),
+    "first_token_skipped": ("for t in range(T - 1, -1, -1):", "for t in range(T - 1, 0, -1):"),
+}
+
+
+@pytest.mark.parametrize("mutant", sorted(UNDO_MUTANTS))
+def test_every_undo_mutant_fails_a_pin(mutant, monkeypatch):
+    import inspect
+    import textwrap
+
+    import numpy as np
+
+    import tests.test_oracle_pins as pins
+    old, new = UNDO_MUTANTS[mutant]
+    src = textwrap.dedent(inspect.getsource(oracle.undo))
+    assert src.count(old) == 1
+    ns = {"np": np}
+    exec(src.replace(old, new), ns)  # noqa: S102 - a planted copy of the oracle's own code
+    monkeypatch.setattr(oracle, "undo", ns["undo"])
+    caught = 0
+    for pin in (pins.test_undo_restores_the_starting_state,
+                pins.test_undo_of_three_decays_of_one_slot):
+        try:
+            pin()
+        except AssertionError:
+            caught += 1
+    assert caught > 0, f"no undo pin detects {mutant}"

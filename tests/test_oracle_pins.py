@@ -63,6 +63,59 @@ def rand_unit(rng, T, S1, S2, d_v, dtype=np.float32):
     return kp, qp, v, alpha, beta, M0
 
 
+# ------------------------------------------------------- the undo log of the in-place update
+def test_undo_log_is_the_state_each_write_found():
+    """Log entry (t, j) is written slot j's row after tokens [0, t): the final state of the
+    pass cut at t, rounded to fp32 the same way, bit for bit; a log of the decayed row or of
+    the row after the write differs."""
+    rng = np.random.default_rng(31)
+    T, S1, S2, d_v, W = 20, 4, 3, 5, 3
+    kp, qp, v, alpha, beta, M0 = rand_unit(rng, T, S1, S2, d_v)
+    r = oracle.run_unit(kp, qp, v, alpha, beta, M0, 0, 0, S1=S1, W=W, R=2, want_log=True)
+    assert len(set(r["idx_w"].ravel().tolist())) < T * W  # slots written more than once
+    for t in (0, 1, 7, T - 1):
+        cut = oracle.run_unit(kp, qp, v, alpha, beta, M0, 0, 0, S1=S1, W=W, R=2, t_end=t)
+        rows = cut["M"][r["idx_w"][t]]
+        np.testing.assert_array_equal(r["wlog"][t].astype(np.float32), rows)
+
+
+def test_undo_restores_the_starting_state():
+    """Replaying the log backwards gives back the state the pass started from, exactly:
+    from M0 and from a continued state, with slots written many times over."""
+    rng = np.random.default_rng(32)
+    T, S1, S2, d_v = 40, 3, 3, 4
+    kp = rng.standard_normal((2, T, 2, S1 + S2)).astype(np.float32)
+    qp = rng.standard_normal((2, T, 2, S1 + S2)).astype(np.float32)
+    v = rng.standard_normal((2, T, 2, d_v)).astype(np.float32)
+    alpha = rng.uniform(0.05, 1.0, (2, T, 2)).astype(np.float32)
+    beta = rng.uniform(0.0, 1.0, (2, T, 2)).astype(np.float32)
+    M0 = rng.standard_normal((2, S1 * S2, d_v)).astype(np.float32)
+    M1 = rng.standard_normal((2, 2, S1 * S2, d_v)).astype(np.float32)
+    for M_init in (M0, M1):
+        r = oracle.forward(kp, qp, v, alpha, beta, M_init, S1=S1, W=3, R=2, want_log=True)
+        start = np.broadcast_to(M_init, r["M"].shape) if M_init.ndim == 3 else M_init
+        assert not np.array_equal(r["M"], start)
+        np.testing.assert_array_equal(oracle.undo(r["M"], r["idx_w"], r["wlog"]),
+                                      start.astype(np.float64))
+
+
+def test_undo_of_three_decays_of_one_slot():
+    """W = 1, beta = 0, alpha = 1/2: tokens 0-2 write slot 0 (8 -> 4 -> 2 -> 1), token 3
+    writes slot 3 (8 -> 4).  The log holds 8, 4, 2, 8 (the row each write found) and the
+    undo gives back 8 everywhere."""
+    kp = np.tile(np.array([5.0, 0.0, 5.0, 0.0], np.float32), (1, 4, 1, 1))
+    kp[0, 3, 0] = [0.0, 5.0, 0.0, 5.0]
+    v = np.ones((1, 4, 1, 1), np.float32)
+    alpha = np.full((1, 4, 1), 0.5, np.float32)
+    beta = np.zeros((1, 4, 1), np.float32)
+    M0 = np.full((1, 4, 1), 8.0, np.float32)
+    r = oracle.forward(kp, kp, v, alpha, beta, M0, S1=2, W=1, R=1, want_log=True)
+    assert r["idx_w"].ravel().tolist() == [0, 0, 0, 3]
+    assert r["wlog"].ravel().tolist() == [8.0, 4.0, 2.0, 8.0]
+    assert r["M"][0, 0, :, 0].tolist() == [1.0, 8.0, 8.0, 4.0]
+    assert oracle.undo(r["M"], r["idx_w"], r["wlog"])[0, 0, :, 0].tolist() == [8.0] * 4
+
+
 # ------------------------------------------------------------------ step 1: selection
 @pytest.mark.parametrize("S1,S2", [(3, 5), (4, 4), (8, 16), (16, 16), (7, 9), (1, 6)])
 def test_select_equals_brute_force_random(S1, S2):

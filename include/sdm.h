@@ -228,6 +228,46 @@ sdm_status sdm_norm_gate(const float *y, const void *gate, const float *gamma, f
                          int32_t act, sdm_shape shape, float *o, void *stream);
 
 /*
+ * Prefill that also keeps the undo log of its in-place writes [m.163.com article on SDM,
+ * section 八, the memory-efficiency paragraph: the state is updated in place and the
+ * updates are undone during backpropagation, so that one state and the overwritten rows,
+ * O(N d + T W d), are kept instead of a state per chunk].  Arguments, engines and results
+ * as sdm_scan_forward (the per-slot rule); in addition, for write j of token row
+ * r = (b * T + t) * H + h, wlog[(r * W + j) * d_v + c] receives the written row as that
+ * write found it, before the write.  wlog: fp32 [B,T,H,W,d_v], device, 16-byte aligned, not
+ * overlapping M or y; NULL is SDM_ERR_INVALID_ARG (T > 0).  Keep sel_out as well: the undo
+ * needs the write slots.  The log holds the engine's own row values: the slot engine's hot
+ * slots are stepped by composed affine maps, so an entry after a slot's first write in a
+ * chunk can differ from a token-by-token state by rounding; each slot's first logged entry
+ * in the pass is the starting row exactly.  To keep a smaller log, pack it afterwards
+ * (sdm_state_pack, B*T*H*W rows of d_v).
+ */
+sdm_status sdm_scan_forward_logged(const void *kp, const void *qp, const void *v,
+                                   const float *alpha, const float *beta, const float *M0,
+                                   float *M, int32_t init, float *y, const void *gate,
+                                   const float *gamma, float eps, int32_t act, float *o,
+                                   int32_t *sel_out, int32_t engine, void *ws, size_t ws_bytes,
+                                   sdm_shape shape, float *wlog, void *stream);
+
+/* Workspace bytes of sdm_state_undo for `shape` (B*H*N 32-bit entries); 0 for an invalid
+ * shape. */
+size_t sdm_undo_workspace_size(sdm_shape shape);
+
+/*
+ * Undoes a logged pass in place: M [B,H,N,d_v] (the state right after the pass) gets back,
+ * for every slot the pass wrote, the row that the slot's first write in the pass found, i.e.
+ * the state the pass started from; other rows are not touched.  sel_w: the pass's write
+ * slots [B,T,H,W] int32 (the first B*T*H*W entries of its sel_out); wlog: its undo log.
+ * ws: at least sdm_undo_workspace_size bytes, 256-byte aligned.  Device pointers, none
+ * overlapping another; invalid arguments return SDM_ERR_INVALID_ARG before any launch; an
+ * out-of-range slot sets SDM_ERR_DEVICE_CHECK (sdm_get_device_status) and is skipped.  A
+ * memset and two launches, asynchronous on `stream`.  With an fp32 log of the same pass, M
+ * is restored bit for bit.
+ */
+sdm_status sdm_state_undo(float *M, const int32_t *sel_w, const float *wlog, sdm_shape shape,
+                          void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Low-precision state rows (state checkpoints) [m.163.com article on SDM, section 八, the
  * memory-efficiency paragraph: the state checkpoints of 128k fine-tuning stored as fp8 or
  * int4, with no loss in training loss or final quality].  A checkpoint row holds one row of
@@ -273,7 +313,8 @@ typedef enum {
     SDM_KERNEL_DECODE = 5,     /* fused decode step                           */
     SDM_KERNEL_SLOT_SORT = 6,  /* slot engine: event build and radix sort      */
     SDM_KERNEL_STATE_ROWS = 7, /* state checkpoint pack / unpack              */
-    SDM_KERNEL_KINDS = 8
+    SDM_KERNEL_UNDO = 8,       /* undo of a logged pass                       */
+    SDM_KERNEL_KINDS = 16
 } sdm_kernel_kind;
 
 /* Kernel timing.  While enabled (on != 0), every kernel launch the library makes is

@@ -29,6 +29,7 @@ from ._binding import (  # noqa: F401
     sdm_profile_read,
     sdm_scan_forward,
     sdm_scan_forward_coupled,
+    sdm_scan_forward_logged,
     sdm_scan_forward_noalloc,
     sdm_select,
     sdm_set_option,
@@ -36,8 +37,10 @@ from ._binding import (  # noqa: F401
     sdm_state_init,
     sdm_state_pack,
     sdm_state_rows_bytes,
+    sdm_state_undo,
     sdm_state_unpack,
     sdm_status_string,
+    sdm_undo_workspace_size,
     sdm_workspace_size,
     shape_of,
 )

@@ -3,6 +3,7 @@
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 
 import torch
@@ -59,6 +60,10 @@ def library():
         "sdm_scan_forward_coupled": ([P, P, P, P, P, P, P, I, P, P, P, F, I, P, P, I, P, Z, S, P],
                                      I),
         "sdm_scan_forward_noalloc": ([P, P, P, P, P, P, P, I, P, P, P, F, I, P, P, S, P], I),
+        "sdm_scan_forward_logged": ([P, P, P, P, P, P, P, I, P, P, P, F, I, P, P, I, P, Z, S, P,
+                                     P], I),
+        "sdm_undo_workspace_size": ([S], Z),
+        "sdm_state_undo": ([P, P, P, S, P, Z, P], I),
         "sdm_norm_gate": ([P, P, P, F, I, S, P, P], I),
         "sdm_get_device_status": ([P], I),
         "sdm_status_string": ([I], ctypes.c_char_p),
@@ -249,6 +254,68 @@ def sdm_scan_forward_coupled(kp, qp, v, alpha, beta, M, **kw):
     return sdm_scan_forward(kp, qp, v, alpha, beta, M, coupled=True, **kw)
 
 
+def sdm_scan_forward_logged(kp, qp, v, alpha, beta, M, *, W: int, R: int, S1: int | None = None,
+                            M0=None, init: str = "m0", y=None, gate=None, gamma=None,
+                            eps: float = 1e-6, act: str = "silu", o=None, want_o: bool = True,
+                            sel_out=None, engine: str = "auto", ws=None, wlog=None,
+                            stream=None):
+    """sdm_scan_forward that also keeps the undo log of its in-place writes: returns
+    dict(y, o, sel, wlog) with wlog [B,T,H,W,d_v] fp32, written row j of token (b, t, h) as
+    its write found it; sel (the write slots, then the read slots) is always returned, since
+    sdm_state_undo needs it."""
+    dev = kp.device
+    shape, y, o, sel_out = _scan_outputs(kp, qp, v, alpha, beta, M, W, R, S1, M0, y, gate,
+                                         gamma, o, want_o, sel_out, True)
+    B, T, H = kp.shape[:3]
+    d_v = v.shape[-1]
+    _expect(wlog, "wlog", (B, T, H, W, d_v))
+    if wlog is None:
+        wlog = torch.empty((B, T, H, W, d_v), dtype=torch.float32, device=dev)
+    _need(wlog, "wlog", torch.float32, dev)
+    need = sdm_workspace_size(shape, engine)
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _need(ws, "ws", torch.uint8, dev)
+    _check(library().sdm_scan_forward_logged(
+        _p(kp), _p(qp), _p(v), _p(alpha), _p(beta), _p(M0), _p(M), INIT[init], _p(y), _p(gate),
+        _p(gamma), float(eps), ACT[act], _p(o), _p(sel_out), ENGINE[engine], _p(ws),
+        ws.numel(), shape, _p(wlog), _stream(stream, dev)), "sdm_scan_forward_logged")
+    return dict(y=y, o=o, sel=sel_out, wlog=wlog)
+
+
+def sdm_undo_workspace_size(shape: SdmShape) -> int:
+    return int(library().sdm_undo_workspace_size(shape))
+
+
+def sdm_state_undo(M, sel, wlog, *, W: int, S1: int | None = None, ws=None, stream=None):
+    """Undoes a logged pass in place: M [B,H,N,d_v] gets back, for every slot the pass wrote,
+    the row its first write found.  sel: the pass's sel output (its first B*T*H*W entries
+    are the write slots); wlog [B,T,H,W,d_v] its undo log."""
+    if M.dim() != 4 or wlog.dim() != 5:
+        raise ValueError("M must be [B, H, N, d_v] and wlog [B, T, H, W, d_v]")
+    B, H, N, d_v = M.shape
+    _, T, _, _, _ = wlog.shape
+    _expect(wlog, "wlog", (B, T, H, W, d_v))
+    if sel.numel() < B * T * H * W:
+        raise ValueError(f"sel has {sel.numel()} entries, fewer than the {B * T * H * W} "
+                         "write slots of the pass")
+    S1 = int(math.isqrt(N)) if S1 is None else int(S1)
+    if S1 < 1 or N % S1:
+        raise ValueError(f"S1 = {S1} does not divide N = {N}")
+    dev = M.device
+    _need(M, "M", torch.float32, dev)
+    _need(sel, "sel", torch.int32, dev)
+    _need(wlog, "wlog", torch.float32, dev)
+    shape = shape_of(B, T, H, S1, N // S1, W, W, d_v, SDM_F32)
+    need = sdm_undo_workspace_size(shape)
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _need(ws, "ws", torch.uint8, dev)
+    _check(library().sdm_state_undo(_p(M), _p(sel), _p(wlog), shape, _p(ws), ws.numel(),
+                                    _stream(stream, dev)), "sdm_state_undo")
+    return M
+
+
 def sdm_scan_forward_noalloc(kp, qp, v, alpha, beta, M, *, W: int, R: int,
                              S1: int | None = None, M0=None, init: str = "m0", y=None,
                              gate=None, gamma=None, eps: float = 1e-6, act: str = "silu",
@@ -410,7 +477,7 @@ def sdm_state_unpack(codes, scales, d_v: int, fmt: str = "e4m3", *, out=None, st
 
 
 KERNEL_KINDS = ("state_init", "select", "scan_seq", "scan_slot", "norm_gate", "decode",
-                "slot_sort", "state_rows")
+                "slot_sort", "state_rows", "undo")
 
 
 def sdm_profile_enable(on: bool = True):
@@ -420,8 +487,8 @@ def sdm_profile_enable(on: bool = True):
 
 def sdm_profile_read() -> dict:
     """{kind: (total ms, launches)} of the launches recorded since the last enable/read."""
-    ms = (ctypes.c_double * 8)()
-    n = (ctypes.c_int64 * 8)()
+    ms = (ctypes.c_double * 16)()
+    n = (ctypes.c_int64 * 16)()
     _check(library().sdm_profile_read(ctypes.cast(ms, ctypes.c_void_p),
                                       ctypes.cast(n, ctypes.c_void_p)), "sdm_profile_read")
     return {k: (ms[i], n[i]) for i, k in enumerate(KERNEL_KINDS)}

@@ -35,6 +35,8 @@ struct SeqArgs {
   float* y;            // [B*T*H, d_v]
   int B, T, H, N, W, R, ldw, ldr, d_v, v_bf16;
   int coupled;  // 1: the coupled delta rule (one prediction shared by the written rows)
+  float* wlog;  // [B*T*H, W, d_v] undo log of the per-slot rule (each written row as its
+                // write found it), or null
 };
 
 constexpr int SEQ_THREADS = 256;
@@ -292,6 +294,9 @@ __global__ void __launch_bounds__(SEQ_THREADS, 1) seq_scan_kernel(SeqArgs a) {
         if (find_writer(s, u - 1, u - D, tw, jw))
           old = reinterpret_cast<const float4*>(stage(tw) + (size_t)jw * CW)[lig];
       }
+      if (a.wlog)
+        __stcs(reinterpret_cast<float4*>(a.wlog + ((tok_row0 + (size_t)u * a.H) * a.W + j) *
+                                                      a.d_v + col0) + lig, old);
       const float kb = be * ww[j];
       const float ka = al * (1.0f - kb);
       float4 nw;

@@ -358,7 +358,23 @@ struct SlotArgs {
   int B, T, H, N, d_v, v_bf16;
   KeyBits kb;
   unsigned long long* cta_stats;  // [SDM_SLOT_STATS_CTAS][4] work per CTA, or null
+  float* wlog;  // [rows, W, d_v] undo log (each written row as its write found it), or null
+  int W;
 };
+
+// Stores the lane's part of a written row, as the write found it, to the undo log entry of
+// write j of token row r (streamed: the log is read back only by an undo).
+template <int NQ>
+__device__ __forceinline__ void log_old_row(const SlotArgs& a, uint32_t r, uint32_t j, int lane,
+                                            const float4 (&m)[NQ]) {
+  float4* lg = reinterpret_cast<float4*>(a.wlog + ((size_t)r * a.W + j) * a.d_v);
+  const int d4 = a.d_v / 4;
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const int c = lane + 32 * q;
+    if (c < d4) __stcs(lg + c, m[q]);
+  }
+}
 
 // Per-CTA work of the chunk kernel (load-balance analysis), added while enabled:
 // [0] events applied from short segments, [1] events of the long segments taken,
@@ -409,10 +425,11 @@ __device__ __forceinline__ bool walk_events(const SlotArgs& a, uint32_t first, u
   bool wrote = false;
   for (uint32_t e = first; e < last; e += 32) {
     const int cnt = static_cast<int>(min(32u, last - e));
-    uint32_t r32 = 0u;
+    uint32_t r32 = 0u, jl = 0u;
     float ca = 0.f, cb = 0.f;
     if (lane < cnt) {
       const uint2 pv = a.vals[e + lane];
+      jl = pv.x & 127u;
       const uint32_t t = pv.x >> 8;
       const uint32_t kind = (pv.x >> 7) & 1u;
       const uint32_t r = ((uint32_t)b * a.T + t) * a.H + (uint32_t)h;
@@ -441,6 +458,8 @@ __device__ __forceinline__ bool walk_events(const SlotArgs& a, uint32_t first, u
         const float Bc = __shfl_sync(FULL_MASK, cb, (i0 + i) & 31);
         if (i0 + i < cnt) {
           if ((rr[i] >> 31) == 0u) {
+            if (!compose && a.wlog)
+              log_old_row<NQ>(a, rr[i], __shfl_sync(FULL_MASK, jl, (i0 + i) & 31), lane, m);
 #pragma unroll
             for (int q = 0; q < NQ; ++q) {
               m[q].x = fmaf(A, m[q].x, Bc * vv[i][q].x);
@@ -661,9 +680,10 @@ __global__ void __launch_bounds__(SLOT_THREADS, (NQ <= 2 ? 4 : 1)) slot_chunk_ke
       kcarry = __shfl_sync(FULL_MASK, ck, cnt - 1);
       const bool head = lane < cnt && ck != kp;
       // this lane's event: state row coefficients and token row
-      uint32_t r32 = 0u;
+      uint32_t r32 = 0u, jl = 0u;
       float ca = 0.f, cb = 0.f;
       if (lane < cnt) {
+        jl = pv.x & 127u;
         const uint32_t t = pv.x >> 8;
         const uint32_t kind = (pv.x >> 7) & 1u;
         const uint32_t eh = (ck >> a.kb.nbits) & hmask;
@@ -711,6 +731,8 @@ __global__ void __launch_bounds__(SLOT_THREADS, (NQ <= 2 ? 4 : 1)) slot_chunk_ke
               dirty = false;
             }
             if ((rr[i] >> 31) == 0u) {
+              if (a.wlog)
+                log_old_row<NQ>(a, rr[i], __shfl_sync(FULL_MASK, jl, (i0 + i) & 31), lane, m);
 #pragma unroll
               for (int q = 0; q < NQ; ++q) {
                 m[q].x = fmaf(A, m[q].x, Bc * vv[i][q].x);

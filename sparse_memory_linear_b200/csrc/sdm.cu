@@ -15,6 +15,7 @@
 #include "decode.cuh"
 #include "norm_init.cuh"
 #include "rows.cuh"
+#include "undo.cuh"
 #include "scan_seq.cuh"
 #include "scan_slot.cuh"
 #include "select.cuh"
@@ -588,7 +589,7 @@ sdm_status launch_slot_chunk_work(const sdm_shape& s, const WsLayout& WL, unsign
 // radix passes, else in k1 / v1.
 sdm_status make_slot_args(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
                           const float* alpha, const float* beta, const void* v, float* M,
-                          float* y, SlotArgs* out) {
+                          float* y, float* wlog, SlotArgs* out) {
   const int passes = (WL.kb.total() + 7) / 8;
   SlotArgs& a = *out;
   a.keys = reinterpret_cast<uint32_t*>(w + (passes % 2 ? WL.off_k1 : WL.off_k0));
@@ -611,6 +612,8 @@ sdm_status make_slot_args(const sdm_shape& s, const WsLayout& WL, unsigned char*
   a.d_v = s.d_v;
   a.v_bf16 = s.in_dtype == SDM_BF16;
   a.kb = WL.kb;
+  a.wlog = wlog;
+  a.W = s.W;
   a.cta_stats = nullptr;
   if (opt(SDM_OPT_SLOT_CTA_STATS)) {
     void* p = nullptr;
@@ -625,9 +628,9 @@ sdm_status make_slot_args(const sdm_shape& s, const WsLayout& WL, unsigned char*
 // steps.
 sdm_status launch_slot(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
                        const float* alpha, const float* beta, const void* v, float* M, float* y,
-                       const DeviceInfo* di, cudaStream_t st) {
+                       float* wlog, const DeviceInfo* di, cudaStream_t st) {
   SlotArgs a;
-  sdm_status rc = make_slot_args(s, WL, w, alpha, beta, v, M, y, &a);
+  sdm_status rc = make_slot_args(s, WL, w, alpha, beta, v, M, y, wlog, &a);
   for (int t0 = 0; rc == SDM_OK && t0 < s.T; t0 += WL.chunk)
     rc = launch_slot_chunk_work(s, WL, w, a, t0, di, st);
   return rc;
@@ -699,9 +702,10 @@ sdm_status launch_select_chunk(const sdm_shape& s, const WsLayout& WL, const Sel
 sdm_status launch_slot_pipelined(const sdm_shape& s, const WsLayout& WL, unsigned char* w,
                                  const SelJob& jw, const SelJob& jr, int bf16,
                                  const float* alpha, const float* beta, const void* v,
-                                 float* M, float* y, const DeviceInfo* di, cudaStream_t st) {
+                                 float* M, float* y, float* wlog, const DeviceInfo* di,
+                                 cudaStream_t st) {
   SlotArgs a;
-  sdm_status rc = make_slot_args(s, WL, w, alpha, beta, v, M, y, &a);
+  sdm_status rc = make_slot_args(s, WL, w, alpha, beta, v, M, y, wlog, &a);
   if (rc != SDM_OK) return rc;
   std::lock_guard<std::mutex> lock(g_pipe_mu);
   PipeStreams* P;
@@ -900,7 +904,8 @@ static sdm_status scan_forward(const void* kp, const void* qp, const void* v, co
                                const float* beta, const float* M0, float* M, int32_t init,
                                float* y, const void* gate, const float* gamma, float eps,
                                int32_t act, float* o, int32_t* sel_out, int32_t engine, void* ws,
-                               size_t ws_bytes, sdm_shape shape, void* stream, bool coupled) {
+                               size_t ws_bytes, sdm_shape shape, void* stream, bool coupled,
+                               float* wlog = nullptr) {
   const sdm_shape& s = shape;
   if (!shape_ok(s, true)) return SDM_ERR_INVALID_ARG;
   if (init != SDM_INIT_FROM_M0 && init != SDM_CONTINUE) return SDM_ERR_INVALID_ARG;
@@ -921,6 +926,12 @@ static sdm_status scan_forward(const void* kp, const void* qp, const void* v, co
     for (const void* p : ptrs)
       if (p && !aligned16(p)) return SDM_ERR_INVALID_ARG;
     if (engine == SDM_ENGINE_SLOT && !slot_engine_fits(s)) return SDM_ERR_UNSUPPORTED;
+    if (wlog) {
+      const size_t nlog = (size_t)s.B * s.T * s.H * s.W * s.d_v * 4;
+      if (!aligned16(wlog) || overlaps(wlog, nlog, M, state_elems(s) * 4) ||
+          overlaps(wlog, nlog, y, (size_t)s.B * s.T * s.H * s.d_v * 4))
+        return SDM_ERR_INVALID_ARG;
+    }
     const size_t need = sdm_workspace_size(s, engine);
     if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN) != 0)
       return SDM_ERR_INVALID_ARG;
@@ -954,7 +965,7 @@ static sdm_status scan_forward(const void* kp, const void* qp, const void* v, co
   const bool pipelined = engine == SDM_ENGINE_SLOT && WL.n_chunks > 1 &&
                          (sched == 2 || (sched == 0 && PIPELINE_BY_DEFAULT));
   if (pipelined) {
-    rc = launch_slot_pipelined(s, WL, w, jw, jr, bf16, alpha, beta, v, M, y, di, st);
+    rc = launch_slot_pipelined(s, WL, w, jw, jr, bf16, alpha, beta, v, M, y, wlog, di, st);
     if (rc != SDM_OK) return rc;
   } else {
     ProfScope ps(SDM_KERNEL_SELECT, st);
@@ -971,7 +982,7 @@ static sdm_status scan_forward(const void* kp, const void* qp, const void* v, co
 
   if (engine == SDM_ENGINE_SLOT) {
     if (!pipelined) {
-      rc = launch_slot(s, WL, w, alpha, beta, v, M, y, di, st);
+      rc = launch_slot(s, WL, w, alpha, beta, v, M, y, wlog, di, st);
       if (rc != SDM_OK) return rc;
     }
     if (o) {
@@ -1002,6 +1013,7 @@ static sdm_status scan_forward(const void* kp, const void* qp, const void* v, co
   a.d_v = s.d_v;
   a.v_bf16 = bf16;
   a.coupled = coupled ? 1 : 0;
+  a.wlog = wlog;
   {
     ProfScope ps(SDM_KERNEL_SCAN_SEQ, st);
     rc = launch_seq(a, st);
@@ -1035,6 +1047,61 @@ sdm_status sdm_scan_forward_coupled(const void* kp, const void* qp, const void* 
   NvtxRange nvtx_range("sdm_scan_forward_coupled");
   return scan_forward(kp, qp, v, alpha, beta, M0, M, init, y, gate, gamma, eps, act, o,
                       sel_out, engine, ws, ws_bytes, shape, stream, true);
+}
+
+sdm_status sdm_scan_forward_logged(const void* kp, const void* qp, const void* v,
+                                   const float* alpha, const float* beta, const float* M0,
+                                   float* M, int32_t init, float* y, const void* gate,
+                                   const float* gamma, float eps, int32_t act, float* o,
+                                   int32_t* sel_out, int32_t engine, void* ws, size_t ws_bytes,
+                                   sdm_shape shape, float* wlog, void* stream) {
+  NvtxRange nvtx_range("sdm_scan_forward_logged");
+  if (!wlog && shape.T > 0) return SDM_ERR_INVALID_ARG;
+  return scan_forward(kp, qp, v, alpha, beta, M0, M, init, y, gate, gamma, eps, act, o,
+                      sel_out, engine, ws, ws_bytes, shape, stream, false, wlog);
+}
+
+size_t sdm_undo_workspace_size(sdm_shape shape) {
+  if (!shape_ok(shape, true)) return 0;
+  return round_up((size_t)shape.B * shape.H * shape.S1 * shape.S2 * 4, WS_ALIGN);
+}
+
+sdm_status sdm_state_undo(float* M, const int32_t* sel_w, const float* wlog, sdm_shape shape,
+                          void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("sdm_state_undo");
+  const sdm_shape& s = shape;
+  if (!shape_ok(s, true)) return SDM_ERR_INVALID_ARG;
+  if (s.T == 0) return SDM_OK;
+  if (!M || !sel_w || !wlog || !ws || !aligned16(M) || !aligned16(sel_w) || !aligned16(wlog) ||
+      (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN) != 0 || ws_bytes < sdm_undo_workspace_size(s))
+    return SDM_ERR_INVALID_ARG;
+  const long long rows = (long long)s.B * s.T * s.H;
+  const size_t nm = state_elems(s) * 4, nsel = (size_t)rows * s.W * 4,
+               nlog = (size_t)rows * s.W * s.d_v * 4, nws = sdm_undo_workspace_size(s);
+  if (overlaps(M, nm, wlog, nlog) || overlaps(M, nm, sel_w, nsel) || overlaps(M, nm, ws, nws) ||
+      overlaps(wlog, nlog, ws, nws) || overlaps(sel_w, nsel, ws, nws))
+    return SDM_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  sdm_status rc = device_info(&di);
+  if (rc != SDM_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int N = s.S1 * s.S2;
+  uint32_t* first = static_cast<uint32_t*>(ws);
+  ProfScope ps(SDM_KERNEL_UNDO, st);
+  SDM_CUDA_TRY(cudaMemsetAsync(first, 0xff, (size_t)s.B * s.H * N * 4, st));  // no write yet
+  const long long n_writes = rows * s.W;
+  long long blocks = (n_writes + 255) / 256;
+  if (blocks > (long long)di->sms * 16) blocks = (long long)di->sms * 16;
+  SDM_CUDA_TRY(launch_pdl(undo_first_kernel, dim3((unsigned)blocks), dim3(256), 0, st, sel_w,
+                          n_writes, s.T, s.H, s.W, N, first));
+  blocks = (rows + 7) / 8;  // a warp per token row
+  if (blocks > (long long)di->sms * 16) blocks = (long long)di->sms * 16;
+  SDM_CUDA_TRY(launch_pdl(undo_restore_kernel, dim3((unsigned)blocks), dim3(256), 0, st, M,
+                          sel_w, wlog, rows, s.T, s.H, s.W, N, s.d_v,
+                          static_cast<const uint32_t*>(first)));
+  g_launches.fetch_add(2, std::memory_order_relaxed);
+  SDM_CUDA_TRY(cudaGetLastError());
+  return SDM_OK;
 }
 
 // One decode step; `chained` launches it with programmatic stream serialisation.

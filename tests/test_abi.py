@@ -211,6 +211,41 @@ def test_state_pack_and_unpack_reject_bad_arguments(sdm):
 
 
 @host_only
+def test_logged_pass_and_undo_reject_bad_arguments(sdm):
+    """The logged prefill needs its log (16-byte aligned, apart from M and y); the undo needs
+    M, the write slots, the log and a large enough aligned workspace, none overlapping."""
+    lib = sdm.library()
+    P = ctypes.c_void_p
+    s = good_shape(sdm)  # B2 T16 H3 S32x32 W8 R8 d_v64
+    GB = 1 << 30
+    M, y, wlog, ws = FAKE, FAKE + GB, FAKE + 2 * GB, FAKE + 4 * GB
+    need = sdm.sdm_workspace_size(s, "auto")
+    with no_launch(sdm):
+        def logged(wl, ys=y):
+            return lib.sdm_scan_forward_logged(
+                P(FAKE + 8 * GB), P(FAKE + 9 * GB), P(FAKE + 10 * GB), P(FAKE + 11 * GB),
+                P(FAKE + 12 * GB), None, P(M), 1, P(ys), None, None, 1e-6, 0, None, None, 0,
+                P(ws), need, s, wl, None)
+        assert logged(None) == 1                      # no log
+        assert logged(P(wlog + 4)) == 1               # misaligned log
+        assert logged(P(M + 4096)) == 1               # log over M
+        assert logged(P(y)) == 1                      # log over y
+        need_u = lib.sdm_undo_workspace_size(s)
+        assert need_u == 2 * 3 * 1024 * 4
+        sel = FAKE + 6 * GB
+        undo = lib.sdm_state_undo
+        assert undo(None, P(sel), P(wlog), s, P(ws), need_u, None) == 1
+        assert undo(P(M), None, P(wlog), s, P(ws), need_u, None) == 1
+        assert undo(P(M), P(sel), None, s, P(ws), need_u, None) == 1
+        assert undo(P(M), P(sel), P(wlog), s, P(ws), need_u - 1, None) == 1   # small ws
+        assert undo(P(M), P(sel), P(wlog), s, P(ws + 16), need_u, None) == 1  # ws alignment
+        assert undo(P(M), P(sel), P(M + 256), s, P(ws), need_u, None) == 1    # log over M
+        assert undo(P(M), P(sel), P(wlog), s, P(wlog + 64), need_u, None) == 1  # ws over log
+        t0 = sdm.shape_of(2, 0, 3, 32, 32, 8, 8, 64, sdm.SDM_BF16)
+        assert undo(None, None, None, t0, None, 0, None) == 0                 # T = 0: nothing
+
+
+@host_only
 def test_noalloc_rejects_shapes_beyond_its_scratch(sdm):
     """4 x 8192 x 8 rows with W = R = 64 need 128 MiB of scratch, beyond the fixed 16 MiB
     of sdm_scan_forward_noalloc: SDM_ERR_INVALID_ARG before any CUDA call or launch."""

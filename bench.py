@@ -497,6 +497,70 @@ def bench_state_rows(args, dist: Dist, dev):
     return out
 
 
+def bench_undo(args, dist: Dist, dev):
+    """The logged prefill (sdm_scan_forward_logged: the step plus its undo log, W rows of
+    d_v fp32 per token-head) and the undo (sdm_state_undo) on the prefill workload, each
+    timed with CUDA events (median of 3 after 3 warm-ups); the undo restores the state after
+    every logged step, so each logged step starts from the same state."""
+    import sparse_memory_linear_b200 as sdm
+
+    stream = torch.cuda.current_stream(dev)
+    peak, peak_kind = hbm_peak()
+    wl = sdm_synth.WORKLOADS[args.workload]
+    g = {k: v.to(dev) for k, v in sdm_synth.make_inputs(wl, device=dev).items()}
+    M = torch.empty((wl.B, wl.H, wl.N, wl.d_v), dtype=torch.float32, device=dev)
+    sdm.sdm_state_init(g["M0"], M)
+    shape = sdm.shape_of(wl.B, wl.T, wl.H, wl.S1, wl.S2, wl.W, wl.R, wl.d_v,
+                         sdm.SDM_BF16 if wl.in_dtype == torch.bfloat16 else sdm.SDM_F32)
+    ws = torch.empty(sdm.sdm_workspace_size(shape), dtype=torch.uint8, device=dev)
+    ws_u = torch.empty(sdm.sdm_undo_workspace_size(shape), dtype=torch.uint8, device=dev)
+    y = torch.empty((wl.B, wl.T, wl.H, wl.d_v), dtype=torch.float32, device=dev)
+    o = torch.empty_like(y)
+    sel = torch.empty(wl.B * wl.T * wl.H * (wl.W + wl.R), dtype=torch.int32, device=dev)
+    wlog = torch.empty((wl.B, wl.T, wl.H, wl.W, wl.d_v), dtype=torch.float32, device=dev)
+    M_start = M.clone()
+
+    def logged():
+        sdm.sdm_scan_forward_logged(g["kp"], g["qp"], g["v"], g["alpha"], g["beta"], M,
+                                    W=wl.W, R=wl.R, S1=wl.S1, init="continue", gate=g["gate"],
+                                    y=y, o=o, sel_out=sel, ws=ws, wlog=wlog, stream=stream)
+
+    def undo():
+        sdm.sdm_state_undo(M, sel, wlog, W=wl.W, S1=wl.S1, ws=ws_u, stream=stream)
+
+    t_log, t_undo = [], []
+    for i in range(6):
+        a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record(stream)
+        logged()
+        b.record(stream)
+        undo()
+        c.record(stream)
+        torch.cuda.synchronize(dev)
+        if i >= 3:
+            t_log.append(a.elapsed_time(b))
+            t_undo.append(b.elapsed_time(c))
+    restored = bool(torch.equal(M, M_start))
+    if sdm.sdm_get_device_status() != 0:
+        raise RuntimeError("device status word set during the undo benchmark")
+    th = wl.B * wl.T * wl.H
+    log_bytes = wlog.numel() * 4
+    ms = float(np.median(t_log))
+    step_bytes = th * algorithmic_bytes(wl) + log_bytes
+    out = {"workload": wl.name, "logged_ms_per_step": ms,
+           "logged_value": th / (ms * 1e-3), "unit": UNIT,
+           "log_bytes_per_step": log_bytes,
+           "logged_whole_step_hbm": {"bytes_per_token_head": step_bytes / th,
+                                     "GBps": step_bytes / (ms * 1e-3) / 1e9,
+                                     "frac": step_bytes / (ms * 1e-3) / 1e9 / peak},
+           "undo_ms": float(np.median(t_undo)),
+           "undo_restored_state_bit_for_bit": restored,
+           "peak_kind": peak_kind}
+    del g, wlog, ws, ws_u, M, M_start, y, o, sel
+    torch.cuda.empty_cache()
+    return out
+
+
 def bench_coupled(args, dist: Dist, dev):
     """The coupled delta rule: prefill of the 1.4B-like workload (sequential engine, the one
     that computes it) and 256 chained decode steps of the batched-decode workload, timed as
@@ -739,7 +803,8 @@ def main(argv=None):
     ap.add_argument("--select-schedule", choices=["default", "serial", "pipelined"],
                     default="default",
                     help="the slot engine's selection schedule (SDM_OPT_SELECT_SCHEDULE)")
-    ap.add_argument("--only", choices=["prefill", "decode", "balance", "rows"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "balance", "rows", "undo"],
+                    default=None,
                     help="run one part (profiling of a small case)")
     ap.add_argument("--override", default="",
                     help="workload fields to change, e.g. B=1,T=4096 (prefill workload)")
@@ -778,6 +843,11 @@ def main(argv=None):
             out = bench_balance(args, dev)
             if dist.rank == 0:
                 print(json.dumps({"balance": out}), flush=True)
+            return 0
+        if args.only == "undo":
+            out = bench_undo(args, dist, dev)
+            if dist.rank == 0:
+                print(json.dumps({"undo": out}), flush=True)
             return 0
         if args.only == "rows":
             out = bench_state_rows(args, dist, dev)
@@ -829,6 +899,7 @@ def main(argv=None):
         if not args.no_configs and args.only is None:
             line["coupled"] = bench_coupled(args, dist, dev)
             line["state_rows"] = bench_state_rows(args, dist, dev)
+            line["undo"] = bench_undo(args, dist, dev)
         if dist.rank == 0:
             print(json.dumps(line), flush=True)
         return 0

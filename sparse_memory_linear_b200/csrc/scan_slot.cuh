@@ -416,7 +416,7 @@ __device__ __forceinline__ void load_v(const void* v, size_t off, bool bf16, int
 // the row, m.  compose == false: writes update m, reads add q * m into y.  compose == true:
 // m starts at 0 and accumulates the affine map's additive part, A_acc its multiplicative
 // part; reads are skipped.  Returns whether any write was applied.
-template <int NQ, int G>
+template <int NQ, int G, bool LOG>
 __device__ __forceinline__ bool walk_events(const SlotArgs& a, uint32_t first, uint32_t last, int b,
                                             int h, int lane, float4 (&m)[NQ], bool compose,
                                             float& A_acc) {
@@ -458,7 +458,7 @@ __device__ __forceinline__ bool walk_events(const SlotArgs& a, uint32_t first, u
         const float Bc = __shfl_sync(FULL_MASK, cb, (i0 + i) & 31);
         if (i0 + i < cnt) {
           if ((rr[i] >> 31) == 0u) {
-            if (!compose && a.wlog)
+            if (LOG && !compose)
               log_old_row<NQ>(a, rr[i], __shfl_sync(FULL_MASK, jl, (i0 + i) & 31), lane, m);
 #pragma unroll
             for (int q = 0; q < NQ; ++q) {
@@ -494,7 +494,9 @@ __host__ __device__ constexpr inline size_t slot_warp_smem(int NQ, int PF) {
 // comment); then every warp takes spans of SLOT_SPAN sorted events from a queue and handles
 // each shorter segment that starts in its span, streaming the segments' state rows through
 // a ring of PF shared-memory rows with cp.async.
-template <int NQ, int G, int PF>
+// LOG: also store each written row, as its write finds it, to the undo log a.wlog (a
+// separate instantiation, so that the plain pass keeps its registers).
+template <int NQ, int G, int PF, bool LOG>
 __global__ void __launch_bounds__(SLOT_THREADS, (NQ <= 2 ? 4 : 1)) slot_chunk_kernel(SlotArgs a, int chunk) {
   // wait for the kernel ahead in the stream (programmatic launch), then let the next one in
   grid_dependency_wait();
@@ -537,7 +539,7 @@ __global__ void __launch_bounds__(SLOT_THREADS, (NQ <= 2 ? 4 : 1)) slot_chunk_ke
 #pragma unroll
       for (int q = 0; q < NQ; ++q) m[q] = make_float4(0.f, 0.f, 0.f, 0.f);
       float A = 1.0f;
-      walk_events<NQ, G>(a, s0, s1, b, h, lane, m, true, A);
+      walk_events<NQ, G, LOG>(a, s0, s1, b, h, lane, m, true, A);
       if (lane == 0) coefA[warp] = A;
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
@@ -568,7 +570,7 @@ __global__ void __launch_bounds__(SLOT_THREADS, (NQ <= 2 ? 4 : 1)) slot_chunk_ke
       __syncthreads();  // every warp has read the row before the last one rewrites it
       // 3. re-walk the slice from its exact start state: the reads, and the final row
       float unused = 1.0f;
-      walk_events<NQ, G>(a, s0, s1, b, h, lane, m, false, unused);
+      walk_events<NQ, G, LOG>(a, s0, s1, b, h, lane, m, false, unused);
       if (warp == SLOT_WARPS - 1) {
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
@@ -731,7 +733,7 @@ __global__ void __launch_bounds__(SLOT_THREADS, (NQ <= 2 ? 4 : 1)) slot_chunk_ke
               dirty = false;
             }
             if ((rr[i] >> 31) == 0u) {
-              if (a.wlog)
+              if (LOG)
                 log_old_row<NQ>(a, rr[i], __shfl_sync(FULL_MASK, jl, (i0 + i) & 31), lane, m);
 #pragma unroll
               for (int q = 0; q < NQ; ++q) {

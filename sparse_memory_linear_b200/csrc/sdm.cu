@@ -136,7 +136,8 @@ sdm_status device_info(DeviceInfo** out) {
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)RS_SCATTER_SMEM));
 #define SDM_SLOT_ATTR(NQ, G, PF) \
-  SDM_CUDA_TRY(allow_max_dynamic_smem(slot_chunk_kernel<NQ, G, PF>, m));
+  SDM_CUDA_TRY(allow_max_dynamic_smem(slot_chunk_kernel<NQ, G, PF, false>, m)); \
+  SDM_CUDA_TRY(allow_max_dynamic_smem(slot_chunk_kernel<NQ, G, PF, true>, m));
     SDM_SLOT_ATTR(1, 4, 6) SDM_SLOT_ATTR(2, 2, 6) SDM_SLOT_ATTR(4, 4, 4) SDM_SLOT_ATTR(8, 2, 2)
 #undef SDM_SLOT_ATTR
     d.attrs_set = true;
@@ -475,21 +476,27 @@ sdm_status launch_state_init(const float* M0, float* M, const sdm_shape& s, cuda
   return SDM_OK;
 }
 
-template <int NQ, int G, int PF>
-sdm_status launch_slot_chunk(const SlotArgs& a, const DeviceInfo* di, cudaStream_t st) {
+template <int NQ, int G, int PF, bool LOG>
+sdm_status launch_slot_chunk_t(const SlotArgs& a, const DeviceInfo* di, cudaStream_t st) {
   const size_t smem = SLOT_WARPS * slot_warp_smem(NQ, PF);
   int per_sm = 0;
   SDM_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-      &per_sm, slot_chunk_kernel<NQ, G, PF>, SLOT_THREADS, smem));
+      &per_sm, slot_chunk_kernel<NQ, G, PF, LOG>, SLOT_THREADS, smem));
   int ctas = per_sm > 0 ? per_sm : 1;
   const int cap = opt(SDM_OPT_SLOT_CTAS_PER_SM);
   if (cap > 0 && cap < ctas) ctas = cap;
   const int grid = di->sms * ctas;
-  SDM_CUDA_TRY(launch_pdl(slot_chunk_kernel<NQ, G, PF>, dim3(grid), dim3(SLOT_THREADS), smem, st,
-                          a, 0));
+  SDM_CUDA_TRY(launch_pdl(slot_chunk_kernel<NQ, G, PF, LOG>, dim3(grid), dim3(SLOT_THREADS), smem,
+                          st, a, 0));
   g_launches.fetch_add(1, std::memory_order_relaxed);
   SDM_CUDA_TRY(cudaGetLastError());
   return SDM_OK;
+}
+
+template <int NQ, int G, int PF>
+sdm_status launch_slot_chunk(const SlotArgs& a, const DeviceInfo* di, cudaStream_t st) {
+  return a.wlog ? launch_slot_chunk_t<NQ, G, PF, true>(a, di, st)
+                : launch_slot_chunk_t<NQ, G, PF, false>(a, di, st);
 }
 
 // One time chunk [t0, t0 + ct) of the slot engine on `st`: the chunk's events, their radix

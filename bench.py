@@ -337,7 +337,7 @@ PREFILL_CONFIGS = ("small", "layer1p4b")
 
 
 def bench_prefill_configs(args, dist: Dist, dev):
-    """The other prefill workloads: the AUTO engine's step and both engines' steps, each
+    """The other prefill workloads: the AUTO engine's step and every engine's step, each
     timed alone with CUDA events (median of the timed steps) after a write of twice the L2
     size (the small workload's inputs and state fit in L2).  One step is one
     sdm_scan_forward with SDM_CONTINUE, as in the headline."""
@@ -356,7 +356,7 @@ def bench_prefill_configs(args, dist: Dist, dev):
         y = torch.empty((wl.B, wl.T, wl.H, wl.d_v), dtype=torch.float32, device=dev)
         o = torch.empty_like(y)
         ms = {}
-        for engine in ("auto", "seq", "slot"):
+        for engine in ("auto", "seq", "slot", "chunk"):
             def step():
                 sdm.sdm_scan_forward(g["kp"], g["qp"], g["v"], g["alpha"], g["beta"], M,
                                      W=wl.W, R=wl.R, S1=wl.S1, init="continue", gate=g["gate"],
@@ -389,7 +389,7 @@ def bench_prefill_configs(args, dist: Dist, dev):
             "workload": wl.name, "shape": wl.note, "metric": METRIC, "unit": UNIT,
             "value": weak_scaling_value(th, step_s, dist.world), "ms_per_step": ms["auto"],
             "engine": "slot" if prof["scan_slot"][1] else "seq",
-            "engine_ms_per_step": {"seq": ms["seq"], "slot": ms["slot"]},
+            "engine_ms_per_step": {"seq": ms["seq"], "slot": ms["slot"], "chunk": ms["chunk"]},
             "whole_step_hbm": {"bytes_per_token_head": algorithmic_bytes(wl),
                                "GBps": th * algorithmic_bytes(wl) / step_s / 1e9,
                                "frac": th * algorithmic_bytes(wl) / step_s / 1e9 / peak,

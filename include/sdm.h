@@ -54,7 +54,12 @@ typedef enum {
 } sdm_status;
 
 typedef enum { SDM_F32 = 0, SDM_BF16 = 1 } sdm_dtype;
-typedef enum { SDM_ENGINE_AUTO = 0, SDM_ENGINE_SEQ = 1, SDM_ENGINE_SLOT = 2 } sdm_engine;
+typedef enum {
+    SDM_ENGINE_AUTO = 0,
+    SDM_ENGINE_SEQ = 1,
+    SDM_ENGINE_SLOT = 2,
+    SDM_ENGINE_CHUNK = 3
+} sdm_engine;
 typedef enum { SDM_INIT_FROM_M0 = 0, SDM_CONTINUE = 1 } sdm_init;
 typedef enum { SDM_GATE_SILU = 0, SDM_GATE_SIGMOID = 1, SDM_GATE_IDENTITY = 2 } sdm_gate_act;
 
@@ -114,6 +119,17 @@ sdm_status sdm_state_init(const float *M0, float *M, sdm_shape shape, void *stre
  *            read slots [B,T,H,R], in selection order (for parity checks).
  *   engine   sdm_engine; ws / ws_bytes caller scratch of at least
  *            sdm_workspace_size(shape, engine) bytes, 256-byte aligned.
+ *            SDM_ENGINE_SEQ walks the tokens of each (b, h) in order; SDM_ENGINE_SLOT
+ *            sorts the writes and reads by slot and runs every slot's recurrence;
+ *            SDM_ENGINE_CHUNK is the chunk-wise form [m.163.com article, section 八, the
+ *            training-implementation paragraph]: chunks of up to 32 tokens, inside a chunk
+ *            the reads as y_t = sum_i q_t(i) e^{L(t,i)} M0[i] + sum_{s<=t} A[t,s] v_s, with
+ *            L(t,i) the summed ln(alpha (1 - beta k)) of slot i's writes in the chunk up to
+ *            t and A[t,s] the sparse inner product of token t's read list and token s's
+ *            write list (a two-pointer merge of the lists in slot order); the state is
+ *            carried from chunk to chunk.  It expects alpha (1 - beta k) >= 0 (alpha >= 0,
+ *            beta k <= 1, as with alpha = exp(-softplus), beta a sigmoid) and agrees with the
+ *            other engines to fp32 rounding of the exponentials.  AUTO picks SEQ or SLOT.
  * T == 0 is valid: only the initialisation (if requested) happens.
  */
 sdm_status sdm_scan_forward(const void *kp, const void *qp, const void *v, const float *alpha,
@@ -314,6 +330,7 @@ typedef enum {
     SDM_KERNEL_SLOT_SORT = 6,  /* slot engine: event build and radix sort      */
     SDM_KERNEL_STATE_ROWS = 7, /* state checkpoint pack / unpack              */
     SDM_KERNEL_UNDO = 8,       /* undo of a logged pass                       */
+    SDM_KERNEL_SCAN_CHUNK = 9, /* steps 2-3, chunk-wise engine                */
     SDM_KERNEL_KINDS = 16
 } sdm_kernel_kind;
 

@@ -9,7 +9,7 @@ import os
 import torch
 
 SDM_F32, SDM_BF16 = 0, 1
-ENGINE = {"auto": 0, "seq": 1, "slot": 2}
+ENGINE = {"auto": 0, "seq": 1, "slot": 2, "chunk": 3}
 INIT = {"m0": 0, "continue": 1}
 ACT = {"silu": 0, "sigmoid": 1, "identity": 2}
 _STATUS = {0: "SDM_OK", 1: "SDM_ERR_INVALID_ARG", 2: "SDM_ERR_UNSUPPORTED", 3: "SDM_ERR_CUDA",
@@ -477,7 +477,7 @@ def sdm_state_unpack(codes, scales, d_v: int, fmt: str = "e4m3", *, out=None, st
 
 
 KERNEL_KINDS = ("state_init", "select", "scan_seq", "scan_slot", "norm_gate", "decode",
-                "slot_sort", "state_rows", "undo")
+                "slot_sort", "state_rows", "undo", "scan_chunk")
 
 
 def sdm_profile_enable(on: bool = True):

@@ -16,6 +16,7 @@
 #include "norm_init.cuh"
 #include "rows.cuh"
 #include "undo.cuh"
+#include "scan_chunk.cuh"
 #include "scan_seq.cuh"
 #include "scan_slot.cuh"
 #include "select.cuh"
@@ -132,6 +133,7 @@ sdm_status device_info(DeviceInfo** out) {
     SDM_SEQ_ATTR(4, 4) SDM_SEQ_ATTR(4, 8) SDM_SEQ_ATTR(8, 4) SDM_SEQ_ATTR(8, 8)
     SDM_SEQ_ATTR(16, 4) SDM_SEQ_ATTR(16, 8) SDM_SEQ_ATTR(32, 4) SDM_SEQ_ATTR(32, 8)
 #undef SDM_SEQ_ATTR
+    SDM_CUDA_TRY(allow_max_dynamic_smem(chunk_scan_kernel, m));
     SDM_CUDA_TRY(cudaFuncSetAttribute(radix_scatter_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)RS_SCATTER_SMEM));
@@ -403,6 +405,32 @@ sdm_status launch_seq_t(const SeqArgs& a, int grid, size_t smem, cudaStream_t st
 }
 
 // Column-slice width CW and prefetch distance D of the sequential engine: one CTA per
+// The chunk-wise engine: 32 tokens per chunk (16 or 8 when the shared memory of wide index
+// lists needs it), column slices of up to 128 values (the largest multiple of 4 that
+// divides d_v), a CTA per (sequence, head, slice).
+sdm_status launch_chunk(ChunkArgs a, const DeviceInfo* di, cudaStream_t st) {
+  a.CW = 4;
+  for (int cw = a.d_v < 128 ? a.d_v : 128; cw >= 4; cw -= 4)
+    if (cw % 4 == 0 && a.d_v % cw == 0) {
+      a.CW = cw;
+      break;
+    }
+  size_t smem = 0;
+  for (a.C = 32; a.C >= 8; a.C /= 2) {
+    a.hash_size = 1;
+    while (a.hash_size < 2 * a.C * a.W) a.hash_size *= 2;
+    smem = chunk_layout(a.C, a.W, a.R, a.CW, a.hash_size).total;
+    if (smem <= (size_t)di->max_smem_optin) break;
+  }
+  if (a.C < 8) return SDM_ERR_UNSUPPORTED;
+  const long long grid = (long long)a.B * a.H * (a.d_v / a.CW);
+  SDM_CUDA_TRY(launch_pdl(chunk_scan_kernel, dim3((unsigned)grid), dim3(CHUNK_THREADS), smem, st,
+                          a));
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  SDM_CUDA_TRY(cudaGetLastError());
+  return SDM_OK;
+}
+
 // (sequence, head, slice) and all CTAs resident at once; wider slices while there are
 // enough CTAs to cover the SMs, then narrower ones.
 sdm_status launch_seq(const SeqArgs& a, cudaStream_t st) {
@@ -763,8 +791,9 @@ const char* sdm_status_string(sdm_status status) {
 
 size_t sdm_workspace_size(sdm_shape shape, int32_t engine) {
   if (!shape_ok(shape, true)) return 0;
-  if (engine < SDM_ENGINE_AUTO || engine > SDM_ENGINE_SLOT) return 0;
+  if (engine < SDM_ENGINE_AUTO || engine > SDM_ENGINE_CHUNK) return 0;
   if (engine == SDM_ENGINE_SLOT && !slot_engine_fits(shape)) return 0;
+  if (engine == SDM_ENGINE_CHUNK) engine = SDM_ENGINE_SEQ;  // the selection's lists only
   // AUTO may pick either engine: size for the larger
   if (engine == SDM_ENGINE_AUTO && slot_engine_fits(shape)) engine = SDM_ENGINE_SLOT;
   return ws_layout(shape, engine).total;
@@ -916,10 +945,12 @@ static sdm_status scan_forward(const void* kp, const void* qp, const void* v, co
   const sdm_shape& s = shape;
   if (!shape_ok(s, true)) return SDM_ERR_INVALID_ARG;
   if (init != SDM_INIT_FROM_M0 && init != SDM_CONTINUE) return SDM_ERR_INVALID_ARG;
-  if (engine < SDM_ENGINE_AUTO || engine > SDM_ENGINE_SLOT) return SDM_ERR_INVALID_ARG;
+  if (engine < SDM_ENGINE_AUTO || engine > SDM_ENGINE_CHUNK) return SDM_ERR_INVALID_ARG;
   // the slot engine treats every slot as its own recurrence, which the shared prediction of
   // the coupled rule breaks
   if (coupled && engine == SDM_ENGINE_SLOT) return SDM_ERR_UNSUPPORTED;
+  // the chunk-wise engine computes the per-slot rule and keeps no undo log
+  if ((coupled || wlog) && engine == SDM_ENGINE_CHUNK) return SDM_ERR_UNSUPPORTED;
   if (!act_ok(act) || !(eps >= 0.0f)) return SDM_ERR_INVALID_ARG;
   if (!M || !aligned16(M)) return SDM_ERR_INVALID_ARG;
   if (init == SDM_INIT_FROM_M0) {
@@ -1021,7 +1052,30 @@ static sdm_status scan_forward(const void* kp, const void* qp, const void* v, co
   a.v_bf16 = bf16;
   a.coupled = coupled ? 1 : 0;
   a.wlog = wlog;
-  {
+  if (engine == SDM_ENGINE_CHUNK) {
+    ChunkArgs c;
+    c.idx_w = idx_w;
+    c.wt_w = wt_w;
+    c.idx_r = idx_r;
+    c.wt_r = wt_r;
+    c.alpha = alpha;
+    c.beta = beta;
+    c.v = v;
+    c.M = M;
+    c.y = y;
+    c.B = s.B;
+    c.T = s.T;
+    c.H = s.H;
+    c.N = s.S1 * s.S2;
+    c.W = s.W;
+    c.R = s.R;
+    c.ldw = WL.ldw;
+    c.ldr = WL.ldr;
+    c.d_v = s.d_v;
+    c.v_bf16 = bf16;
+    ProfScope ps(SDM_KERNEL_SCAN_CHUNK, st);
+    rc = launch_chunk(c, di, st);
+  } else {
     ProfScope ps(SDM_KERNEL_SCAN_SEQ, st);
     rc = launch_seq(a, st);
   }

@@ -457,6 +457,7 @@ def bench_state_rows(args, dist: Dist, dev):
     codes plus the per-row scales, each once."""
     import sparse_memory_linear_b200 as sdm
 
+    torch.cuda.empty_cache()  # the parts before may leave tens of GB cached
     stream = torch.cuda.current_stream(dev)
     peak, peak_kind = hbm_peak()
     wl = sdm_synth.WORKLOADS[args.workload]
@@ -504,6 +505,7 @@ def bench_undo(args, dist: Dist, dev):
     every logged step, so each logged step starts from the same state."""
     import sparse_memory_linear_b200 as sdm
 
+    torch.cuda.empty_cache()  # the parts before may leave tens of GB cached
     stream = torch.cuda.current_stream(dev)
     peak, peak_kind = hbm_peak()
     wl = sdm_synth.WORKLOADS[args.workload]

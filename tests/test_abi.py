@@ -92,6 +92,9 @@ def test_workspace_size(sdm):
     assert sdm.sdm_workspace_size(s) == slot
     assert sdm.sdm_workspace_size(good_shape(sdm, W=40)) == 0  # W > S
     assert sdm.sdm_workspace_size(good_shape(sdm, d_v=12)) == 0  # bf16 needs d_v % 8 == 0
+    # the chunk-wise engine keeps only the selections, as the sequential one
+    assert sdm.sdm_workspace_size(s, "chunk") == want
+    assert sdm.library().sdm_workspace_size(s, 4) == 0  # no such engine
 
 
 FAKE = 0x10000  # aligned, never dereferenced: validation rejects the call first
@@ -300,6 +303,25 @@ def test_coupled_prefill_refuses_the_slot_engine_before_any_launch(sdm):
                                           None, 1e-6, 0, None, None, 2, P(FAKE), 1 << 40,
                                           good_shape(sdm), None)
     assert rc == 2  # SDM_ERR_UNSUPPORTED
+
+
+@host_only
+def test_chunk_engine_refuses_the_coupled_rule_and_the_undo_log(sdm):
+    """The chunk-wise engine computes the per-slot rule and keeps no log: the coupled and the
+    logged prefill refuse it (SDM_ERR_UNSUPPORTED) before any launch; an unknown engine is an
+    invalid argument."""
+    lib = sdm.library()
+    P = ctypes.c_void_p
+    s = good_shape(sdm)
+    GB = 1 << 30
+    need = sdm.sdm_workspace_size(s, "chunk")
+    args = (P(FAKE), P(FAKE + GB), P(FAKE + 2 * GB), P(FAKE + 3 * GB), P(FAKE + 4 * GB), None,
+            P(FAKE + 5 * GB), 1, P(FAKE + 6 * GB), None, None, 1e-6, 0, None, None)
+    with no_launch(sdm):
+        assert lib.sdm_scan_forward_coupled(*args, 3, P(FAKE + 8 * GB), need, s, None) == 2
+        assert lib.sdm_scan_forward_logged(*args, 3, P(FAKE + 8 * GB), need, s,
+                                           P(FAKE + 16 * GB), None) == 2
+        assert lib.sdm_scan_forward(*args, 4, P(FAKE + 8 * GB), need, s, None) == 1
 
 
 def test_status_strings(sdm):

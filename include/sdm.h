@@ -148,8 +148,9 @@ sdm_status sdm_scan_forward(const void *kp, const void *qp, const void *v, const
  *   M[i] = alpha_t * M[i] + beta_t * k_i * (v_t - p_t)      for i in I_w
  * (with I_w all N slots: M_t = alpha_t (I - beta_t k k^T) M_{t-1} + beta_t k v_t^T).  The
  * read and step 4 are those of sdm_scan_forward, and so are the arguments.  The sequential
- * engine computes it (SDM_ENGINE_AUTO takes it); the slot engine, which treats every slot as
- * its own recurrence, cannot: SDM_ENGINE_SLOT returns SDM_ERR_UNSUPPORTED.
+ * engine computes it (SDM_ENGINE_AUTO takes it); the slot and chunk-wise engines, which treat
+ * every slot as its own recurrence, cannot: SDM_ENGINE_SLOT and SDM_ENGINE_CHUNK return
+ * SDM_ERR_UNSUPPORTED.
  */
 sdm_status sdm_scan_forward_coupled(const void *kp, const void *qp, const void *v,
                                     const float *alpha, const float *beta, const float *M0,
@@ -252,7 +253,8 @@ sdm_status sdm_norm_gate(const float *y, const void *gate, const float *gamma, f
  * r = (b * T + t) * H + h, wlog[(r * W + j) * d_v + c] receives the written row as that
  * write found it, before the write.  wlog: fp32 [B,T,H,W,d_v], device, 16-byte aligned, not
  * overlapping M or y; NULL is SDM_ERR_INVALID_ARG (T > 0).  Keep sel_out as well: the undo
- * needs the write slots.  The log holds the engine's own row values: the slot engine's hot
+ * needs the write slots.  The sequential and slot engines keep the log; SDM_ENGINE_CHUNK
+ * returns SDM_ERR_UNSUPPORTED.  The log holds the engine's own row values: the slot engine's hot
  * slots are stepped by composed affine maps, so an entry after a slot's first write in a
  * chunk can differ from a token-by-token state by rounding; each slot's first logged entry
  * in the pass is the starting row exactly.  To keep a smaller log, pack it afterwards

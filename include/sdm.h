@@ -372,7 +372,10 @@ typedef enum {
                                        work on an internal high-priority one, joined
                                        back to the caller's stream), 0 the library's
                                        default; every schedule gives the same
-                                       selections and state                             */
+                                       selections and state.  The internal streams are
+                                       per device and shared by the process: pipelined
+                                       calls from several host threads are enqueued one
+                                       at a time and run one after another.             */
 } sdm_option;
 
 /* Sets an option.  SDM_ERR_INVALID_ARG (and no change) for an unknown option or a value
